@@ -1,0 +1,338 @@
+"""Throughput of on-device decoding of entropy-coded weights (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
+
+A step decodes the whole Int8 8192x8192 Laplace weight (H = 2.0 bits, 64 KiB chunks, 128
+interleaved streams, run 8) from its rANS stream in HBM into bf16 in HBM: one eq_decode launch.
+Every rank decodes its own copy (weak scaling; the decode has no exchange step).  Timing: CUDA
+events on the launching stream around each step, the L2 flushed between steps by writing a
+256 MiB buffer, max over ranks.  `e2e` repeats the step through the C ABI with host buffers:
+pinned host -> device copy of the coded arrays, decode, device -> host copy of the bf16 weight.
+Secondary lines under "also": the fused decode-GEMV on the 13B MLP (batch 1/4/16) and the DFloat11
+decode, each with its own roofline.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "int8_8k"
+METRIC = "decoded params/s (rANS decode to bf16)"
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def prepare_rans(eq, wl_name: str):
+    """Quantise + encode the workload with the library's own host compressor (no oracle)."""
+    wl = synth.WORKLOADS[wl_name]
+    spec = wl.tensors[0]
+    w = spec.generate()
+    fmt = eq.EQ_SYM_E4M3 if wl.symfmt == "e4m3" else eq.EQ_SYM_INT8
+    sym, sc = eq.codec.quantize(w, fmt, wl.int8_div)
+    del w
+    h = eq.codec.rans_encode(sym, sc, fmt, wl.chunk_symbols, wl.streams, wl.run)
+    return wl, h
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e-3)
+    return times
+
+
+def run_ours(args):
+    import torch
+
+    import decoding_interleaved_rans_b200 as eq
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+    wl, h = prepare_rans(eq, WORKLOAD)
+    t = eq.DeviceRans.upload(h, dev)
+    out = torch.empty(h.rows, h.cols, dtype=torch.bfloat16, device=dev)
+    status = eq.new_status(dev)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    def step():
+        eq.decode([t], [out], status, stream)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        times = time_steps(step, args.steps, args.warmup, flush, stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    assert int(status.item()) == 0, "decode reported corrupt data"
+    mean_s = statistics.mean(times)
+    mean_s = max_over_ranks(world, mean_s)
+    numel = h.rows * h.cols
+    alg_bytes = t.compressed_bytes + 2 * numel
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    pin = {k: torch.from_numpy(np.ascontiguousarray(v).view(dt)).pin_memory()
+           for k, v, dt in [("states", h.states, np.int32), ("word_off", h.word_off, np.int64),
+                            ("words", h.words, np.int16), ("scales", h.scales, np.int16)]}
+    out_host = torch.empty(h.rows, h.cols, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = out_host.numel() * 2
+
+    def e2e_step():
+        t.states.copy_(pin["states"], non_blocking=True)
+        t.word_off.copy_(pin["word_off"], non_blocking=True)
+        t.words.copy_(pin["words"], non_blocking=True)
+        t.scales.copy_(pin["scales"], non_blocking=True)
+        eq.decode([t], [out], status, stream)
+        out_host.copy_(out, non_blocking=True)
+
+    e2e_times = time_steps(e2e_step, max(3, args.steps // 4), 2, flush, stream)
+    e2e_s = max_over_ranks(world, statistics.mean(e2e_times))
+    assert int(status.item()) == 0
+
+    also = []
+    if not args.no_extra:
+        also = extra_measurements(eq, dev, stream, flush, peaks, args)
+    barrier(world)
+    if rank != 0:
+        return
+    achieved = alg_bytes / mean_s / 1e9
+    line = {
+        "metric": METRIC, "value": numel * world / mean_s, "unit": "params/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
+        "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
+                               "chunks, 128 streams, run 8 -> bf16",
+                   "params_per_gpu": numel, "compressed_bytes": t.compressed_bytes,
+                   "bits_per_param": 8 * t.compressed_bytes / numel,
+                   "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{world}"},
+        "gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_src": peaks["src"], "kernel": "rans_decode_kernel<4,8,INT8>",
+                     "alg_bytes_per_launch": alg_bytes},
+        "e2e": {"value": numel * world / e2e_s, "unit": "params/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "also": also,
+    }
+    if not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(h, numel)
+    print(json.dumps(line), flush=True)
+
+
+def extra_measurements(eq, dev, stream, flush, peaks, args):
+    """Fused decode-GEMV and DFloat11 decode, when the library provides them."""
+    out = []
+    return out
+
+
+def cpu_baseline(h, numel, seconds_budget: float = 20.0):
+    """The oracle's decoder (plain C, chunk-parallel over the host cores) on the same container."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    o = oracle.RansTensor(h.rows, h.cols, h.symfmt, h.prob_bits, h.chunk_symbols, h.streams,
+                          h.run, h.freqs, h.states, h.word_off, h.words, h.scales)
+    n_chunks = o.num_chunks
+    # time a small probe, then size the sample to stay within the budget
+    probe = list(range(min(n_chunks, cores)))
+    t0 = time.perf_counter()
+    oracle.rans_decode_bf16(o, chunks=probe, threads=cores)
+    per_chunk = (time.perf_counter() - t0) / max(1, len(probe)) * cores
+    take = max(1, min(n_chunks, int(seconds_budget / max(per_chunk / cores, 1e-9))))
+    chunks = list(range(take))
+    t0 = time.perf_counter()
+    rc, _ = oracle.rans_decode_bf16(o, chunks=chunks, threads=cores)
+    dt = time.perf_counter() - t0
+    assert rc == 0
+    syms = sum(min(h.chunk_symbols, numel - c * h.chunk_symbols) for c in chunks)
+    return {"value": syms / dt, "unit": "params/s", "cores": cores, "kind": "oracle",
+            "sample": f"{take} of {n_chunks} chunks ({syms} params), decode + dequant to bf16, "
+                      f"{cores} threads", "seconds": dt}
+
+
+def run_reference(args):
+    """The oracle timed on the host cores, same workload/metric; rank 0 only."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    wl = synth.WORKLOADS[WORKLOAD]
+    sym, sc = oracle.quantize(wl.tensors[0].generate(), oracle.INT8, wl.int8_div)
+    o = oracle.rans_encode(sym, sc, oracle.INT8, wl.chunk_symbols, wl.streams, wl.run)
+    h = o
+    cores = len(os.sched_getaffinity(0))
+    take = min(o.num_chunks, max(cores * 4, 64))
+    chunks = list(range(take))
+    for _ in range(args.warmup):
+        oracle.rans_decode_bf16(o, chunks=chunks[:cores], threads=cores)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        rc, _ = oracle.rans_decode_bf16(o, chunks=chunks, threads=cores)
+        times.append(time.perf_counter() - t0)
+        assert rc == 0
+    dt = statistics.mean(times)
+    syms = take * h.chunk_symbols
+    v = syms / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "params/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
+            "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
+                                   "chunks, 128 streams, run 8 -> bf16",
+                       "sample_chunks": take, "parallelism": "host cores"},
+            "cpu_baseline": {"value": v, "unit": "params/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{take} of {o.num_chunks} chunks per step"},
+            "e2e": {"value": v, "unit": "params/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the GEMV / DFloat11 lines")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+"""Python face of the C ABI: device-resident coded tensors and the four decode calls.
+
+PyTorch supplies device memory and the current stream; the library's kernels do all the work.
+Every wrapper passes raw pointers and the stream handle to libeq.so and checks the returned
+status; nothing here computes a decoded value.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+
+def _stream(stream) -> C.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: torch.Tensor | None) -> C.c_void_p:
+    return C.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dev(a: np.ndarray, device, as_dtype) -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    return torch.from_numpy(a.view(as_dtype)).to(device, non_blocking=False)
+
+
+def table_bytes(kind: int) -> int:
+    return int(L.lib().eq_table_bytes(kind))
+
+
+def build_tables(kind: int, host_in, prob_bits: int, d_tables: torch.Tensor, stream=None) -> None:
+    """eq_build_tables: frequencies (rANS) or code lengths (Huffman) -> device tables."""
+    arr = (C.c_uint32 * 256)(*[int(v) for v in np.asarray(host_in).ravel()[:256]])
+    L.check(L.lib().eq_build_tables(kind, arr, prob_bits, _ptr(d_tables), _stream(stream)),
+            "eq_build_tables")
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+@dataclass
+class DeviceRans:
+    """An interleaved-rANS-coded weight resident in device memory (eq_rans_tensor)."""
+    rows: int
+    cols: int
+    symfmt: int
+    prob_bits: int
+    chunk_symbols: int
+    streams: int
+    run: int
+    num_chunks: int
+    states: torch.Tensor
+    word_off: torch.Tensor
+    words: torch.Tensor
+    scales: torch.Tensor
+    tables: torch.Tensor
+
+    @property
+    def numel(self) -> int:
+        return self.rows * self.cols
+
+    @property
+    def compressed_bytes(self) -> int:
+        """Bytes the decoder reads from memory: words in use, states, offsets, scales, table."""
+        used_words = int(self.word_off[-1].item()) if self.num_chunks else 0
+        return (2 * used_words + 4 * self.states.numel() + 8 * self.word_off.numel()
+                + 2 * self.scales.numel() + 256 * 2)
+
+    def desc(self) -> L.RansTensorDesc:
+        chunk = self.chunk_symbols if self.chunk_symbols else self.cols
+        return L.RansTensorDesc(L.EQ_ABI_VERSION, self.symfmt, self.rows, self.cols,
+                                self.prob_bits, chunk, self.streams, self.run, self.num_chunks,
+                                self.states.data_ptr(), self.word_off.data_ptr(),
+                                self.words.data_ptr(), self.scales.data_ptr(),
+                                self.tables.data_ptr())
+
+    @classmethod
+    def upload(cls, h, device="cuda", stream=None) -> "DeviceRans":
+        """Copy a host container (fields rows, cols, symfmt, prob_bits, chunk_symbols, streams,
+        run, freqs, states, word_off, words, scales) to the device and build its table."""
+        words = np.ascontiguousarray(h.words, dtype=np.uint16)
+        if words.size % 8:
+            words = np.concatenate([words, np.zeros(8 - words.size % 8, np.uint16)])
+        if words.size == 0:
+            words = np.zeros(8, np.uint16)
+        t = cls(int(h.rows), int(h.cols), int(h.symfmt), int(h.prob_bits), int(h.chunk_symbols),
+                int(h.streams), int(h.run), int(len(h.word_off) - 1),
+                _dev(np.asarray(h.states, np.uint32), device, np.int32),
+                _dev(np.asarray(h.word_off, np.uint64), device, np.int64),
+                _dev(words, device, np.int16),
+                _dev(np.asarray(h.scales, np.uint16), device, np.int16),
+                torch.empty(table_bytes(L.EQ_TABLE_RANS), dtype=torch.uint8, device=device))
+        build_tables(L.EQ_TABLE_RANS, h.freqs, t.prob_bits, t.tables, stream)
+        return t
+
+
+@dataclass
+class DeviceHuff:
+    """A DFloat11-coded bf16 weight resident in device memory (eq_huff_tensor)."""
+    n: int
+    total_bits: int
+    bytes_per_thread: int
+    threads_per_block: int
+    enc_exp: torch.Tensor
+    sign_mant: torch.Tensor
+    gaps: torch.Tensor
+    block_out: torch.Tensor
+    tables: torch.Tensor
+
+    @property
+    def threads(self) -> int:
+        return (self.total_bits + 63) // 64
+
+    @property
+    def compressed_bytes(self) -> int:
+        return (8 * self.threads + self.n + (5 * self.threads + 7) // 8
+                + 8 * self.block_out.numel() + 256)
+
+    def desc(self) -> L.HuffTensorDesc:
+        return L.HuffTensorDesc(self.n, self.total_bits, self.bytes_per_thread,
+                                self.threads_per_block, self.enc_exp.data_ptr(),
+                                self.sign_mant.data_ptr(), self.gaps.data_ptr(),
+                                self.block_out.data_ptr(), self.tables.data_ptr())
+
+    @classmethod
+    def upload(cls, h, device="cuda", stream=None) -> "DeviceHuff":
+        """Copy a host container (fields n, total_bits, threads_per_block, lengths, enc_exp,
+        sign_mant, gaps, block_out) to the device and build its tables."""
+        sm = np.asarray(h.sign_mant, np.uint8)
+        if sm.size == 0:
+            sm = np.zeros(16, np.uint8)
+        t = cls(int(h.n), int(h.total_bits), 8, int(h.threads_per_block),
+                _dev(np.asarray(h.enc_exp, np.uint8), device, np.uint8),
+                _dev(sm, device, np.uint8),
+                _dev(np.asarray(h.gaps, np.uint8), device, np.uint8),
+                _dev(np.asarray(h.block_out, np.uint64), device, np.int64),
+                torch.empty(table_bytes(L.EQ_TABLE_HUFF), dtype=torch.uint8, device=device))
+        build_tables(L.EQ_TABLE_HUFF, h.lengths, 0, t.tables, stream)
+        return t
+
+
+def decode(tensors, outs=None, status=None, stream=None):
+    """eq_decode over a list of DeviceRans.  Returns (list of bf16 outputs, status tensor)."""
+    tensors = list(tensors)
+    dev = tensors[0].words.device
+    if outs is None:
+        outs = [torch.empty(t.rows, t.cols, dtype=torch.bfloat16, device=dev) for t in tensors]
+    if status is None:
+        status = new_status(dev)
+    descs = (L.RansTensorDesc * len(tensors))(*[t.desc() for t in tensors])
+    ptrs = (C.c_void_p * len(tensors))(*[o.data_ptr() for o in outs])
+    L.check(L.lib().eq_decode(descs, len(tensors), ptrs, _ptr(status), _stream(stream)),
+            "eq_decode")
+    return outs, status
+
+
+def decode_gemv(t: DeviceRans, x: torch.Tensor, y=None, status=None, stream=None):
+    """eq_decode_gemv: y[b] = W x[b] with W decoded on chip.  x bf16 [batch, cols]."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape[-1] == t.cols
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty(batch, t.rows, dtype=torch.float32, device=x.device)
+    if status is None:
+        status = new_status(x.device)
+    d = t.desc()
+    L.check(L.lib().eq_decode_gemv(C.byref(d), _ptr(x), batch, _ptr(y), _ptr(status),
+                                   _stream(stream)), "eq_decode_gemv")
+    return y, status
+
+
+def huff_bf16_decode(h: DeviceHuff, out=None, status=None, stream=None):
+    """eq_huff_bf16_decode: DFloat11 -> bf16 [n]."""
+    dev = h.enc_exp.device
+    if out is None:
+        out = torch.empty(max(h.n, 1), dtype=torch.bfloat16, device=dev)[:h.n]
+    if status is None:
+        status = new_status(dev)
+    d = h.desc()
+    L.check(L.lib().eq_huff_bf16_decode(C.byref(d), _ptr(out), _ptr(status), _stream(stream)),
+            "eq_huff_bf16_decode")
+    return out, status
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    """Raw uint16 patterns of a bf16 tensor (device or host)."""
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)

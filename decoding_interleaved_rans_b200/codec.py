@@ -1,0 +1,130 @@
+"""Host-side compressor (include/eq_encode.h): numpy in, host containers out.
+
+The pages compress once, offline; this is that step, run by libeq.so on CPU threads.  The
+containers hold exactly the arrays DeviceRans.upload / DeviceHuff.upload expect.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import _lib as L
+
+
+def _p(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+@dataclass
+class HostRans:
+    rows: int
+    cols: int
+    symfmt: int
+    prob_bits: int
+    chunk_symbols: int
+    streams: int
+    run: int
+    freqs: np.ndarray
+    states: np.ndarray
+    word_off: np.ndarray
+    words: np.ndarray
+    scales: np.ndarray
+
+    @property
+    def numel(self) -> int:
+        return self.rows * self.cols
+
+
+@dataclass
+class HostHuff:
+    n: int
+    total_bits: int
+    threads_per_block: int
+    lengths: np.ndarray
+    enc_exp: np.ndarray
+    sign_mant: np.ndarray
+    gaps: np.ndarray
+    block_out: np.ndarray
+
+
+def quantize(w: np.ndarray, symfmt: int, int8_div: float = 0.0, threads: int = 0):
+    """Per-row AbsMax quantisation -> (symbols uint8 [rows, cols], bf16 scales uint16 [rows])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    sym = np.empty((rows, cols), np.uint8)
+    sc = np.empty(rows, np.uint16)
+    L.check(L.lib().eq_quantize_host(_p(w), rows, cols, symfmt, float(int8_div), _p(sym), _p(sc),
+                                     threads), "eq_quantize_host")
+    return sym, sc
+
+
+def rans_freqs(sym: np.ndarray, prob_bits: int = 12) -> np.ndarray:
+    sym = np.ascontiguousarray(sym, dtype=np.uint8).ravel()
+    f = np.zeros(256, np.uint32)
+    L.check(L.lib().eq_rans_freqs_host(_p(sym) if sym.size else None, sym.size, prob_bits, _p(f)),
+            "eq_rans_freqs_host")
+    return f
+
+
+def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols: int,
+                streams: int, run: int, freqs=None, threads: int = 0) -> HostRans:
+    sym = np.ascontiguousarray(sym, dtype=np.uint8)
+    rows, cols = sym.shape
+    if freqs is None:
+        freqs = rans_freqs(sym)
+    freqs = np.ascontiguousarray(freqs, dtype=np.uint32)
+    chunk = chunk_symbols if chunk_symbols else cols
+    nchunks = (rows * cols + chunk - 1) // chunk
+    states = np.empty(max(1, nchunks * streams), np.uint32)
+    word_off = np.zeros(nchunks + 1, np.uint64)
+    wp, nw = C.c_void_p(), C.c_uint64()
+    L.check(L.lib().eq_rans_encode_host(_p(sym) if sym.size else None, rows, cols, _p(freqs),
+                                        chunk_symbols, streams, run, threads, _p(states),
+                                        _p(word_off), C.byref(wp), C.byref(nw)),
+            "eq_rans_encode_host")
+    try:
+        words = np.ctypeslib.as_array(C.cast(wp, C.POINTER(C.c_uint16)), (nw.value,)).copy()
+    finally:
+        L.lib().eq_free_host(wp)
+    return HostRans(rows, cols, symfmt, 12, chunk_symbols, streams, run, freqs,
+                    states[:nchunks * streams], word_off, words,
+                    np.ascontiguousarray(scales, np.uint16))
+
+
+def huff_lengths(counts: np.ndarray, max_len: int = 32) -> np.ndarray:
+    counts = np.ascontiguousarray(counts, dtype=np.uint64)
+    lens = np.zeros(256, np.uint32)
+    L.check(L.lib().eq_huff_lengths_host(_p(counts), max_len, _p(lens)), "eq_huff_lengths_host")
+    return lens
+
+
+def exponent_counts(w_bf16: np.ndarray) -> np.ndarray:
+    e = (np.asarray(w_bf16, dtype=np.uint16).ravel() >> 7) & 0xFF
+    return np.bincount(e, minlength=256).astype(np.uint64)
+
+
+def huff_encode(w_bf16: np.ndarray, threads_per_block: int = 256, lengths=None,
+                max_len: int = 32) -> HostHuff:
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16).ravel()
+    n = w.size
+    if lengths is None:
+        lengths = huff_lengths(exponent_counts(w), max_len)
+    lengths = np.ascontiguousarray(lengths, dtype=np.uint32)
+    tb = C.c_uint64()
+    wp = _p(w) if n else None
+    L.check(L.lib().eq_huff_plan_host(wp, n, _p(lengths), C.byref(tb)), "eq_huff_plan_host")
+    total_bits = tb.value
+    threads = (total_bits + 63) // 64
+    blocks = (threads + threads_per_block - 1) // threads_per_block
+    enc = np.zeros(threads * 8 + 16, np.uint8)
+    sm = np.zeros(max(1, n), np.uint8)
+    gaps = np.zeros((5 * threads + 7) // 8 + 8, np.uint8)
+    block_out = np.zeros(blocks + 1, np.uint64)
+    L.check(L.lib().eq_huff_encode_host(wp, n, _p(lengths), threads_per_block, total_bits,
+                                        _p(enc), _p(sm), _p(gaps), _p(block_out)),
+            "eq_huff_encode_host")
+    return HostHuff(n, total_bits, threads_per_block, lengths.astype(np.uint8), enc, sm[:n],
+                    gaps, block_out)

@@ -1,0 +1,146 @@
+// Internal helpers shared by the library's CUDA sources (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "eq.h"
+
+namespace eq {
+
+// ------------------------------------------------------------------------------------------------
+// device decode-table layouts written by eq_build_tables
+// ------------------------------------------------------------------------------------------------
+
+// rANS: 16-byte header, then one 32-bit entry per slot of the 4096-slot probability space:
+//   bits 31..24 symbol, bits 23..12 frequency (1..4095), bits 11..0 slot - cum[symbol].
+// A table whose single symbol owns all 4096 slots cannot store its frequency in 12 bits; the
+// header flags it instead and the decoders take a separate path.
+constexpr uint32_t kRansProbBits = 12;
+constexpr uint32_t kRansSlots = 1u << kRansProbBits;
+constexpr uint32_t kRansL = 1u << 16;
+struct RansTableHeader {
+  uint32_t magic;        // kRansMagic
+  uint32_t flags;        // kRansFlag*
+  uint32_t single_sym;   // symbol of a one-symbol table
+  uint32_t reserved;
+};
+constexpr uint32_t kRansMagic = 0x52414E53u;  // "RANS"
+constexpr uint32_t kRansFlagNaN7F = 1u;       // frequency of byte 0x7F is nonzero
+constexpr uint32_t kRansFlagNaNFF = 2u;       // frequency of byte 0xFF is nonzero
+constexpr uint32_t kRansFlagSingle = 4u;      // one symbol owns every slot
+constexpr size_t kRansTableBytes = sizeof(RansTableHeader) + kRansSlots * 4;
+
+// Huffman (DFloat11 exponent): 16-byte header, then up to kHuffMaxTables tables of 256 uint16
+// entries.  Table 0 is indexed by the next 8 code bits; an entry is either
+//   a leaf   (bit 15 clear): bits 7..0 exponent value, bits 11..8 bits used at this level (1..8)
+//   a pointer (bit 15 set):  bits 7..0 index of the child table, which reads the next 8 bits
+//   0xFFFF: no code starts with this bit pattern.
+constexpr uint32_t kHuffMaxTables = 32;
+struct HuffTableHeader {
+  uint32_t magic;        // kHuffMagic
+  uint32_t num_tables;
+  uint32_t max_len;
+  uint32_t reserved;
+};
+constexpr uint32_t kHuffMagic = 0x48554646u;  // "HUFF"
+constexpr uint16_t kHuffInvalid = 0xFFFFu;
+constexpr size_t kHuffTableBytes = sizeof(HuffTableHeader) + kHuffMaxTables * 256 * 2;
+
+// ------------------------------------------------------------------------------------------------
+// host helpers
+// ------------------------------------------------------------------------------------------------
+
+inline eq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EQ_OK : EQ_ERR_CUDA; }
+
+inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int device_sm_count();  // SMs of the current device (cached per device)
+
+// floor(n / d) for n < 2^40 and 1 <= d < 2^32 as __umul64hi(n, m) with m = ceil(2^64 / d).
+inline uint64_t div_magic(uint64_t d) { return d <= 1 ? 0 : (~0ull) / d + 1; }
+
+// ------------------------------------------------------------------------------------------------
+// device helpers
+// ------------------------------------------------------------------------------------------------
+
+#ifdef __CUDACC__
+
+__device__ __forceinline__ uint64_t div_by_magic(uint64_t n, uint64_t magic) {
+  return magic ? __umul64hi(n, magic) : n;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// mbarrier + 1-D bulk copy (TMA engine, global -> this CTA's shared memory, no multicast)
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after ~1 s (or 2^26 polls).  Returns false on
+// timeout; the caller records EQ_DEV_TIMEOUT and stops using the buffer.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0; i < (1u << 26); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && global_timer_ns() - t0 > 1000000000ull) break;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void report(uint32_t *d_status, uint32_t bits) {
+  if (bits) atomicOr(d_status, bits);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+#endif  // __CUDACC__
+
+}  // namespace eq

@@ -1,0 +1,182 @@
+// eq_build_tables / eq_table_bytes and the small ABI utilities.
+//
+// The rANS slot table follows the decoding rule of the interleaved rANS format in eq.h
+// ("Float8@2bits" summary, "Codificacion de Pesos": ANS over the flattened symbol stream).
+// The Huffman tables follow the DFloat11 page, "Decodificacion basada en LUT jerarquicas": the
+// canonical code tree is cut into height-8 subtrees, each a 256-entry lookup table; entries that
+// lead deeper point at the child table.  The page reuses the never-seen exponents 240..255 as the
+// pointers inside 8-bit entries; here entries are 16 bits wide (a pointer bit, the bits used at
+// this level and the value), so every exponent value, including 240..255, stays decodable.
+#include <algorithm>
+#include <vector>
+
+#include "eq_internal.cuh"
+
+namespace eq {
+
+struct RansBuildArgs {
+  uint32_t *dst;           // device table (header + 4096 entries)
+  uint32_t flags, single;  // header fields
+  uint16_t freq[256];
+};
+
+// one block of 256 threads: prefix sum of the frequencies, then every slot finds its symbol
+__global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__ RansBuildArgs a) {
+  __shared__ uint32_t cum[257];
+  const uint32_t t = threadIdx.x;
+  if (t == 0) {
+    uint32_t c = 0;
+    for (int s = 0; s < 256; ++s) {
+      cum[s] = c;
+      c += a.freq[s];
+    }
+    cum[256] = c;
+    RansTableHeader h{kRansMagic, a.flags, a.single, 0u};
+    *reinterpret_cast<RansTableHeader *>(a.dst) = h;
+  }
+  __syncthreads();
+  uint32_t *lut = a.dst + sizeof(RansTableHeader) / 4;
+  for (uint32_t slot = t; slot < kRansSlots; slot += blockDim.x) {
+    // largest s with cum[s] <= slot: that symbol owns the slot
+    int lo = 0, hi = 255;
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (cum[mid] <= slot) lo = mid; else hi = mid - 1;
+    }
+    uint32_t f = a.freq[lo];
+    uint32_t fe = (f >= kRansSlots) ? 0u : f;  // a one-symbol table is handled by the flag
+    lut[slot] = (uint32_t(lo) << 24) | (fe << 12) | (slot - cum[lo]);
+  }
+}
+
+struct HuffBuildArgs {
+  uint32_t *dst;
+  HuffTableHeader h;
+  uint16_t t[kHuffMaxTables][256];
+};
+
+__global__ void __launch_bounds__(256) huff_build_kernel(const __grid_constant__ HuffBuildArgs a) {
+  if (threadIdx.x == 0) *reinterpret_cast<HuffTableHeader *>(a.dst) = a.h;
+  uint16_t *out = reinterpret_cast<uint16_t *>(a.dst + sizeof(HuffTableHeader) / 4);
+  const uint16_t *src = &a.t[0][0];
+  for (uint32_t i = threadIdx.x; i < a.h.num_tables * 256; i += blockDim.x) out[i] = src[i];
+}
+
+// Hierarchical tables of a canonical code given by its lengths.  Returns EQ_OK and fills `a`.
+static eq_status huff_tables_from_lengths(const uint32_t *len, HuffBuildArgs &a) {
+  uint64_t kraft = 0;  // sum of 2^(32 - len), compared with 2^32
+  uint32_t max_len = 0;
+  for (int s = 0; s < 256; ++s) {
+    if (len[s] > 32) return EQ_ERR_FORMAT;
+    if (len[s]) kraft += 1ull << (32 - len[s]);
+    max_len = std::max(max_len, len[s]);
+  }
+  if (kraft > (1ull << 32)) return EQ_ERR_FORMAT;
+  for (auto &tbl : a.t) std::fill(std::begin(tbl), std::end(tbl), kHuffInvalid);
+  uint32_t ntab = 1;
+  // canonical order: by (length, value); code values increase by one, shifted as length grows
+  uint64_t code = 0;
+  uint32_t prev = 0;
+  for (uint32_t l = 1; l <= 32; ++l)
+    for (int s = 0; s < 256; ++s) {
+      if (len[s] != l) continue;
+      if (prev) code <<= (l - prev);
+      prev = l;
+      uint32_t table = 0, rem = l;
+      while (rem > 8) {  // walk / create the pointer chain for the leading 8-bit groups
+        uint32_t idx = uint32_t(code >> (rem - 8)) & 0xFFu;
+        uint16_t &e = a.t[table][idx];
+        if (e == kHuffInvalid) {
+          if (ntab >= kHuffMaxTables) return EQ_ERR_UNSUPPORTED;
+          e = uint16_t(0x8000u | ntab);
+          ++ntab;
+        } else if (!(e & 0x8000u)) {
+          return EQ_ERR_FORMAT;  // a shorter code is a prefix of this one
+        }
+        table = e & 0xFFu;
+        rem -= 8;
+      }
+      uint32_t lo = uint32_t(code & ((1ull << rem) - 1)) << (8 - rem);
+      for (uint32_t k = 0; k < (1u << (8 - rem)); ++k) {
+        uint16_t &e = a.t[table][lo + k];
+        if (e != kHuffInvalid) return EQ_ERR_FORMAT;
+        e = uint16_t((rem << 8) | uint32_t(s));
+      }
+      code += 1;
+    }
+  a.h = HuffTableHeader{kHuffMagic, ntab, max_len, 0u};
+  return EQ_OK;
+}
+
+static int g_sm_count[64];
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && g_sm_count[dev]) return g_sm_count[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev < 64) g_sm_count[dev] = n;
+  return n;
+}
+
+}  // namespace eq
+
+using namespace eq;
+
+extern "C" size_t eq_table_bytes(eq_table_kind kind) {
+  if (kind == EQ_TABLE_RANS) return kRansTableBytes;
+  if (kind == EQ_TABLE_HUFF) return kHuffTableBytes;
+  return 0;
+}
+
+extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in,
+                                     uint32_t prob_bits, void *d_tables, void *stream) {
+  if (!host_in || !d_tables || !aligned(d_tables, 16)) return EQ_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (kind == EQ_TABLE_RANS) {
+    if (prob_bits != kRansProbBits) return EQ_ERR_UNSUPPORTED;
+    RansBuildArgs a;
+    a.dst = static_cast<uint32_t *>(d_tables);
+    uint64_t sum = 0;
+    uint32_t used = 0, single = 0;
+    for (int s = 0; s < 256; ++s) {
+      if (host_in[s] > kRansSlots) return EQ_ERR_FORMAT;
+      a.freq[s] = uint16_t(host_in[s]);
+      sum += host_in[s];
+      if (host_in[s]) {
+        ++used;
+        single = uint32_t(s);
+      }
+    }
+    if (sum != kRansSlots) return EQ_ERR_FORMAT;
+    a.flags = (host_in[0x7F] ? kRansFlagNaN7F : 0u) | (host_in[0xFF] ? kRansFlagNaNFF : 0u) |
+              (used == 1 ? kRansFlagSingle : 0u);
+    a.single = used == 1 ? single : 0u;
+    rans_build_kernel<<<1, 256, 0, st>>>(a);
+    return cuda_status(cudaGetLastError());
+  }
+  if (kind == EQ_TABLE_HUFF) {
+    static thread_local HuffBuildArgs a;  // 16 KB: too large for the stack of some callers
+    a.dst = static_cast<uint32_t *>(d_tables);
+    eq_status s = huff_tables_from_lengths(host_in, a);
+    if (s != EQ_OK) return s;
+    huff_build_kernel<<<1, 256, 0, st>>>(a);
+    return cuda_status(cudaGetLastError());
+  }
+  return EQ_ERR_ARG;
+}
+
+extern "C" const char *eq_status_string(eq_status s) {
+  switch (s) {
+    case EQ_OK: return "ok";
+    case EQ_ERR_ARG: return "invalid argument";
+    case EQ_ERR_FORMAT: return "malformed coded tensor or table";
+    case EQ_ERR_UNSUPPORTED: return "unsupported format parameters";
+    case EQ_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+extern "C" uint32_t eq_abi_version(void) { return EQ_ABI_VERSION; }

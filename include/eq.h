@@ -1,0 +1,181 @@
+/*
+ * eq.h -- C ABI of the B200 (sm_100a) entropy-coded weight decoder.
+ *
+ * The library turns entropy-coded LLM weights that live in device memory back into bf16, or
+ * multiplies them straight from their coded form:
+ *
+ *   eq_build_tables      frequency table or Huffman code lengths -> device decode tables
+ *   eq_decode            interleaved-rANS Float8-E4M3 / Int8 symbols -> bf16 weights
+ *   eq_decode_gemv       interleaved-rANS weights times activations, y = W x, W never in HBM
+ *   eq_huff_bf16_decode  DFloat11 (Huffman-coded exponent + raw sign/mantissa) -> bf16
+ *
+ * Conventions shared by every call:
+ *   - Every pointer inside a tensor descriptor is DEVICE memory owned by the caller; the library
+ *     never allocates, frees or keeps device memory, and keeps no pointer after the call.
+ *   - Descriptors and other host arguments are read during the call and may be freed when it
+ *     returns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream).  Nothing synchronises the host.
+ *   - Argument and format errors found on the host return an eq_status without launching.
+ *     A failed launch returns EQ_ERR_CUDA.
+ *   - Corrupt data is reported on the device: the kernels OR EQ_DEV_* bits into *d_status (a
+ *     caller-zeroed uint32 in device memory) and never trap.  Output written for a chunk whose
+ *     status bit is set is unspecified.
+ *
+ * Where the pages leave a format open, the reading used is stated at the field.
+ */
+#ifndef EQ_H
+#define EQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define EQ_ABI_VERSION 1u
+
+typedef enum {
+  EQ_OK = 0,
+  EQ_ERR_ARG = 1,         /* a pointer is NULL, a size is out of range, or fields disagree */
+  EQ_ERR_FORMAT = 2,      /* a table or header violates the coded format                   */
+  EQ_ERR_UNSUPPORTED = 3, /* valid format, but outside what this build decodes              */
+  EQ_ERR_CUDA = 4         /* a CUDA call or launch failed                                   */
+} eq_status;
+
+/* device-side status bits, OR-ed into *d_status */
+#define EQ_DEV_CORRUPT_STATE 1u  /* a rANS stream did not end in state 2^16                   */
+#define EQ_DEV_OVERRUN 2u        /* a chunk asked for more words / bits than it holds         */
+#define EQ_DEV_BAD_CODE 4u       /* Huffman: a bit pattern matches no code                    */
+#define EQ_DEV_COUNT_MISMATCH 8u /* Huffman: codes found in a block differ from block_out     */
+#define EQ_DEV_TIMEOUT 16u       /* a bounded wait on an asynchronous copy gave up            */
+
+typedef enum { EQ_SYM_E4M3 = 1, EQ_SYM_INT8 = 2 } eq_symfmt;
+typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
+
+/*
+ * One interleaved-rANS-coded weight W[rows][cols] ("Float8@2bits: Entropy Coding Enables
+ * Data-Free Model Compression", summary sections "Codificacion de Pesos" and "Decodificacion en
+ * Tiempo de Inferencia": the optimised weights, Float8-E4M3 or Int8 symbols with one scale per
+ * output channel, are flattened into one symbol stream and ANS-coded; a parallel ANS decoder
+ * restores them on the GPU before the layer runs).  The pages fix no rANS variant; this one is:
+ *
+ *   probabilities M = 2^prob_bits (prob_bits = 12), state x in [2^16, 2^32), 16-bit words.
+ *   The row-major symbol stream is cut into chunks of chunk_symbols symbols (the last one may be
+ *   shorter); chunk c is coded on its own by `streams` interleaved rANS states.  Inside a chunk,
+ *   symbol j belongs to run r = j / run, stream r % streams, round r / streams, position j % run;
+ *   the decoder visits (round, position, stream) in increasing order and skips streams that hold
+ *   no symbol at that step.  Decoding symbol s from x: slot = x mod M, s is the symbol with
+ *   cum[s] <= slot < cum[s] + freq[s], x = freq[s] * (x / M) + slot - cum[s]; then, if x < 2^16,
+ *   x = x * 2^16 + the chunk's next word.  A well-formed chunk ends with every state at 2^16 and
+ *   every word read.
+ *   Dequantisation: out = bf16_rne( value(s) * scale[row] ), value(s) being the E4M3 value of the
+ *   byte (NaN codes 0x7F/0xFF give the bf16 quiet NaN 0x7FC0 / 0xFFC0) or the byte read as int8.
+ */
+typedef struct {
+  uint32_t version;       /* EQ_ABI_VERSION                                                    */
+  uint32_t symfmt;        /* eq_symfmt                                                         */
+  uint32_t rows, cols;    /* W is rows x cols, row-major; rows*cols < 2^40                     */
+  uint32_t prob_bits;     /* 12                                                                */
+  uint32_t chunk_symbols; /* symbols per chunk (>= 1); a multiple of `run`                     */
+  uint32_t streams;       /* interleaved states per chunk: 32, 64, 96 ... 256                  */
+  uint32_t run;           /* consecutive symbols per stream visit: 1 or 8; 8 needs cols % 8 == 0 */
+  uint64_t num_chunks;    /* ceil(rows * cols / chunk_symbols)                                 */
+  const uint32_t *states; /* [num_chunks][streams] final encoder states                         */
+  const uint64_t *word_off; /* [num_chunks + 1] start of each chunk's words, in words           */
+  const uint16_t *words;  /* all chunks' words, decoder order; allocation padded with zeros to a
+                             multiple of 8 words (16 bytes); base 16-byte aligned               */
+  const uint16_t *scales; /* [rows] bf16 per-output-channel scales                              */
+  const void *tables;     /* eq_table_bytes(EQ_TABLE_RANS) bytes from eq_build_tables(RANS);
+                             16-byte aligned                                                    */
+} eq_rans_tensor;
+
+/*
+ * One DFloat11-coded bf16 weight (DFloat11 page, "Formato DFloat11": the 8-bit exponent is
+ * Huffman-coded and bit-packed into EncodedExponent, sign and mantissa stay raw in
+ * PackedSignMantissa; "Kernels GPU de 2 etapas y metadatos auxiliares": each thread owns 8
+ * contiguous bytes of EncodedExponent and decodes the codes that start there, Gaps gives each
+ * thread's first code offset in 5 bits, and one output position is stored per thread block).
+ *
+ *   exponent e = bits 14..7 of the bf16; PackedSignMantissa byte = sign << 7 | low 7 bits.
+ *   Codes are canonical (symbols ordered by (length, value) get consecutive codes), written
+ *   MSB-first from bit 0 of byte 0.  Thread t owns bits [64 t, 64 t + 64); Gap[t] is the offset
+ *   from 64 t of the first code starting at or after 64 t (0..31, 5 bits, LSB-first packing).
+ *   threads = ceil(total_bits / 64); blocks = ceil(threads / threads_per_block);
+ *   block_out[b] = index of the first weight decoded by block b; block_out[blocks] = n.
+ */
+typedef struct {
+  uint64_t n;                  /* number of bf16 weights                                      */
+  uint64_t total_bits;         /* length of the code stream in bits                           */
+  uint32_t bytes_per_thread;   /* 8                                                           */
+  uint32_t threads_per_block;  /* 256                                                         */
+  const uint8_t *enc_exp;      /* EncodedExponent, threads * 8 bytes + 16 zero bytes           */
+  const uint8_t *sign_mant;    /* PackedSignMantissa [n]                                      */
+  const uint8_t *gaps;         /* ceil(5 threads / 8) bytes + 8 zero bytes                    */
+  const uint64_t *block_out;   /* [blocks + 1]                                                */
+  const void *tables;          /* eq_table_bytes(EQ_TABLE_HUFF) bytes from eq_build_tables(HUFF) */
+} eq_huff_tensor;
+
+/* Bytes of device memory eq_build_tables writes for `kind` (0 for an unknown kind). */
+size_t eq_table_bytes(eq_table_kind kind);
+
+/*
+ * Build the device decode tables of one tensor into d_tables (eq_table_bytes(kind) bytes,
+ * 16-byte aligned, caller-owned).  The table contents travel as kernel arguments: no host
+ * buffer outlives the call and no copy engine is used.
+ *   EQ_TABLE_RANS: host_in[256] = symbol frequencies, summing to 2^prob_bits (prob_bits = 12).
+ *     Builds the slot table: one 32-bit entry per slot holding the slot's symbol, its frequency
+ *     and slot - cum[symbol].
+ *   EQ_TABLE_HUFF: host_in[256] = code length of each exponent value (0 = absent), prob_bits
+ *     ignored.  Builds the hierarchical lookup tables of the DFloat11 page ("Decodificacion
+ *     basada en LUT jerarquicas"): the code tree is cut into height-8 subtrees, each a 256-entry
+ *     table.  EQ_ERR_FORMAT if a length exceeds 32 or the lengths violate the Kraft inequality;
+ *     EQ_ERR_UNSUPPORTED if more than 32 subtables would be needed.
+ */
+eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in, uint32_t prob_bits,
+                          void *d_tables, void *stream);
+
+/*
+ * Decode n_tensors rANS-coded weights to bf16 (one launch per group of tensors that share
+ * symfmt, streams and run).  d_out[i] points to rows*cols bf16 values (16-byte aligned) for
+ * tensor i; the array d_out itself is host memory.  Decoding all tensors of a transformer block
+ * in one call follows the pages' block-wise decompression (DFloat11 page, "Descompresion por
+ * bloque transformer"; "Float8@2bits" summary: decompression alternates with the forward
+ * kernels block by block).
+ */
+eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uint16_t *const *d_out,
+                    uint32_t *d_status, void *stream);
+
+/*
+ * y[b][r] = sum_c W[r][c] * x[b][c] for b < batch, with W decoded from its rANS stream on chip
+ * and never written to memory ("Float8@2bits" summary, closing section: fused decompression
+ * kernels are the next step; the decoded values are consumed where they are produced).
+ * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].
+ * Requires chunk_symbols to be a multiple of cols (every chunk holds whole rows) and run == 8.
+ * batch 1..16; batch >= 8 runs the product on the tensor cores.  The fp32 result is within a
+ * relative L2 error of 1e-3 of the exact product of the decoded bf16 weights.
+ */
+eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x, uint32_t batch, float *d_y,
+                         uint32_t *d_status, void *stream);
+
+/*
+ * Reconstruct n bf16 weights from their DFloat11 coding, bit-exactly (DFloat11 page, "Kernels
+ * GPU de 2 etapas y metadatos auxiliares": stage 1 decodes and counts, a block-wide prefix sum
+ * gives every thread its output position, stage 2 decodes again into shared memory and the block
+ * writes its span once, coalesced).  d_out: n bf16 values.
+ */
+eq_status eq_huff_bf16_decode(const eq_huff_tensor *h, uint16_t *d_out, uint32_t *d_status,
+                              void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *eq_status_string(eq_status s);
+
+/* EQ_ABI_VERSION of the loaded library. */
+uint32_t eq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQ_H */

@@ -1,0 +1,75 @@
+/*
+ * eq_encode.h -- host-side compressor of the library (the offline step that produces what the
+ * decoders in eq.h consume).
+ *
+ * The pages compress once, offline, then keep the weights coded in GPU memory ("Float8@2bits"
+ * summary, "Codificacion de Pesos": per-channel AbsMax scales, Float8/Int8 symbols, ANS over the
+ * flattened stream; DFloat11 page, "Formato DFloat11": Huffman-coded bf16 exponents).  These calls
+ * run on the host CPU with worker threads; none of them touches the GPU.  The formats are the ones
+ * defined in eq.h.  Arrays are host memory owned by the caller unless stated otherwise.
+ */
+#ifndef EQ_ENCODE_H
+#define EQ_ENCODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "eq.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Per-output-channel AbsMax quantisation of an fp32 weight w[rows][cols].
+ *   E4M3: scale[r] = bf16(max_c |w[r][c]| / 448), sym = E4M3(w / scale[r]) (round to nearest even,
+ *         saturating at 448).
+ *   INT8: scale[r] = bf16(max_c |w[r][c]| / int8_div), sym = clamp(rne(w / scale[r]), -127, 127).
+ * A row of zeros gets scale 1.0.  threads = 0 uses every available core.
+ */
+eq_status eq_quantize_host(const float *w, uint32_t rows, uint32_t cols, uint32_t symfmt,
+                           float int8_div, uint8_t *sym, uint16_t *scales, uint32_t threads);
+
+/*
+ * Frequency table for rANS, summing to 2^prob_bits: f = 0 for absent symbols, else
+ * max(1, floor(count * 2^prob_bits / n)); the remainder goes to the most frequent symbol (lowest
+ * byte on ties); an excess is taken back one unit at a time from the largest f > 1 (lowest byte
+ * on ties).  n = 0 gives f[0] = 2^prob_bits.
+ */
+eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t prob_bits, uint32_t *freqs);
+
+/*
+ * Interleaved-rANS encoding of a symbol matrix sym[rows][cols] in the format of eq_rans_tensor.
+ * chunk_symbols = 0 means one row per chunk.  states: [num_chunks * streams]; word_off:
+ * [num_chunks + 1].  The words are returned in a buffer the library allocates (*words, *n_words
+ * words, zero-padded to a multiple of 8); release it with eq_free_host.
+ */
+eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint32_t cols,
+                              const uint32_t *freqs, uint32_t chunk_symbols, uint32_t streams,
+                              uint32_t run, uint32_t threads, uint32_t *states, uint64_t *word_off,
+                              uint16_t **words, uint64_t *n_words);
+
+/* Optimal Huffman code lengths (no length above max_len) for 256 symbol counts. */
+eq_status eq_huff_lengths_host(const uint64_t *counts, uint32_t max_len, uint32_t *lengths);
+
+/*
+ * DFloat11 coding of n bf16 weights (eq_huff_tensor format) with the given code lengths.
+ * First call eq_huff_plan_host to learn total_bits; the caller then allocates
+ *   enc_exp   threads * 8 + 16 bytes,   sign_mant n bytes,
+ *   gaps      ceil(5 * threads / 8) + 8 bytes,   block_out blocks + 1 entries,
+ * with threads = ceil(total_bits / 64) and blocks = ceil(threads / threads_per_block), zeroed.
+ */
+eq_status eq_huff_plan_host(const uint16_t *w, uint64_t n, const uint32_t *lengths,
+                            uint64_t *total_bits);
+eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const uint32_t *lengths,
+                              uint32_t threads_per_block, uint64_t total_bits, uint8_t *enc_exp,
+                              uint8_t *sign_mant, uint8_t *gaps, uint64_t *block_out);
+
+/* Release a buffer returned by eq_rans_encode_host. */
+void eq_free_host(void *p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EQ_ENCODE_H */

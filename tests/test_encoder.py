@@ -1,0 +1,86 @@
+"""The library's host compressor (include/eq_encode.h) against the oracle: same symbols, scales,
+frequency tables, rANS containers and DFloat11 containers, bit for bit (the formats leave no
+freedom once the tables are fixed)."""
+import numpy as np
+import pytest
+
+import synth
+
+
+@pytest.fixture(scope="module")
+def eq():
+    import decoding_interleaved_rans_b200 as m
+    m.lib()
+    return m
+
+
+@pytest.mark.parametrize("name", ["e4m3_1k", "int8_8k", "mlp_13b"])
+def test_quantize_matches_oracle(eq, orc, name):
+    wl = synth.WORKLOADS[name]
+    spec = wl.tensors[0]
+    w = spec.generate(row_lo=0, row_hi=min(spec.rows, 300))
+    fmt = 1 if wl.symfmt == "e4m3" else 2
+    a = eq.codec.quantize(w, fmt, wl.int8_div)
+    b = orc.quantize(w, fmt, wl.int8_div)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_quantize_edge_values(eq, orc):
+    rng = np.random.default_rng(1)
+    w = (rng.standard_normal((40, 300)) * 10.0 ** rng.uniform(-8, 3, (40, 300))).astype(np.float32)
+    w[0] = 0.0
+    w[1, :5] = [448.0 * 3, -1e-30, 1e-40, -0.0, 7.0]
+    for fmt in (1, 2):
+        a = eq.codec.quantize(w, fmt, 3.7)
+        b = orc.quantize(w, fmt, 3.7)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("chunk,S,G", [(16384, 32, 8), (65536, 128, 8), (0, 64, 8), (999, 32, 1),
+                                       (4096, 256, 8)])
+def test_rans_encode_matches_oracle(eq, orc, chunk, S, G):
+    w = synth.normal_with_outliers(96, 1024, 0.02, 0.01, 8.0, 5)
+    sym, sc = orc.quantize(w, orc.E4M3)
+    fa = eq.codec.rans_freqs(sym)
+    assert np.array_equal(fa, orc.rans_freqs(sym))
+    a = eq.codec.rans_encode(sym, sc, 1, chunk, S, G)
+    b = orc.rans_encode(sym, sc, 1, chunk, S, G)
+    assert np.array_equal(a.states, b.states)
+    assert np.array_equal(a.word_off, b.word_off)
+    assert np.array_equal(a.words, b.words)
+
+
+def test_rans_freqs_edge_cases(eq, orc):
+    for sym in [np.zeros(0, np.uint8), np.full(10, 3, np.uint8), np.arange(256, dtype=np.uint8),
+                np.repeat(np.arange(256, dtype=np.uint8), np.arange(1, 257))]:
+        assert np.array_equal(eq.codec.rans_freqs(sym), orc.rans_freqs(sym))
+
+
+@pytest.mark.parametrize("tpb", [256, 32, 1])
+def test_huff_encode_matches_oracle(eq, orc, tpb):
+    w = synth.bf16_normal(32, 4096, 0.015, 6)
+    a = eq.codec.huff_encode(w, tpb)
+    b = orc.huff_encode_bf16(w, tpb)
+    assert np.array_equal(a.lengths, b.lengths)
+    assert a.total_bits == b.total_bits
+    for f in ("enc_exp", "sign_mant", "gaps", "block_out"):
+        assert np.array_equal(getattr(a, f), getattr(b, f)), f
+
+
+def test_huff_lengths_optimal_and_capped(eq, orc):
+    rng = np.random.default_rng(2)
+    for _ in range(100):
+        counts = np.zeros(256, np.uint64)
+        k = int(rng.integers(1, 80))
+        counts[rng.choice(256, k, replace=False)] = rng.integers(1, 10 ** 6, k).astype(np.uint64)
+        a = eq.codec.huff_lengths(counts).astype(np.int64)
+        b = orc.huff_lengths(counts).astype(np.int64)
+        assert (a * counts.astype(np.int64)).sum() == (b * counts.astype(np.int64)).sum()
+    fib = [1, 1]
+    while len(fib) < 40:
+        fib.append(fib[-1] + fib[-2])
+    counts = np.zeros(256, np.uint64)
+    counts[:40] = fib
+    a = eq.codec.huff_lengths(counts, 32)
+    b = orc.huff_lengths(counts, 32)
+    assert a.max() <= 32 and np.array_equal(a, b.astype(np.uint32))

@@ -245,8 +245,28 @@ def run_ours(args):
 
 
 def extra_measurements(eq, dev, stream, flush, peaks, args):
-    """Fused decode-GEMV and DFloat11 decode, when the library provides them."""
+    """Fused decode-GEMV (13B MLP, batch 1/4/16) and DFloat11 decode (8192x28672 bf16)."""
+    import torch
     out = []
+    steps = max(5, args.steps // 2)
+    # DFloat11: algorithmic bytes = EncodedExponent + PackedSignMantissa + Gaps + block_out
+    # read, 2 B/weight written
+    w = synth.WORKLOADS["df11_8k"].tensors[0].generate().ravel()
+    hh = eq.codec.huff_encode(w)
+    del w
+    dh = eq.DeviceHuff.upload(hh, dev)
+    ob = torch.empty(dh.n, dtype=torch.bfloat16, device=dev)
+    st = eq.new_status(dev)
+    ts = time_steps(lambda: eq.huff_bf16_decode(dh, ob, st, stream), steps, 3, flush, stream)
+    assert int(st.item()) == 0
+    sec = statistics.mean(ts)
+    alg = dh.compressed_bytes + 2 * dh.n
+    out.append({"what": "DFloat11 bf16 decode, 8192x28672 N(0,0.015)", "params": dh.n,
+                "ms": sec * 1e3, "params_per_s": dh.n / sec, "gbs": alg / sec / 1e9,
+                "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"],
+                "bits_per_param": 8 * dh.compressed_bytes / dh.n,
+                "kernel": "huff_decode_kernel"})
+    del dh, ob
     return out
 
 
@@ -313,8 +333,38 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def profile_kernel(kind: str, launches: int = 5):
+    """A few launches of one kernel on its workload, nothing else: the command ncu captures."""
+    import torch
+
+    import decoding_interleaved_rans_b200 as eq
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    if kind == "decode":
+        _, h = prepare_rans(eq, WORKLOAD)
+        t = eq.DeviceRans.upload(h, dev)
+        out = torch.empty(h.rows, h.cols, dtype=torch.bfloat16, device=dev)
+        st = eq.new_status(dev)
+        fn = lambda: eq.decode([t], [out], st)  # noqa: E731
+    elif kind == "huff":
+        w = synth.WORKLOADS["df11_8k"].tensors[0].generate(row_lo=0, row_hi=2048).ravel()
+        dh = eq.DeviceHuff.upload(eq.codec.huff_encode(w), dev)
+        ob = torch.empty(dh.n, dtype=torch.bfloat16, device=dev)
+        st = eq.new_status(dev)
+        fn = lambda: eq.huff_bf16_decode(dh, ob, st)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown kernel {kind}")
+    for _ in range(launches):
+        fn()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    print(f"profiled {kind}: {launches} launches ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile-kernel", default=None, choices=["decode", "huff", "gemv"],
+                    help="launch one kernel a few times and exit (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
@@ -324,6 +374,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile_kernel:
+        profile_kernel(args.profile_kernel)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

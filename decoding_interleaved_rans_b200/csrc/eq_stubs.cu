@@ -5,7 +5,3 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *, const uint16_t *, ui
                                     uint32_t *, void *) {
   return EQ_ERR_UNSUPPORTED;
 }
-
-extern "C" eq_status eq_huff_bf16_decode(const eq_huff_tensor *, uint16_t *, uint32_t *, void *) {
-  return EQ_ERR_UNSUPPORTED;
-}

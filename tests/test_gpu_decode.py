@@ -148,7 +148,7 @@ def test_corruption_sets_status(eq, orc):
     h.states = h.states.copy()
     h.states[40] ^= 0x1234
     _, st = run_decode(eq, [h])
-    assert st & 1
+    assert st & 3  # the stream ends in a wrong state or runs past its words
     # truncated chunk: drop its last word (offsets shifted, stream shorter than it needs)
     h = orc.rans_encode(sym, sc, orc.E4M3, 16384, 32, 8)
     h.word_off = h.word_off.copy()

@@ -267,6 +267,34 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                 "bits_per_param": 8 * dh.compressed_bytes / dh.n,
                 "kernel": "huff_decode_kernel"})
     del dh, ob
+    # fused decode + GEMV over the three 13B MLP weights (gate, up 13824x5120; down 5120x13824);
+    # algorithmic bytes = the coded weights read (+ x and y)
+    wl = synth.WORKLOADS["mlp_13b"]
+    mats = []
+    for spec in wl.tensors:
+        sym, sc = eq.codec.quantize(spec.generate(), eq.EQ_SYM_E4M3)
+        h = eq.codec.rans_encode(sym, sc, eq.EQ_SYM_E4M3, wl.chunk_for(spec), wl.streams, wl.run)
+        mats.append(eq.DeviceRans.upload(h, dev))
+        del sym, sc, h
+    params = sum(m.numel for m in mats)
+    coded = sum(m.compressed_bytes for m in mats)
+    for batch in wl.batches:
+        xs = [torch.randn(batch, m.cols, device=dev).to(torch.bfloat16) for m in mats]
+        ys = [torch.empty(batch, m.rows, dtype=torch.float32, device=dev) for m in mats]
+        st = eq.new_status(dev)
+
+        def layer():
+            for m, x, y in zip(mats, xs, ys):
+                eq.decode_gemv(m, x, y, st, stream)
+        ts = time_steps(layer, steps, 3, flush, stream)
+        assert int(st.item()) == 0
+        sec = statistics.mean(ts)
+        alg = coded + sum(x.numel() * 2 for x in xs) + sum(y.numel() * 4 for y in ys)
+        out.append({"what": f"fused decode+GEMV, 13B MLP gate/up/down, batch {batch}",
+                    "params": params, "ms": sec * 1e3, "params_per_s": params / sec,
+                    "gbs": alg / sec / 1e9, "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"],
+                    "bits_per_param": 8 * coded / params, "kernel": "rans_gemv_kernel",
+                    "launches_per_step": len(mats)})
     return out
 
 
@@ -352,6 +380,16 @@ def profile_kernel(kind: str, launches: int = 5):
         ob = torch.empty(dh.n, dtype=torch.bfloat16, device=dev)
         st = eq.new_status(dev)
         fn = lambda: eq.huff_bf16_decode(dh, ob, st)  # noqa: E731
+    elif kind == "gemv":
+        wl = synth.WORKLOADS["mlp_13b"]
+        spec = wl.tensors[2]
+        sym, sc = eq.codec.quantize(spec.generate(), eq.EQ_SYM_E4M3)
+        t = eq.DeviceRans.upload(eq.codec.rans_encode(sym, sc, eq.EQ_SYM_E4M3, wl.chunk_for(spec),
+                                                      wl.streams, wl.run), dev)
+        x = torch.randn(1, t.cols, device=dev).to(torch.bfloat16)
+        y = torch.empty(1, t.rows, dtype=torch.float32, device=dev)
+        st = eq.new_status(dev)
+        fn = lambda: eq.decode_gemv(t, x, y, st)  # noqa: E731
     else:
         raise SystemExit(f"unknown kernel {kind}")
     for _ in range(launches):

@@ -79,7 +79,7 @@ def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols:
     chunk = chunk_symbols if chunk_symbols else cols
     nchunks = (rows * cols + chunk - 1) // chunk
     states = np.empty(max(1, nchunks * streams), np.uint32)
-    word_off = np.zeros(nchunks + 1, np.uint64)
+    word_off = np.zeros(nchunks * ((streams + 31) // 32) + 1, np.uint64)
     wp, nw = C.c_void_p(), C.c_uint64()
     L.check(L.lib().eq_rans_encode_host(_p(sym) if sym.size else None, rows, cols, _p(freqs),
                                         chunk_symbols, streams, run, threads, _p(states),

@@ -146,15 +146,15 @@ extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint
   for (int s = 0; s < 256; ++s) cum[s + 1] = cum[s] + freqs[s];
   if (cum[256] != 4096u) return EQ_ERR_FORMAT;
   const uint64_t nchunks = (N + chunk - 1) / chunk;
-  std::vector<std::vector<uint16_t>> pieces(nchunks);
+  const uint32_t groups = (streams + 31) / 32;  // 32 streams share one word substream
+  std::vector<std::vector<uint16_t>> pieces(nchunks * groups);
   std::atomic<int> bad{0};
   parallel_for(nchunks, threads, [&](uint64_t c) {
     const uint64_t j0 = c * chunk;
     const uint64_t n = std::min(chunk, N - j0);
     const uint8_t *s = sym + j0;
     std::vector<uint32_t> x(streams, 1u << 16);
-    std::vector<uint16_t> &out = pieces[c];  // emitted in encoder order, reversed at the end
-    out.reserve(n / 2 + 16);
+    std::vector<uint16_t> *out = &pieces[c * groups];  // encoder order, reversed at the end
     const uint64_t nruns = (n + run - 1) / run;
     const uint64_t nrounds = (nruns + streams - 1) / streams;
     for (uint64_t rr = nrounds; rr-- > 0;)
@@ -169,24 +169,25 @@ extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint
           }
           uint32_t v = x[st];
           if (uint64_t(v) >= (uint64_t(f) << 20)) {
-            out.push_back(uint16_t(v));
+            out[st / 32].push_back(uint16_t(v));
             v >>= 16;
           }
           x[st] = (v / f) * 4096u + v % f + cum[q];
         }
-    std::reverse(out.begin(), out.end());
+    for (uint32_t g = 0; g < groups; ++g) std::reverse(out[g].begin(), out[g].end());
     std::memcpy(states + c * streams, x.data(), streams * sizeof(uint32_t));
   });
   if (bad) return EQ_ERR_FORMAT;
+  const uint64_t units = nchunks * groups;
   word_off[0] = 0;
-  for (uint64_t c = 0; c < nchunks; ++c) word_off[c + 1] = word_off[c] + pieces[c].size();
-  const uint64_t total = word_off[nchunks];
+  for (uint64_t u = 0; u < units; ++u) word_off[u + 1] = word_off[u] + pieces[u].size();
+  const uint64_t total = word_off[units];
   const uint64_t padded = std::max<uint64_t>(8, (total + 7) / 8 * 8);
   uint16_t *buf = static_cast<uint16_t *>(std::calloc(padded, sizeof(uint16_t)));
   if (!buf) return EQ_ERR_ARG;
-  parallel_for(nchunks, threads, [&](uint64_t c) {
-    if (!pieces[c].empty())
-      std::memcpy(buf + word_off[c], pieces[c].data(), pieces[c].size() * sizeof(uint16_t));
+  parallel_for(units, threads, [&](uint64_t u) {
+    if (!pieces[u].empty())
+      std::memcpy(buf + word_off[u], pieces[u].data(), pieces[u].size() * sizeof(uint16_t));
   });
   *words = buf;
   *n_words = padded;

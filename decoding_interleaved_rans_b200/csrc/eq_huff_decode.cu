@@ -10,8 +10,9 @@
 //
 // Different from the page's kernel, which decodes every segment twice (count, then decode again
 // and write): a B200 SM has room to keep the first pass, so each thread decodes once into a
-// private 64-byte shared-memory slot (a 64-bit segment holds at most 64 code starts), and after
-// the scan copies its exponents to their block position.  The block scan is a warp-shuffle scan
+// private 64-byte shared-memory slot (a 64-bit segment holds at most 64 code starts; the slots are
+// interleaved so that a warp's byte stores fall in distinct banks), and after the scan copies its
+// exponents to their block position.  The block scan is a warp-shuffle scan
 // rather than Blelloch's tree.
 #include "eq_internal.cuh"
 
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(1024) huff_decode_kernel(const __grid_constant
     buf <<= gap;
     int valid = 64 - int(gap);
     bool more = true;
-    uint8_t *mine = priv + tid * 64;
+    uint8_t *mine = priv + tid;  // column-major: code k of thread t at priv[k * T + t]
     while (pos < end) {
       if (valid < 32 && more) {  // pull in the 32 bits after the segment (codes reach <= 31 past it)
         buf |= uint64_t(nxt) << (32 - valid);
@@ -98,7 +99,8 @@ __global__ void __launch_bounds__(1024) huff_decode_kernel(const __grid_constant
         break;
       }
       const uint32_t len = used + rem;
-      mine[cnt++] = uint8_t(e & 0xFFu);
+      mine[cnt * T] = uint8_t(e & 0xFFu);
+      ++cnt;
       buf <<= len;
       valid -= int(len);
       pos += len;
@@ -142,7 +144,7 @@ __global__ void __launch_bounds__(1024) huff_decode_kernel(const __grid_constant
   //      8-aligned in shared memory) ----
   const uint32_t shift = uint32_t(o0 & 7);
   for (uint32_t k = 0; k < cnt; ++k)
-    if (off + k < m) ebuf[shift + off + k] = priv[tid * 64 + k];
+    if (off + k < m) ebuf[shift + off + k] = priv[k * T + tid];
   __syncthreads();
 
   // ---- merge with PackedSignMantissa and write the block's span ----

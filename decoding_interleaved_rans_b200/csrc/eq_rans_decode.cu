@@ -3,27 +3,26 @@
 // What it computes is fixed by the format in eq.h ("Float8@2bits" summary: Float8-E4M3 / Int8
 // symbols with per-channel scales, flattened and ANS-coded, decoded on the GPU into a buffer before
 // the layer runs).  How, on B200:
-//   * one warp decodes one chunk; lane l runs the K = streams/32 states l, l+32, ... so the K
-//     dependency chains of a lane interleave and hide the shared-memory latency;
+//   * one warp decodes one group of 32 streams of a chunk, one rANS state per lane; the groups of a
+//     chunk read separate word substreams, so a 64 KiB chunk keeps several warps busy and an SM
+//     holds dozens of independent decoders to hide the shared-memory latency of each step;
 //   * the 4096-entry slot table (16 KiB) sits in shared memory, one 32-bit load per symbol;
-//   * the chunk's 16-bit words stream through a per-warp shared-memory ring fed by 1-D bulk copies
-//     (TMA engine, completion on an mbarrier), so HBM reads are large and asynchronous;
-//   * renormalisation is warp-cooperative: a ballot of the states that need a word, a popcount
-//     rank gives each its word, in stream order, from the ring;
-//   * with run = 8 a lane emits eight consecutive bf16 per state and round: one 16-byte store,
-//     a warp writes 512 contiguous bytes per state index;
+//   * the group's 16-bit words stream through a per-warp shared-memory ring fed by 1-D bulk copies
+//     (TMA engine, completion on an mbarrier), checked and refilled once per round of 8 steps;
+//   * renormalisation is warp-cooperative: a ballot of the lanes whose state fell below 2^16, a
+//     popcount rank hands each its word, in stream order;
+//   * with run = 8 a lane emits eight consecutive bf16 per round: one 16-byte store, the warp
+//     writes 512 contiguous bytes;
 //   * dequantisation (value * row scale, one rounding) happens in registers before the store.
 // Many tensors go in one launch (the pages decode all weights of a transformer block together).
 #include <algorithm>
 #include <vector>
 
 #include "eq_dequant.cuh"
+#include "eq_rans_core.cuh"
 
 namespace eq {
 
-constexpr uint32_t kSegBytes = 1024;
-constexpr uint32_t kNumSeg = 4;
-constexpr uint32_t kRingBytes = kSegBytes * kNumSeg;
 constexpr int kMaxDecodeTensors = 192;
 
 struct RansDesc {
@@ -34,10 +33,10 @@ struct RansDesc {
   const uint32_t *table;  // RansTableHeader followed by the slot table
   uint16_t *out;
   uint64_t numel;
-  uint64_t num_chunks;
+  uint64_t units;         // num_chunks * groups: one warp each
   uint64_t row_magic;     // floor(j / cols) = __umul64hi(j, row_magic) (0: cols == 1)
-  uint32_t cols;
   uint32_t chunk_symbols;
+  uint32_t groups;        // streams / 32
   uint32_t cta_begin;     // first CTA of this tensor in the launch
   uint32_t pad;
 };
@@ -45,193 +44,96 @@ struct RansDesc {
 struct RansDecodeParams {
   uint32_t *status;
   uint32_t n;
-  uint32_t warps;  // warps per CTA = chunks per CTA
+  uint32_t warps;  // warps (= groups decoded) per CTA
   RansDesc d[kMaxDecodeTensors];
 };
 
-__host__ __device__ constexpr size_t decode_smem_bytes(uint32_t warps) {
-  return kRansSlots * 4 + warps * (kRingBytes + kNumSeg * 8);
+// ------------------------------------------------------------------------------------------------
+// one round (G steps) of one group; FULL: every lane holds a run this round
+// ------------------------------------------------------------------------------------------------
+template <bool FULL, int G, int FMT>
+__device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
+                                             const uint32_t *lut, const WordRing &R, uint32_t &q,
+                                             uint32_t lt, uint64_t jrun, bool nan_codes) {
+  uint32_t sym[(G + 3) / 4] = {};
+#pragma unroll
+  for (int p = 0; p < G; ++p) {
+    const uint32_t e = rans_step<FULL>(x, act, lut, R, q, lt);
+    sym[p >> 2] = put_sym(sym[p >> 2], e, p & 3);
+  }
+  if (FULL || act) {
+    const float sc = bf16_bits_to_float(D.scales[div_by_magic(jrun, D.row_magic)]);
+    if constexpr (G == 8) {
+      const uint2 a = dequant4<FMT>(sym[0], sc, nan_codes);
+      const uint2 b = dequant4<FMT>(sym[1], sc, nan_codes);
+      *reinterpret_cast<uint4 *>(D.out + jrun) = make_uint4(a.x, a.y, b.x, b.y);
+    } else {
+      D.out[jrun] = dequant1<FMT>(sym[0], sc);
+    }
+  }
 }
 
-// ------------------------------------------------------------------------------------------------
-// per-warp word ring: segment s of the chunk's (16-byte aligned) word span lives in slot s % 4
-// ------------------------------------------------------------------------------------------------
-struct WordRing {
-  unsigned char *buf;
-  uint64_t *bar;
-  const unsigned char *A;  // chunk word span start, rounded down to 16 bytes
-  uint32_t off0;           // bytes from A to the chunk's first word
-  uint32_t span;           // bytes to copy (multiple of 16)
-  uint32_t nseg;
-  uint32_t issued;         // segments handed to the copy engine
-  uint32_t ready;          // segments waited for
-
-  __device__ __forceinline__ void issue(uint32_t lane) {
-    if (lane == 0) {
-      const uint32_t s = issued, slot = s % kNumSeg;
-      const uint32_t bytes = min(kSegBytes, span - s * kSegBytes);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_expect_tx(&bar[slot], bytes);
-      bulk_g2s(buf + slot * kSegBytes, A + size_t(s) * kSegBytes, bytes, &bar[slot]);
-    }
-    ++issued;
-  }
-  // make every segment up to `last` readable; false on timeout
-  __device__ __forceinline__ bool wait_upto(uint32_t last) {
-    while (ready <= last) {
-      if (!mbar_wait_bounded(&bar[ready % kNumSeg], (ready / kNumSeg) & 1u)) return false;
-      ++ready;
-    }
-    return true;
-  }
-  // refill slots whose segment lies entirely before word `ptr`
-  __device__ __forceinline__ void refill(uint32_t ptr, uint32_t lane) {
-    const uint32_t cur = (off0 + 2 * ptr) / kSegBytes;
-    if (issued < nseg && issued < cur + kNumSeg) {
-      __syncwarp();
-      do issue(lane);
-      while (issued < nseg && issued < cur + kNumSeg);
-    }
-  }
-  __device__ __forceinline__ uint32_t word(uint32_t idx) const {
-    return *reinterpret_cast<const uint16_t *>(buf + ((off0 + 2 * idx) & (kRingBytes - 1)));
-  }
-};
-
-// ------------------------------------------------------------------------------------------------
-// one chunk, K states per lane, run length G, symbol format FMT
-// ------------------------------------------------------------------------------------------------
-template <int K, int G, int FMT>
-__device__ __forceinline__ uint32_t decode_chunk(const RansDesc &D, const uint32_t *lut,
-                                                 uint32_t flags, uint32_t single_sym,
-                                                 WordRing &R, uint64_t chunk, uint32_t lane) {
-  constexpr uint32_t S = 32 * K;
+template <int G, int FMT>
+__device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32_t *lut,
+                                                 uint32_t flags, uint32_t single_sym, WordRing &R,
+                                                 uint64_t unit, uint32_t lane) {
+  const uint64_t chunk = unit / D.groups;
+  const uint32_t g = uint32_t(unit - chunk * D.groups);
+  const uint32_t S = 32 * D.groups, s = 32 * g + lane;
   const uint64_t j0 = chunk * uint64_t(D.chunk_symbols);
   const uint32_t n = uint32_t(D.numel - j0 < D.chunk_symbols ? D.numel - j0 : D.chunk_symbols);
-  const uint64_t w0 = D.word_off[chunk], w1 = D.word_off[chunk + 1];
-  if (w1 < w0 || w1 - w0 >= (1ull << 31)) return EQ_DEV_OVERRUN;
+  const uint64_t w0 = D.word_off[unit], w1 = D.word_off[unit + 1];
+  if (w1 < w0 || w1 - w0 >= (1ull << 30)) return EQ_DEV_OVERRUN;
   const uint32_t nwords = uint32_t(w1 - w0);
+  const uint32_t runs = (n + G - 1) / G;
+  const uint32_t rounds = (runs + S - 1) / S;
+  uint32_t x = D.states[chunk * S + s];
   uint32_t status = 0;
 
-  uint32_t x[K];
-#pragma unroll
-  for (int k = 0; k < K; ++k) x[k] = D.states[chunk * S + lane + 32 * k];
-
   if (flags & kRansFlagSingle) {  // one symbol owns every slot: states never move, no words
-    bool ok = nwords == 0;
-#pragma unroll
-    for (int k = 0; k < K; ++k) ok &= x[k] == kRansL;
-    if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
-    for (uint32_t i = lane; i < n; i += 32) {
-      const uint64_t j = j0 + i;
-      const float sc = bf16_bits_to_float(D.scales[div_by_magic(j, D.row_magic)]);
-      D.out[j] = dequant1<FMT>(single_sym, sc);
+    if (!__all_sync(0xFFFFFFFFu, nwords == 0 && x == kRansL)) status |= EQ_DEV_CORRUPT_STATE;
+    for (uint32_t r = 0; r < rounds; ++r) {
+      const uint32_t run = r * S + s;
+      if (run >= runs) continue;
+      for (uint32_t i = 0; i < uint32_t(G); ++i) {
+        const uint64_t j = j0 + uint64_t(run) * G + i;
+        if (j >= j0 + n) break;
+        D.out[j] = dequant1<FMT>(single_sym, bf16_bits_to_float(D.scales[div_by_magic(j, D.row_magic)]));
+      }
     }
     return status;
   }
 
-  // word ring for this chunk
-  const unsigned char *g = reinterpret_cast<const unsigned char *>(D.words + w0);
-  R.A = reinterpret_cast<const unsigned char *>(reinterpret_cast<uintptr_t>(g) & ~uintptr_t(15));
-  R.off0 = uint32_t(g - R.A);
-  R.span = (R.off0 + 2 * nwords + 15u) & ~15u;
-  R.nseg = (R.span + kSegBytes - 1) / kSegBytes;
-  R.issued = 0;
-  R.ready = 0;
-  while (R.issued < min(R.nseg, kNumSeg)) R.issue(lane);
-
+  R.start(D.words, w0, nwords, lane);
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (flags & (kRansFlagNaN7F | kRansFlagNaNFF));
   const uint32_t lt = lanemask_lt();
-  const uint32_t runs = (n + G - 1) / G;
-  const uint32_t rounds = (runs + S - 1) / S;
-  uint32_t ptr = 0;
-
+  // rounds in which all 32 lanes of this group hold a run
+  const uint32_t full = runs >= 32 * g + 32 ? (runs - 32 * g - 32) / S + 1 : 0;
+  uint32_t q = R.off0;
   for (uint32_t r = 0; r < rounds; ++r) {
-    bool act[K];
-#pragma unroll
-    for (int k = 0; k < K; ++k) act[k] = r * S + lane + 32 * k < runs;
-    uint32_t sym[K][(G + 3) / 4];
-#pragma unroll
-    for (int k = 0; k < K; ++k)
-#pragma unroll
-      for (int i = 0; i < (G + 3) / 4; ++i) sym[k][i] = 0;
-
-#pragma unroll
-    for (int p = 0; p < G; ++p) {
-      // the words this step can read must have landed
-      if (R.nseg) {
-        const uint32_t last = min(R.nseg - 1, (R.off0 + 2 * (ptr + S) - 1) / kSegBytes);
-        if (!R.wait_upto(last)) {
-          status |= EQ_DEV_TIMEOUT;
-          goto drain;
-        }
-      }
-      uint32_t mask[K];
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        const uint32_t e = lut[x[k] & (kRansSlots - 1)];
-        const uint32_t nx = ((e >> 12) & 0xFFFu) * (x[k] >> kRansProbBits) + (e & 0xFFFu);
-        if (act[k]) x[k] = nx;
-        // symbol byte -> byte p % 4 of sym[k][p / 4]
-        sym[k][p >> 2] = __byte_perm(sym[k][p >> 2], e, (0x3210u & ~(0xFu << (4 * (p & 3)))) |
-                                                            (0x7u << (4 * (p & 3))));
-        mask[k] = __ballot_sync(0xFFFFFFFFu, act[k] && x[k] < kRansL);
-      }
-      uint32_t base = ptr;
-#pragma unroll
-      for (int k = 0; k < K; ++k) {
-        if ((mask[k] >> lane) & 1u) x[k] = (x[k] << 16) | R.word(base + __popc(mask[k] & lt));
-        base += __popc(mask[k]);
-      }
-      ptr = base;
-      if (ptr > nwords) {
-        status |= EQ_DEV_OVERRUN;
-        goto drain;
-      }
-      R.refill(ptr, lane);
-
-      if constexpr (G == 1) {
-#pragma unroll
-        for (int k = 0; k < K; ++k)
-          if (act[k]) {
-            const uint64_t j = j0 + uint64_t(r * S + lane + 32 * k);
-            const float sc = bf16_bits_to_float(D.scales[div_by_magic(j, D.row_magic)]);
-            D.out[j] = dequant1<FMT>(sym[k][0], sc);
-          }
-      }
-    }
-    if constexpr (G == 8) {
-#pragma unroll
-      for (int k = 0; k < K; ++k)
-        if (act[k]) {
-          const uint64_t j = j0 + uint64_t(r * S + lane + 32 * k) * 8;
-          const float sc = bf16_bits_to_float(D.scales[div_by_magic(j, D.row_magic)]);
-          const uint2 a = dequant4<FMT>(sym[k][0], sc, nan_codes);
-          const uint2 b = dequant4<FMT>(sym[k][1], sc, nan_codes);
-          *reinterpret_cast<uint4 *>(D.out + j) = make_uint4(a.x, a.y, b.x, b.y);
-        }
-    }
-  }
-  {
-    bool ok = ptr == nwords;
-#pragma unroll
-    for (int k = 0; k < K; ++k) ok &= x[k] == kRansL;
-    if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
-  }
-drain:
-  // every copy handed to the engine must land before the ring is reused or the CTA exits
-  while (R.ready < R.issued) {
-    if (!mbar_wait_bounded(&R.bar[R.ready % kNumSeg], (R.ready / kNumSeg) & 1u)) {
+    if (!R.wait_below(q + 2 * kRoundWords)) {
       status |= EQ_DEV_TIMEOUT;
       break;
     }
-    ++R.ready;
+    const uint32_t run = r * S + s;
+    const uint64_t jrun = j0 + uint64_t(run) * G;
+    if (r < full) decode_round<true, G, FMT>(D, x, true, lut, R, q, lt, jrun, nan_codes);
+    else decode_round<false, G, FMT>(D, x, run < runs, lut, R, q, lt, jrun, nan_codes);
+    if (q - R.off0 > 2 * nwords) {
+      status |= EQ_DEV_OVERRUN;
+      break;
+    }
+    R.refill(q, lane);
   }
+  if (!status && !__all_sync(0xFFFFFFFFu, q - R.off0 == 2 * nwords && x == kRansL))
+    status |= EQ_DEV_CORRUPT_STATE;
+  // every copy handed to the engine must land before the ring is reused or the CTA exits
+  status |= R.drain();
   return status;
 }
 
-template <int K, int G, int FMT>
-__global__ void __launch_bounds__(256) rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
+template <int G, int FMT>
+__global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
   unsigned char *rings = smem + kRansSlots * 4;
@@ -251,19 +153,14 @@ __global__ void __launch_bounds__(256) rans_decode_kernel(const __grid_constant_
   for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
     reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
   WordRing R;
-  R.buf = rings + warp * kRingBytes;
-  R.bar = bars + warp * kNumSeg;
-  if (lane == 0) {
-    for (uint32_t s = 0; s < kNumSeg; ++s) mbar_init(&R.bar[s], 1);
-    fence_mbar_init();
-  }
+  ring_init(R, rings, bars, warp, lane);
   __syncthreads();
 
-  const uint64_t chunk = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
-  if (chunk >= D.num_chunks) return;
+  const uint64_t unit = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
+  if (unit >= D.units) return;
   uint32_t status = 0;
   if (hdr.magic != kRansMagic) status = EQ_DEV_CORRUPT_STATE;
-  else status = decode_chunk<K, G, FMT>(D, lut, hdr.flags, hdr.single_sym, R, chunk, lane);
+  else status = decode_group<G, FMT>(D, lut, hdr.flags, hdr.single_sym, R, unit, lane);
   if (lane == 0) report(P.status, status);
 }
 
@@ -272,26 +169,11 @@ __global__ void __launch_bounds__(256) rans_decode_kernel(const __grid_constant_
 // ------------------------------------------------------------------------------------------------
 using KernelFn = void (*)(RansDecodeParams);
 
-template <int K, int G, int FMT>
-static KernelFn kernel_for() {
-  return rans_decode_kernel<K, G, FMT>;
-}
-
-template <int G, int FMT>
-static KernelFn pick_k(uint32_t K) {
-  switch (K) {
-    case 1: return kernel_for<1, G, FMT>();
-    case 2: return kernel_for<2, G, FMT>();
-    case 4: return kernel_for<4, G, FMT>();
-    case 8: return kernel_for<8, G, FMT>();
-  }
-  return nullptr;
-}
-
-static KernelFn pick_kernel(uint32_t symfmt, uint32_t streams, uint32_t run) {
-  const uint32_t K = streams / 32;
-  if (run == 8) return symfmt == EQ_SYM_E4M3 ? pick_k<8, EQ_SYM_E4M3>(K) : pick_k<8, EQ_SYM_INT8>(K);
-  if (run == 1) return symfmt == EQ_SYM_E4M3 ? pick_k<1, EQ_SYM_E4M3>(K) : pick_k<1, EQ_SYM_INT8>(K);
+static KernelFn pick_kernel(uint32_t symfmt, uint32_t run) {
+  if (run == 8)
+    return symfmt == EQ_SYM_E4M3 ? rans_decode_kernel<8, EQ_SYM_E4M3> : rans_decode_kernel<8, EQ_SYM_INT8>;
+  if (run == 1)
+    return symfmt == EQ_SYM_E4M3 ? rans_decode_kernel<1, EQ_SYM_E4M3> : rans_decode_kernel<1, EQ_SYM_INT8>;
   return nullptr;
 }
 
@@ -301,8 +183,7 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   if (t.symfmt != EQ_SYM_E4M3 && t.symfmt != EQ_SYM_INT8) return EQ_ERR_ARG;
   if (t.prob_bits != kRansProbBits) return EQ_ERR_UNSUPPORTED;
   if (t.run != 1 && t.run != 8) return EQ_ERR_UNSUPPORTED;
-  const uint32_t K = t.streams / 32;
-  if (t.streams % 32 || (K != 1 && K != 2 && K != 4 && K != 8)) return EQ_ERR_UNSUPPORTED;
+  if (t.streams == 0 || t.streams % 32 || t.streams > 1024) return EQ_ERR_UNSUPPORTED;
   const uint64_t numel = uint64_t(t.rows) * t.cols;
   if (numel >= (1ull << 40)) return EQ_ERR_UNSUPPORTED;
   if (numel == 0) return t.num_chunks == 0 ? EQ_OK : EQ_ERR_ARG;
@@ -316,26 +197,26 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   return EQ_OK;
 }
 
-static bool g_attr_set[64][2][2][9];
+static bool g_attr_set[64][2][2];
 
 static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
                               uint16_t *const *d_out, uint32_t *d_status, cudaStream_t st) {
   const eq_rans_tensor &t0 = ts[idx[0]];
-  KernelFn fn = pick_kernel(t0.symfmt, t0.streams, t0.run);
+  KernelFn fn = pick_kernel(t0.symfmt, t0.run);
   if (!fn) return EQ_ERR_UNSUPPORTED;
-  uint64_t total_chunks = 0;
-  for (uint32_t i : idx) total_chunks += ts[i].num_chunks;
-  // warps (= chunks) per CTA: enough CTAs to spread over every SM a few times
+  uint64_t total_units = 0;
+  for (uint32_t i : idx) total_units += ts[i].num_chunks * (ts[i].streams / 32);
+  // warps (= groups) per CTA: 16 when the work covers every SM several times over
   const uint64_t sms = uint64_t(device_sm_count());
-  uint32_t warps = 8;
-  while (warps > 1 && (total_chunks + warps - 1) / warps < 3 * sms) warps >>= 1;
-  const size_t smem = decode_smem_bytes(warps);
+  uint32_t warps = 16;
+  while (warps > 1 && (total_units + warps - 1) / warps < 4 * sms) warps >>= 1;
+  const size_t smem = rans_smem_bytes(warps);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8][t0.streams / 32];
+  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8];
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(decode_smem_bytes(8)));
+                                         int(rans_smem_bytes(16)));
     if (e != cudaSuccess) return EQ_ERR_CUDA;
     attr = true;
   }
@@ -357,13 +238,13 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
       D.table = static_cast<const uint32_t *>(t.tables);
       D.out = d_out[idx[q]];
       D.numel = uint64_t(t.rows) * t.cols;
-      D.num_chunks = t.num_chunks;
+      D.groups = t.streams / 32;
+      D.units = t.num_chunks * D.groups;
       D.row_magic = div_magic(t.cols);
-      D.cols = t.cols;
       D.chunk_symbols = t.chunk_symbols;
       D.cta_begin = uint32_t(ctas);
       D.pad = 0;
-      ctas += (t.num_chunks + warps - 1) / warps;
+      ctas += (D.units + warps - 1) / warps;
     }
     if (P.n == 0) continue;
     if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
@@ -389,20 +270,12 @@ extern "C" eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uin
     if (ts[i].num_chunks && (!d_out[i] || !aligned(d_out[i], ts[i].run == 8 ? 16 : 2)))
       return EQ_ERR_ARG;
   }
-  // group by the compile-time parameters of the kernel
-  std::vector<std::vector<uint32_t>> groups;
-  std::vector<uint32_t> keys;
-  for (uint32_t i = 0; i < n_tensors; ++i) {
-    const uint32_t key = ts[i].symfmt * 10000 + ts[i].streams * 10 + ts[i].run;
-    auto it = std::find(keys.begin(), keys.end(), key);
-    if (it == keys.end()) {
-      keys.push_back(key);
-      groups.emplace_back();
-      it = keys.end() - 1;
-    }
-    groups[it - keys.begin()].push_back(i);
-  }
+  // one launch per kernel variant (symbol format x run length)
+  std::vector<std::vector<uint32_t>> groups(4);
+  for (uint32_t i = 0; i < n_tensors; ++i)
+    groups[(ts[i].symfmt - 1) * 2 + (ts[i].run == 8)].push_back(i);
   for (auto &g : groups) {
+    if (g.empty()) continue;
     eq_status s = launch_group(ts, g, d_out, d_status, static_cast<cudaStream_t>(stream));
     if (s != EQ_OK) return s;
   }

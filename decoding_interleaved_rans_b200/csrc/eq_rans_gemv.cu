@@ -1,0 +1,228 @@
+// eq_decode_gemv: y = W x with W decoded from its interleaved-rANS stream on chip (sm_100a).
+//
+// The pages name fused decompression + compute kernels as the next step after block-wise
+// decompression ("Float8@2bits" summary, closing section; DFloat11 page, forum section: a GEMM that
+// decompresses each tile before the arithmetic).  Here the decoded weights never reach memory:
+//   * one warp decodes one chunk of whole rows with the same core as eq_decode (slot table in
+//     shared memory, word ring fed by bulk copies, ballot/popcount renormalisation);
+//   * each run of 8 symbols is dequantised exactly as eq_decode would write it (bf16 of
+//     value * row scale), so y is the product of the very weights eq_decode returns;
+//   * the lane multiplies its 8 weights by the matching 8 activations of every batch row
+//     (16-byte loads of x, which stays in L1/L2) and accumulates in fp32;
+//   * at the end of each weight row the warp reduces its partial sums with shuffles and writes
+//     y[b][row] once.  The reduction order is fixed, so results are reproducible.
+// The chunk has one group of 32 streams (streams == 32), so its partial sums never leave the warp.
+// With chunks of several rows, a round (32 * 8 symbols) must not straddle a row, so cols must be a
+// multiple of 256.
+#include <algorithm>
+
+#include "eq_dequant.cuh"
+#include "eq_rans_core.cuh"
+
+namespace eq {
+
+eq_status validate_rans_tensor(const eq_rans_tensor &t);  // eq_rans_decode.cu
+
+struct GemvParams {
+  const uint32_t *states;
+  const uint64_t *word_off;
+  const uint16_t *words;
+  const uint16_t *scales;
+  const uint32_t *table;
+  const uint16_t *x;
+  float *y;
+  uint32_t *status;
+  uint64_t numel;
+  uint64_t num_chunks;
+  uint32_t rows, cols, chunk_symbols, rows_per_chunk, rounds_per_row, batch, warps;
+};
+
+__device__ __forceinline__ float lo_bf16(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// acc[b] += sum_i w[i] * x[b][col + i] over one run of 8 weights (packed bf16 pairs)
+template <int BMAX>
+__device__ __forceinline__ void fma_run(float (&acc)[BMAX], uint2 wa, uint2 wb, const uint16_t *x,
+                                        uint32_t cols, uint32_t col, uint32_t batch) {
+  const float wv[8] = {lo_bf16(wa.x), hi_bf16(wa.x), lo_bf16(wa.y), hi_bf16(wa.y),
+                       lo_bf16(wb.x), hi_bf16(wb.x), lo_bf16(wb.y), hi_bf16(wb.y)};
+#pragma unroll
+  for (int b = 0; b < BMAX; ++b) {
+    if (b < int(batch)) {
+      const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + size_t(b) * cols + col));
+      float a = acc[b];
+      a = fmaf(wv[0], lo_bf16(xv.x), a);
+      a = fmaf(wv[1], hi_bf16(xv.x), a);
+      a = fmaf(wv[2], lo_bf16(xv.y), a);
+      a = fmaf(wv[3], hi_bf16(xv.y), a);
+      a = fmaf(wv[4], lo_bf16(xv.z), a);
+      a = fmaf(wv[5], hi_bf16(xv.z), a);
+      a = fmaf(wv[6], lo_bf16(xv.w), a);
+      a = fmaf(wv[7], hi_bf16(xv.w), a);
+      acc[b] = a;
+    }
+  }
+}
+
+// One warp = one chunk of whole rows, 32 streams (one per lane), run length 8.
+template <int FMT, int BMAX>
+__global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ GemvParams P) {
+  constexpr uint32_t S = 32;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
+  unsigned char *rings = smem + kRansSlots * 4;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * kRingBytes);
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
+  const uint4 *src = reinterpret_cast<const uint4 *>(P.table + sizeof(RansTableHeader) / 4);
+  for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
+    reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+  WordRing R;
+  ring_init(R, rings, bars, warp, lane);
+  __syncthreads();
+
+  const uint64_t chunk = uint64_t(blockIdx.x) * P.warps + warp;
+  if (chunk >= P.num_chunks) return;
+  uint32_t status = hdr.magic == kRansMagic ? 0u : EQ_DEV_CORRUPT_STATE;
+  const bool single = hdr.flags & kRansFlagSingle;
+  const bool nan_codes = (FMT == EQ_SYM_E4M3) && (hdr.flags & (kRansFlagNaN7F | kRansFlagNaNFF));
+  const uint64_t j0 = chunk * uint64_t(P.chunk_symbols);
+  const uint32_t n = uint32_t(P.numel - j0 < P.chunk_symbols ? P.numel - j0 : P.chunk_symbols);
+  const uint64_t w0 = P.word_off[chunk], w1 = P.word_off[chunk + 1];
+  if (w1 < w0 || w1 - w0 >= (1ull << 30)) status |= EQ_DEV_OVERRUN;
+  uint32_t x = P.states[chunk * S + lane];
+  if (status) {
+    if (lane == 0) report(P.status, status);
+    return;
+  }
+  const uint32_t nwords = uint32_t(w1 - w0);
+  if (!single) R.start(P.words, w0, nwords, lane);
+
+  const uint32_t lt = lanemask_lt();
+  const uint32_t runs = n / 8;
+  const uint32_t rounds = (runs + S - 1) / S;
+  const uint32_t row0 = uint32_t(chunk * P.rows_per_chunk);
+  const uint32_t batch = P.batch;
+  float acc[BMAX];
+#pragma unroll
+  for (int b = 0; b < BMAX; ++b) acc[b] = 0.0f;
+  uint32_t row_local = 0;
+  float sc = bf16_bits_to_float(P.scales[row0]);
+  uint32_t q = R.off0;
+
+  for (uint32_t r = 0; r < rounds; ++r) {
+    const bool act = r * S + lane < runs;
+    uint32_t sym[2] = {0u, 0u};
+    if (single) {
+      sym[0] = sym[1] = hdr.single_sym * 0x01010101u;
+    } else {
+      if (!R.wait_below(q + 2 * kRoundWords)) {
+        status |= EQ_DEV_TIMEOUT;
+        break;
+      }
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const uint32_t e = rans_step<false>(x, act, lut, R, q, lt);
+        sym[p >> 2] = put_sym(sym[p >> 2], e, p & 3);
+      }
+      if (q - R.off0 > 2 * nwords) {
+        status |= EQ_DEV_OVERRUN;
+        break;
+      }
+      R.refill(q, lane);
+    }
+    if (act) {  // the weights exactly as eq_decode writes them, times the activations
+      const uint32_t col = (r * S + lane) * 8 - row_local * P.cols;
+      fma_run<BMAX>(acc, dequant4<FMT>(sym[0], sc, nan_codes), dequant4<FMT>(sym[1], sc, nan_codes),
+                    P.x, P.cols, col, batch);
+    }
+    // end of a weight row: reduce across the warp and write y
+    const bool row_end = (r + 1 == rounds) || (P.rows_per_chunk > 1 && (r + 1) % P.rounds_per_row == 0);
+    if (row_end) {
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) {
+        float v = acc[b];
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, d);
+        if (lane == 0 && b < int(batch)) P.y[size_t(b) * P.rows + row0 + row_local] = v;
+        acc[b] = 0.0f;
+      }
+      ++row_local;
+      if (row_local < P.rows_per_chunk && r + 1 < rounds)
+        sc = bf16_bits_to_float(P.scales[row0 + row_local]);
+    }
+  }
+  if (!status) {
+    const bool ok = single ? (nwords == 0 && x == kRansL) : (q - R.off0 == 2 * nwords && x == kRansL);
+    if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
+  }
+  if (!single) status |= R.drain();
+  if (lane == 0) report(P.status, status);
+}
+
+using GemvFn = void (*)(GemvParams);
+
+template <int FMT>
+static GemvFn pick_b(uint32_t batch) {
+  if (batch <= 1) return rans_gemv_kernel<FMT, 1>;
+  if (batch <= 2) return rans_gemv_kernel<FMT, 2>;
+  if (batch <= 4) return rans_gemv_kernel<FMT, 4>;
+  if (batch <= 8) return rans_gemv_kernel<FMT, 8>;
+  return rans_gemv_kernel<FMT, 16>;
+}
+
+static bool g_gemv_attr[64][2][5];
+
+}  // namespace eq
+
+using namespace eq;
+
+extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x, uint32_t batch,
+                                    float *d_y, uint32_t *d_status, void *stream) {
+  if (!t || !d_status) return EQ_ERR_ARG;
+  eq_status s = validate_rans_tensor(*t);
+  if (s != EQ_OK) return s;
+  if (batch < 1 || batch > 16) return EQ_ERR_ARG;
+  if (t->rows == 0 || t->cols == 0) return EQ_OK;
+  if (!d_x || !d_y || !aligned(d_x, 16) || !aligned(d_y, 4)) return EQ_ERR_ARG;
+  if (t->run != 8 || t->streams != 32 || t->chunk_symbols % t->cols) return EQ_ERR_UNSUPPORTED;
+  const uint32_t rpc = t->chunk_symbols / t->cols;
+  if (rpc > 1 && t->cols % (t->streams * 8)) return EQ_ERR_UNSUPPORTED;
+  GemvFn fn = t->symfmt == EQ_SYM_E4M3 ? pick_b<EQ_SYM_E4M3>(batch) : pick_b<EQ_SYM_INT8>(batch);
+  const uint64_t sms = uint64_t(device_sm_count());
+  uint32_t warps = 16;
+  while (warps > 1 && (t->num_chunks + warps - 1) / warps < 4 * sms) warps >>= 1;
+  const uint64_t ctas = (t->num_chunks + warps - 1) / warps;
+  if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
+  const int bi = batch <= 1 ? 0 : batch <= 2 ? 1 : batch <= 4 ? 2 : batch <= 8 ? 3 : 4;
+  bool &attr = g_gemv_attr[dev][t->symfmt - 1][bi];
+  if (!attr) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(rans_smem_bytes(16))) != cudaSuccess)
+      return EQ_ERR_CUDA;
+    attr = true;
+  }
+  GemvParams P;
+  P.states = t->states;
+  P.word_off = t->word_off;
+  P.words = t->words;
+  P.scales = t->scales;
+  P.table = static_cast<const uint32_t *>(t->tables);
+  P.x = d_x;
+  P.y = d_y;
+  P.status = d_status;
+  P.numel = uint64_t(t->rows) * t->cols;
+  P.num_chunks = t->num_chunks;
+  P.rows = t->rows;
+  P.cols = t->cols;
+  P.chunk_symbols = t->chunk_symbols;
+  P.rows_per_chunk = rpc;
+  P.rounds_per_row = rpc > 1 ? t->cols / (t->streams * 8) : 0;
+  P.batch = batch;
+  P.warps = warps;
+  fn<<<uint32_t(ctas), 32 * warps, rans_smem_bytes(warps), static_cast<cudaStream_t>(stream)>>>(P);
+  return cuda_status(cudaGetLastError());
+}

@@ -66,10 +66,12 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
  *   shorter); chunk c is coded on its own by `streams` interleaved rANS states.  Inside a chunk,
  *   symbol j belongs to run r = j / run, stream r % streams, round r / streams, position j % run;
  *   the decoder visits (round, position, stream) in increasing order and skips streams that hold
- *   no symbol at that step.  Decoding symbol s from x: slot = x mod M, s is the symbol with
- *   cum[s] <= slot < cum[s] + freq[s], x = freq[s] * (x / M) + slot - cum[s]; then, if x < 2^16,
- *   x = x * 2^16 + the chunk's next word.  A well-formed chunk ends with every state at 2^16 and
- *   every word read.
+ *   no symbol at that step.  The streams form groups of 32 (group g = streams 32g .. 32g + 31);
+ *   each group reads its own word substream, so the groups of a chunk decode independently.
+ *   Decoding symbol s from x: slot = x mod M, s is the symbol with cum[s] <= slot < cum[s] +
+ *   freq[s], x = freq[s] * (x / M) + slot - cum[s]; then, if x < 2^16, x = x * 2^16 + the next
+ *   word of the stream's group.  A well-formed chunk ends with every state at 2^16 and every
+ *   word read.
  *   Dequantisation: out = bf16_rne( value(s) * scale[row] ), value(s) being the E4M3 value of the
  *   byte (NaN codes 0x7F/0xFF give the bf16 quiet NaN 0x7FC0 / 0xFFC0) or the byte read as int8.
  */
@@ -79,13 +81,14 @@ typedef struct {
   uint32_t rows, cols;    /* W is rows x cols, row-major; rows*cols < 2^40                     */
   uint32_t prob_bits;     /* 12                                                                */
   uint32_t chunk_symbols; /* symbols per chunk (>= 1); a multiple of `run`                     */
-  uint32_t streams;       /* interleaved states per chunk: 32, 64, 96 ... 256                  */
+  uint32_t streams;       /* interleaved states per chunk: a multiple of 32, at most 1024      */
   uint32_t run;           /* consecutive symbols per stream visit: 1 or 8; 8 needs cols % 8 == 0 */
   uint64_t num_chunks;    /* ceil(rows * cols / chunk_symbols)                                 */
   const uint32_t *states; /* [num_chunks][streams] final encoder states                         */
-  const uint64_t *word_off; /* [num_chunks + 1] start of each chunk's words, in words           */
-  const uint16_t *words;  /* all chunks' words, decoder order; allocation padded with zeros to a
-                             multiple of 8 words (16 bytes); base 16-byte aligned               */
+  const uint64_t *word_off; /* [num_chunks * streams / 32 + 1]: substream (c, g) is words
+                             [word_off[c * streams / 32 + g], word_off[... + 1])                */
+  const uint16_t *words;  /* all substreams, chunk-major, decoder order; allocation padded with
+                             zeros to a multiple of 8 words (16 bytes); base 16-byte aligned    */
   const uint16_t *scales; /* [rows] bf16 per-output-channel scales                              */
   const void *tables;     /* eq_table_bytes(EQ_TABLE_RANS) bytes from eq_build_tables(RANS);
                              16-byte aligned                                                    */
@@ -150,11 +153,13 @@ eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uint16_t *cons
 /*
  * y[b][r] = sum_c W[r][c] * x[b][c] for b < batch, with W decoded from its rANS stream on chip
  * and never written to memory ("Float8@2bits" summary, closing section: fused decompression
- * kernels are the next step; the decoded values are consumed where they are produced).
- * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].
- * Requires chunk_symbols to be a multiple of cols (every chunk holds whole rows) and run == 8.
- * batch 1..16; batch >= 8 runs the product on the tensor cores.  The fp32 result is within a
- * relative L2 error of 1e-3 of the exact product of the decoded bf16 weights.
+ * kernels are the next step; the decoded values are consumed where they are produced).  W is
+ * taken exactly as eq_decode would return it (bf16 of value * scale), products and sums in fp32.
+ * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].  batch 1..16.
+ * Requires run == 8, streams == 32 (one warp owns a chunk, so its sums never leave the warp)
+ * and whole rows per chunk (chunk_symbols a multiple of cols); a chunk of several rows also needs
+ * cols % 256 == 0, so that one decode round never straddles two rows.  Otherwise
+ * EQ_ERR_UNSUPPORTED.
  */
 eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x, uint32_t batch, float *d_y,
                          uint32_t *d_status, void *stream);

@@ -41,8 +41,9 @@ eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t prob_bits,
 /*
  * Interleaved-rANS encoding of a symbol matrix sym[rows][cols] in the format of eq_rans_tensor.
  * chunk_symbols = 0 means one row per chunk.  states: [num_chunks * streams]; word_off:
- * [num_chunks + 1].  The words are returned in a buffer the library allocates (*words, *n_words
- * words, zero-padded to a multiple of 8); release it with eq_free_host.
+ * [num_chunks * ceil(streams / 32) + 1] (one word substream per chunk and group of 32 streams).
+ * The words are returned in a buffer the library allocates (*words, *n_words words, zero-padded
+ * to a multiple of 8); release it with eq_free_host.
  */
 eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint32_t cols,
                               const uint32_t *freqs, uint32_t chunk_symbols, uint32_t streams,

@@ -64,8 +64,9 @@ def lib() -> C.CDLL:
             "orc_dequant_one": (C.c_uint16, [C.c_uint8, C.c_uint16, i32]),
             "orc_dequant": (None, [p, p, i64, i64, i32, p]),
             "orc_rans_normalize": (i32, [p, u32, p]),
-            "orc_rans_encode_chunk": (i64, [p, i64, p, u32, u32, u32, p, p]),
-            "orc_rans_decode_chunk": (i32, [p, i64, p, i64, p, u32, u32, u32, p]),
+            "orc_rans_groups": (i64, [u32]),
+            "orc_rans_encode_chunk": (i64, [p, i64, p, u32, u32, u32, p, p, p]),
+            "orc_rans_decode_chunk": (i32, [p, p, p, i64, p, u32, u32, u32, p]),
             "orc_rans_decode_bf16": (i32, [p, p, p, p, p, i64, i64, i32, u32, i64, u32, u32,
                                            i64, i64, p]),
             "orc_gemv_f64": (None, [p, p, i64, i64, i64, p]),
@@ -177,11 +178,17 @@ def entropy_bits(sym: np.ndarray) -> float:
 # rANS containers
 # ----------------------------------------------------------------------------------------------
 
+def rans_groups(streams: int) -> int:
+    """Streams form groups of 32, each with its own word substream."""
+    return (streams + 31) // 32
+
+
 @dataclass
 class RansTensor:
     """One interleaved-rANS-coded weight (format of the library's eq_rans_tensor).
 
-    words are padded with zeros to a multiple of 8 (16 bytes)."""
+    word_off has num_chunks * groups + 1 entries (one substream per chunk and group of 32
+    streams); words are padded with zeros to a multiple of 8 (16 bytes)."""
     rows: int
     cols: int
     symfmt: int
@@ -191,7 +198,7 @@ class RansTensor:
     run: int
     freqs: np.ndarray     # uint32[256], sums to 2^prob_bits
     states: np.ndarray    # uint32[num_chunks * streams]
-    word_off: np.ndarray  # uint64[num_chunks + 1]
+    word_off: np.ndarray  # uint64[num_chunks * groups + 1]
     words: np.ndarray     # uint16
     scales: np.ndarray    # uint16[rows] (bf16 bits)
 
@@ -200,8 +207,12 @@ class RansTensor:
         return self.rows * self.cols
 
     @property
+    def groups(self) -> int:
+        return rans_groups(self.streams)
+
+    @property
     def num_chunks(self) -> int:
-        return len(self.word_off) - 1
+        return (len(self.word_off) - 1) // self.groups
 
     @property
     def payload_bytes(self) -> int:
@@ -226,27 +237,36 @@ def rans_freqs(sym: np.ndarray, prob_bits: int = PROB_BITS) -> np.ndarray:
 
 def rans_encode_chunk(sym: np.ndarray, freqs: np.ndarray, streams: int, run: int,
                       prob_bits: int = PROB_BITS):
-    """Encode one chunk; returns (states uint32[S], words uint16 in decoder order)."""
+    """Encode one chunk; returns (states uint32[S], words uint16 (group substreams one after the
+    other, decoder order), per-group word counts int64[ceil(S / 32)])."""
     sym = np.ascontiguousarray(sym, dtype=np.uint8).ravel()
     freqs = np.ascontiguousarray(freqs, dtype=np.uint32)
     states = np.empty(streams, dtype=np.uint32)
     words = np.empty(max(1, sym.size), dtype=np.uint16)
-    nw = lib().orc_rans_encode_chunk(_p(sym), sym.size, _p(freqs), prob_bits, streams, run,
-                                     _p(states), _p(words))
+    counts = np.zeros(rans_groups(streams), dtype=np.int64)
+    nw = lib().orc_rans_encode_chunk(_p(sym) if sym.size else _p(np.zeros(1, np.uint8)),
+                                     sym.size, _p(freqs), prob_bits, streams, run, _p(states),
+                                     _p(words), _p(counts))
     if nw < 0:
         raise ValueError(ERRORS.get(nw, nw))
-    return states, words[:nw].copy()
+    return states, words[:nw].copy(), counts
 
 
 def rans_decode_chunk(words: np.ndarray, states: np.ndarray, n: int, freqs: np.ndarray,
-                      streams: int, run: int, prob_bits: int = PROB_BITS):
-    """Decode one chunk; returns (status, symbols uint8[n])."""
+                      streams: int, run: int, counts=None, prob_bits: int = PROB_BITS):
+    """Decode one chunk; returns (status, symbols uint8[n]).  counts: words per group (default:
+    all words belong to the one group)."""
     words = np.ascontiguousarray(words, dtype=np.uint16)
     states = np.ascontiguousarray(states, dtype=np.uint32)
     freqs = np.ascontiguousarray(freqs, dtype=np.uint32)
+    if counts is None:
+        assert rans_groups(streams) == 1
+        counts = [words.size]
+    goff = np.zeros(len(counts) + 1, dtype=np.int64)
+    np.cumsum(np.asarray(counts, dtype=np.int64), out=goff[1:])
     out = np.zeros(max(1, n), dtype=np.uint8)
     wp = _p(words) if words.size else _p(np.zeros(1, np.uint16))
-    rc = lib().orc_rans_decode_chunk(wp, words.size, _p(states), n, _p(freqs), prob_bits,
+    rc = lib().orc_rans_decode_chunk(wp, _p(goff), _p(states), n, _p(freqs), prob_bits,
                                      streams, run, _p(out))
     return rc, out[:n]
 
@@ -263,14 +283,17 @@ def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols:
     if freqs is None:
         freqs = rans_freqs(flat, prob_bits)
     nchunks = (N + chunk - 1) // chunk
+    ng = rans_groups(streams)
     states = np.empty(nchunks * streams, dtype=np.uint32)
     pieces = [None] * nchunks
+    counts = np.zeros((nchunks, ng), dtype=np.uint64)
 
     def one(c):
         j0 = c * chunk
-        st, w = rans_encode_chunk(flat[j0:j0 + chunk], freqs, streams, run, prob_bits)
+        st, w, cnt = rans_encode_chunk(flat[j0:j0 + chunk], freqs, streams, run, prob_bits)
         states[c * streams:(c + 1) * streams] = st
         pieces[c] = w
+        counts[c] = cnt
 
     if nchunks <= 4 or N < (1 << 20):
         for c in range(nchunks):
@@ -278,13 +301,12 @@ def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols:
     else:
         with ThreadPoolExecutor(_threads(threads)) as ex:
             list(ex.map(one, range(nchunks)))
-    counts = np.array([p.size for p in pieces], dtype=np.uint64)
-    word_off = np.zeros(nchunks + 1, dtype=np.uint64)
-    np.cumsum(counts, out=word_off[1:])
+    word_off = np.zeros(nchunks * ng + 1, dtype=np.uint64)
+    np.cumsum(counts.ravel(), out=word_off[1:])
     total = int(word_off[-1])
     words = np.zeros(((total + 7) // 8) * 8 if total else 8, dtype=np.uint16)
-    if nchunks:
-        words[:total] = np.concatenate(pieces) if total else []
+    if nchunks and total:
+        words[:total] = np.concatenate(pieces)
     return RansTensor(rows, cols, symfmt, prob_bits, chunk_symbols, streams, run,
                       np.ascontiguousarray(freqs, dtype=np.uint32), states, word_off, words,
                       np.ascontiguousarray(scales, dtype=np.uint16))

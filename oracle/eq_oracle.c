@@ -227,16 +227,21 @@ int orc_rans_normalize(const uint64_t *counts, uint32_t prob_bits, uint32_t *fre
  * Layout of one chunk of n symbols (j = 0..n-1, in row-major order of the weight):
  *   run r = j / G, stream = r mod S, round = r / S, position p = j mod G;
  *   decode steps go in order (round, p, stream); a stream with no symbol at a step is skipped.
+ * Streams form groups of 32 (group g = streams 32g .. 32g+31, the last group may be smaller);
+ *   every group has its own word substream, holding the words its streams read, in the order
+ *   they read them.  Groups never share words, so a chunk's groups decode independently.
  * Encoder: all S states start at L = 2^16; steps are taken in exactly the reverse order.  Before
  *   coding s with frequency f and cumulative frequency c, if x >= f * 2^(32 - prob_bits) the low 16
- *   bits of x are emitted and x >>= 16; then x = floor(x / f) * M + (x mod f) + c.
- *   The emitted words, reversed, are the chunk's words in decoder-forward order.
+ *   bits of x are emitted onto its group's stack and x >>= 16; then x = floor(x / f) * M +
+ *   (x mod f) + c.  Each group's stack, reversed, is its substream in decoder-forward order; the
+ *   chunk's words are the substreams of groups 0, 1, ... one after the other.
  * Decoder: slot = x mod M; s is the symbol with c_s <= slot < c_s + f_s;
- *   x = f_s * floor(x / M) + slot - c_s; if x < L then x = x * 2^16 + next word.
- *   At the end every x is L again and every word has been read.
+ *   x = f_s * floor(x / M) + slot - c_s; if x < L then x = x * 2^16 + next word of its group.
+ *   At the end every x is L again and every group has read all of its words.
  * ========================================================================================== */
 
 #define RANS_L 65536u
+#define RANS_GROUP 32
 
 static void cum_of(const uint32_t *freqs, uint32_t *cum) {
   uint32_t c = 0;
@@ -246,16 +251,23 @@ static void cum_of(const uint32_t *freqs, uint32_t *cum) {
   }
 }
 
-/* Returns the number of words written to words_out (capacity must be >= n), or < 0. */
+int64_t orc_rans_groups(uint32_t S) { return ((int64_t)S + RANS_GROUP - 1) / RANS_GROUP; }
+
+/* Returns the number of words written to words_out (capacity must be >= n), or < 0.
+ * group_count[g] receives the length of group g's substream (ceil(S / 32) entries). */
 int64_t orc_rans_encode_chunk(const uint8_t *sym, int64_t n, const uint32_t *freqs,
                               uint32_t prob_bits, uint32_t S, uint32_t G, uint32_t *states_out,
-                              uint16_t *words_out) {
+                              uint16_t *words_out, int64_t *group_count) {
   if (S < 1 || G < 1 || n < 0) return ORC_ERR_ARG;
   uint32_t cum[256];
   cum_of(freqs, cum);
+  const int64_t ng = orc_rans_groups(S);
   uint32_t *x = (uint32_t *)malloc(S * sizeof(uint32_t));
+  /* one stack per group, each with room for every symbol of the chunk */
+  uint16_t *stack = (uint16_t *)malloc((size_t)(ng * (n > 0 ? n : 1)) * sizeof(uint16_t));
+  int64_t *depth = (int64_t *)calloc((size_t)ng, sizeof(int64_t));
   for (uint32_t s = 0; s < S; ++s) x[s] = RANS_L;
-  int64_t runs = (n + G - 1) / G, rounds = (runs + S - 1) / S, nw = 0;
+  int64_t runs = (n + G - 1) / G, rounds = (runs + S - 1) / S;
   for (int64_t round = rounds - 1; round >= 0; --round)
     for (int64_t p = (int64_t)G - 1; p >= 0; --p)
       for (int64_t s = (int64_t)S - 1; s >= 0; --s) {
@@ -264,43 +276,55 @@ int64_t orc_rans_encode_chunk(const uint8_t *sym, int64_t n, const uint32_t *fre
         uint32_t f = freqs[sym[j]];
         if (f == 0) {
           free(x);
+          free(stack);
+          free(depth);
           return ORC_ERR_SYMBOL;
         }
         uint64_t xmax = (uint64_t)f << (32 - prob_bits);
         uint32_t xs = x[s];
         if ((uint64_t)xs >= xmax) {
-          words_out[nw++] = (uint16_t)(xs & 0xFFFFu);
+          int64_t g = s / RANS_GROUP;
+          stack[g * n + depth[g]++] = (uint16_t)(xs & 0xFFFFu);
           xs >>= 16;
         }
         x[s] = ((xs / f) << prob_bits) + (xs % f) + cum[sym[j]];
       }
-  for (int64_t i = 0; i < nw / 2; ++i) {
-    uint16_t t = words_out[i];
-    words_out[i] = words_out[nw - 1 - i];
-    words_out[nw - 1 - i] = t;
+  int64_t nw = 0;
+  for (int64_t g = 0; g < ng; ++g) {
+    for (int64_t i = depth[g] - 1; i >= 0; --i) words_out[nw++] = stack[g * n + i];
+    group_count[g] = depth[g];
   }
   memcpy(states_out, x, S * sizeof(uint32_t));
   free(x);
+  free(stack);
+  free(depth);
   return nw;
 }
 
-int orc_rans_decode_chunk(const uint16_t *words, int64_t nwords, const uint32_t *states, int64_t n,
-                          const uint32_t *freqs, uint32_t prob_bits, uint32_t S, uint32_t G,
-                          uint8_t *sym_out) {
+/* group_off[g] .. group_off[g + 1]: group g's words inside `words` (ceil(S / 32) + 1 entries). */
+int orc_rans_decode_chunk(const uint16_t *words, const int64_t *group_off, const uint32_t *states,
+                          int64_t n, const uint32_t *freqs, uint32_t prob_bits, uint32_t S,
+                          uint32_t G, uint8_t *sym_out) {
   if (S < 1 || G < 1 || n < 0) return ORC_ERR_ARG;
   const uint32_t M = 1u << prob_bits;
+  const int64_t ng = orc_rans_groups(S);
   uint32_t cum[256];
   cum_of(freqs, cum);
   uint8_t *slot_sym = (uint8_t *)malloc(M);
   for (int s = 0; s < 256; ++s)
     for (uint32_t k = 0; k < freqs[s]; ++k) slot_sym[cum[s] + k] = (uint8_t)s;
   uint32_t *x = (uint32_t *)malloc(S * sizeof(uint32_t));
+  int64_t *ptr = (int64_t *)malloc((size_t)ng * sizeof(int64_t));
   int rc = ORC_OK;
+  for (int64_t g = 0; g < ng; ++g) {
+    ptr[g] = group_off[g];
+    if (group_off[g + 1] < group_off[g]) rc = ORC_ERR_ARG;
+  }
   for (uint32_t s = 0; s < S; ++s) {
     x[s] = states[s];
     if (x[s] < RANS_L) rc = ORC_ERR_CORRUPT;
   }
-  int64_t runs = (n + G - 1) / G, rounds = (runs + S - 1) / S, ptr = 0;
+  int64_t runs = (n + G - 1) / G, rounds = (runs + S - 1) / S;
   for (int64_t round = 0; round < rounds && rc == ORC_OK; ++round)
     for (int64_t p = 0; p < (int64_t)G && rc == ORC_OK; ++p)
       for (int64_t s = 0; s < (int64_t)S; ++s) {
@@ -310,42 +334,50 @@ int orc_rans_decode_chunk(const uint16_t *words, int64_t nwords, const uint32_t 
         uint8_t q = slot_sym[slot];
         x[s] = freqs[q] * (x[s] >> prob_bits) + slot - cum[q];
         if (x[s] < RANS_L) {
-          if (ptr >= nwords) {
+          int64_t g = s / RANS_GROUP;
+          if (ptr[g] >= group_off[g + 1]) {
             rc = ORC_ERR_OVERRUN;
             break;
           }
-          x[s] = (x[s] << 16) | words[ptr++];
+          x[s] = (x[s] << 16) | words[ptr[g]++];
         }
         sym_out[j] = q;
       }
   if (rc == ORC_OK) {
     for (uint32_t s = 0; s < S; ++s)
       if (x[s] != RANS_L) rc = ORC_ERR_CORRUPT;
-    if (ptr != nwords) rc = ORC_ERR_CORRUPT;
+    for (int64_t g = 0; g < ng; ++g)
+      if (ptr[g] != group_off[g + 1]) rc = ORC_ERR_CORRUPT;
   }
   free(x);
+  free(ptr);
   free(slot_sym);
   return rc;
 }
 
 /* Decode chunks [c0, c1) of a tensor container and dequantise them to bf16 (the whole job of the
- * GPU decode, done plainly).  Chunk c holds symbols [c*chunk, min(N, (c+1)*chunk)). */
+ * GPU decode, done plainly).  Chunk c holds symbols [c*chunk, min(N, (c+1)*chunk)); its group g
+ * substream is words[word_off[c * groups + g] .. word_off[c * groups + g + 1]). */
 int orc_rans_decode_bf16(const uint16_t *words, const uint64_t *word_off, const uint32_t *states,
                          const uint32_t *freqs, const uint16_t *scales, int64_t rows, int64_t cols,
                          int symfmt, uint32_t prob_bits, int64_t chunk, uint32_t S, uint32_t G,
                          int64_t c0, int64_t c1, uint16_t *out) {
   int64_t N = rows * cols;
+  const int64_t ng = orc_rans_groups(S);
   uint8_t *tmp = (uint8_t *)malloc((size_t)(chunk > 0 ? chunk : 1));
+  int64_t *goff = (int64_t *)malloc((size_t)(ng + 1) * sizeof(int64_t));
   int rc = ORC_OK;
   for (int64_t c = c0; c < c1 && rc == ORC_OK; ++c) {
     int64_t j0 = c * chunk, n = (N - j0 < chunk) ? N - j0 : chunk;
-    rc = orc_rans_decode_chunk(words + word_off[c], (int64_t)(word_off[c + 1] - word_off[c]),
-                               states + (size_t)c * S, n, freqs, prob_bits, S, G, tmp);
+    for (int64_t g = 0; g <= ng; ++g) goff[g] = (int64_t)(word_off[c * ng + g] - word_off[c * ng]);
+    rc = orc_rans_decode_chunk(words + word_off[c * ng], goff, states + (size_t)c * S, n, freqs,
+                               prob_bits, S, G, tmp);
     for (int64_t i = 0; i < n && rc == ORC_OK; ++i) {
       int64_t j = j0 + i;
       out[j] = orc_dequant_one(tmp[i], scales[j / cols], symfmt);
     }
   }
+  free(goff);
   free(tmp);
   return rc;
 }

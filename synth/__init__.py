@@ -174,6 +174,13 @@ class Workload:
     run: int = 8                   # consecutive symbols a stream decodes before the next stream
     int8_div: float = 0.0          # Int8: scale = absmax(row) / int8_div
     batches: tuple = field(default=())
+    chunk_rows: int = 0            # > 0: chunks of this many whole rows (overrides chunk_symbols)
+
+    def chunk_for(self, spec: "TensorSpec") -> int:
+        """Chunk length in symbols for one tensor of the workload."""
+        if self.chunk_rows:
+            return self.chunk_rows * spec.cols
+        return self.chunk_symbols if self.chunk_symbols else spec.cols
 
     @property
     def numel(self) -> int:
@@ -207,7 +214,8 @@ WORKLOADS = {
     "mlp_13b": Workload("mlp_13b", (TensorSpec("gate", 13824, 5120, "normal", 4, 0),
                                     TensorSpec("up", 13824, 5120, "normal", 4, 1),
                                     TensorSpec("down", 5120, 13824, "normal", 4, 2)),
-                        symfmt="e4m3", chunk_symbols=0, streams=64, run=8, batches=(1, 4, 16)),
+                        symfmt="e4m3", chunk_symbols=0, streams=32, run=8, batches=(1, 4, 16),
+                        chunk_rows=4),
     "df11_8k": Workload("df11_8k", (TensorSpec("w", 8192, 28672, "bf16_normal", 5, 0,
                                                std=0.015),), symfmt="bf16"),
 }
@@ -223,4 +231,4 @@ def scaled(w: Workload, row_div: int = 1, layers: int | None = None) -> Workload
                           t.std, t.b, t.clip, t.frac, t.mult) for t in ts)
     return Workload(w.name + (f"/rows{row_div}" if row_div > 1 else "")
                     + (f"/layers{layers}" if layers is not None else ""), ts, w.symfmt,
-                    w.chunk_symbols, w.streams, w.run, w.int8_div, w.batches)
+                    w.chunk_symbols, w.streams, w.run, w.int8_div, w.batches, w.chunk_rows)

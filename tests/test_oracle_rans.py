@@ -41,14 +41,14 @@ TABLES = [
 def test_bruteforce_roundtrip_all_short_sequences(orc, ti):
     f = TABLES[ti]
     alphabet = np.nonzero(f)[0]
-    for S, G in [(1, 1), (2, 1), (2, 8), (32, 1), (32, 8), (3, 2)]:
+    for S, G in [(1, 1), (2, 1), (2, 8), (32, 1), (32, 8), (3, 2), (40, 1), (64, 8)]:
         for n in range(0, 8):
             for seq in itertools.product(alphabet, repeat=n):
                 sym = np.array(seq, np.uint8)
-                st, words = orc.rans_encode_chunk(sym, f, S, G)
-                rc, out = orc.rans_decode_chunk(words, st, n, f, S, G)
+                st, words, cnt = orc.rans_encode_chunk(sym, f, S, G)
+                rc, out = orc.rans_decode_chunk(words, st, n, f, S, G, cnt)
                 assert rc == 0 and np.array_equal(out, sym), (ti, S, G, seq)
-            if n >= 5 and S == 32:
+            if n >= 5 and S >= 32:
                 break
 
 
@@ -61,7 +61,7 @@ def test_uniform_table_closed_form(orc):
     rng = np.random.default_rng(5)
     for S, G, n in [(1, 1, 9), (32, 8, 1000), (32, 1, 777), (4, 8, 333), (64, 8, 100)]:
         sym = rng.integers(0, 256, n, dtype=np.uint8)
-        st, words = orc.rans_encode_chunk(sym, f, S, G)
+        st, words, _ = orc.rans_encode_chunk(sym, f, S, G)
         stream = (np.arange(n) // G) % S
         expect_words = 0
         for s in range(S):
@@ -81,9 +81,9 @@ def test_single_symbol_table_emits_nothing(orc):
     f = table({42: M})
     for S, G in [(1, 1), (32, 8), (128, 8)]:
         sym = np.full(5000, 42, np.uint8)
-        st, words = orc.rans_encode_chunk(sym, f, S, G)
-        assert words.size == 0 and (st == 1 << 16).all()
-        rc, out = orc.rans_decode_chunk(words, st, sym.size, f, S, G)
+        st, words, cnt = orc.rans_encode_chunk(sym, f, S, G)
+        assert words.size == 0 and (st == 1 << 16).all() and (cnt == 0).all()
+        rc, out = orc.rans_decode_chunk(words, st, sym.size, f, S, G, cnt)
         assert rc == 0 and (out == 42).all()
 
 
@@ -94,15 +94,33 @@ def test_stream_assignment_matches_slicing(orc):
     sym = synth.symbols_from_pmf(np.exp(-np.arange(256) / 9.0), 5000, 4)
     sym = sym[f[sym] > 0]
     n = sym.size
-    for S, G in [(32, 8), (64, 1), (5, 3)]:
-        st, words = orc.rans_encode_chunk(sym, f, S, G)
+    for S, G in [(32, 8), (64, 1), (5, 3), (96, 8)]:
+        st, words, cnt = orc.rans_encode_chunk(sym, f, S, G)
         total = 0
         for s in range(S):
             sl = sym[((np.arange(n) // G) % S) == s]
-            st1, w1 = orc.rans_encode_chunk(sl, f, 1, 1)
+            st1, w1, _ = orc.rans_encode_chunk(sl, f, 1, 1)
             assert st1[0] == st[s]
             total += w1.size
-        assert total == words.size
+        assert total == words.size == cnt.sum()
+
+
+def test_group_substream_is_a_32_stream_chunk(orc):
+    """Group g of a chunk (streams 32g .. 32g+31) codes the runs r with r mod S in its range; its
+    substream and states are exactly those of a 32-stream chunk made of those runs in order."""
+    sym = synth.symbols_from_pmf(np.exp(-np.arange(256) / 4.0), 30000, 11)
+    f = orc.rans_freqs(sym)
+    for S, G in [(64, 8), (128, 8), (96, 1)]:
+        n = sym.size - sym.size % 7
+        s = sym[:n]
+        st, words, cnt = orc.rans_encode_chunk(s, f, S, G)
+        offs = np.concatenate([[0], np.cumsum(cnt)])
+        runs = np.arange(n) // G
+        for g in range(S // 32):
+            mine = s[((runs % S) // 32) == g]
+            st1, w1, c1 = orc.rans_encode_chunk(mine, f, 32, G)
+            assert np.array_equal(st1, st[32 * g:32 * g + 32])
+            assert np.array_equal(w1, words[offs[g]:offs[g + 1]])
 
 
 def big_ans_encode(sym, f, cum):
@@ -134,7 +152,7 @@ def test_size_matches_arbitrary_precision_ans(orc):
     assert np.array_equal(back, sym) and x0 == 1 << 16
     ideal = sum(math.log2(M / f[s]) for s in sym.tolist())
     assert abs((math.log2(X) - 16) - ideal) < 1.0
-    st, words = orc.rans_encode_chunk(sym, f, 1, 1)
+    st, words, _ = orc.rans_encode_chunk(sym, f, 1, 1)
     coded = 16 * words.size + math.log2(int(st[0])) - 16
     assert abs(coded - (math.log2(X) - 16)) <= 0.002 * ideal + 1
 
@@ -142,7 +160,7 @@ def test_size_matches_arbitrary_precision_ans(orc):
 def test_corruption_is_reported(orc):
     sym = synth.symbols_from_pmf(np.exp(-np.arange(256) / 5.0), 20000, 9)
     f = orc.rans_freqs(sym)
-    st, words = orc.rans_encode_chunk(sym, f, 32, 8)
+    st, words, cnt = orc.rans_encode_chunk(sym, f, 32, 8)
     assert orc.rans_decode_chunk(words[:-1], st, sym.size, f, 32, 8)[0] != 0   # truncated
     bad = st.copy()
     bad[3] ^= 0x40
@@ -150,6 +168,8 @@ def test_corruption_is_reported(orc):
     bad = st.copy()
     bad[0] = 5                                                                   # state below L
     assert orc.rans_decode_chunk(words, bad, sym.size, f, 32, 8)[0] != 0
+    st2, w2, c2 = orc.rans_encode_chunk(sym, f, 64, 8)                         # words of the
+    assert orc.rans_decode_chunk(w2, st2, sym.size, f, 64, 8, c2[::-1])[0] != 0  # other group
     flipped = 0
     for k in range(40):
         w = words.copy()

@@ -43,7 +43,11 @@ def measured_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms in the background.
+
+    The sampler starts before the warm-up and a one-second untimed soak, so the clock has settled
+    and samples exist even when the timed steps take only milliseconds; summary() reports the
+    samples taken from 0.25 s before the timed region starts to its end (mark() brackets it)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -51,14 +55,15 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
-        self.lines: list[str] = []
+        self.samples: list[tuple[float, str]] = []
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except (OSError, FileNotFoundError):
@@ -67,10 +72,22 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, start: bool):
+        if start:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
+
+    def wait_first_sample(self, timeout: float = 5.0):
+        end = time.time() + timeout
+        while self.proc and not self.samples and time.time() < end:
+            time.sleep(0.05)
 
     def __exit__(self, *a):
         if self.proc:
+            time.sleep(0.3)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -78,22 +95,29 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], None, set()
+        lo = (self.t0 or 0) - 0.25
+        hi = (self.t1 or time.time()) + 0.05
+        sm, mx, reasons, pw = [], None, set(), []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.samples:
+            if not lo <= ts <= hi:
+                continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
             try:
                 sm.append(float(f[1]))
                 mx = float(f[2])
+                pw.append(float(f[3]))
             except ValueError:
                 continue
             for n, v in zip(names, f[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(pw) if pw else None,
+                "window_s": round(hi - lo, 3)}
 
 
 def dist_setup():
@@ -182,8 +206,17 @@ def run_ours(args):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
+        clk.wait_first_sample()
+        soak_end = time.time() + 1.0  # untimed: let the clocks settle under load
+        while time.time() < soak_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        barrier(world)
+        clk.mark(True)
         times = time_steps(step, args.steps, args.warmup, flush, stream)
         torch.cuda.synchronize()
+        clk.mark(False)
     barrier(world)
     assert int(status.item()) == 0, "decode reported corrupt data"
     mean_s = statistics.mean(times)

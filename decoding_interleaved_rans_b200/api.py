@@ -90,8 +90,11 @@ class DeviceRans:
             words = np.concatenate([words, np.zeros(8 - words.size % 8, np.uint16)])
         if words.size == 0:
             words = np.zeros(8, np.uint16)
+        chunk = int(h.chunk_symbols) if h.chunk_symbols else int(h.cols)
+        nchunks = (int(h.rows) * int(h.cols) + chunk - 1) // chunk
+        assert len(h.word_off) == nchunks * ((int(h.streams) + 31) // 32) + 1, "word_off length"
         t = cls(int(h.rows), int(h.cols), int(h.symfmt), int(h.prob_bits), int(h.chunk_symbols),
-                int(h.streams), int(h.run), int(len(h.word_off) - 1),
+                int(h.streams), int(h.run), nchunks,
                 _dev(np.asarray(h.states, np.uint32), device, np.int32),
                 _dev(np.asarray(h.word_off, np.uint64), device, np.int64),
                 _dev(words, device, np.int16),

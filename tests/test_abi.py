@@ -83,3 +83,57 @@ def test_gemv_and_huff_reject_bad_input_on_host(eq):
     h = eq._lib.HuffTensorDesc(10, 30, 8, 256, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
     h.bytes_per_thread = 4
     assert L.eq_huff_bf16_decode(C.byref(h), C.c_void_p(1 << 20), C.c_void_p(1 << 20), None) in (1, 3)
+
+
+class _FakeDev:
+    """Stands in for a device tensor: only its address is used, and only by host validation."""
+
+    def __init__(self, n_elems):
+        self._n = n_elems
+
+    def data_ptr(self):
+        return 1 << 24
+
+    def numel(self):
+        return self._n
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="launches would run on fake pointers; host-only check")
+@pytest.mark.parametrize("chunk,streams,run", [(16384, 32, 8), (65536, 128, 8), (0, 64, 8),
+                                               (999, 96, 1)])
+def test_binding_descriptors_pass_host_validation(eq, orc, chunk, streams, run):
+    """Descriptors built by the Python binding from a real container pass every host check; with
+    no CUDA device the call then stops at the first CUDA query (EQ_ERR_CUDA), never earlier."""
+    import synth
+    w = synth.normal(40, 1024, 0.02, 3)
+    sym, sc = orc.quantize(w, orc.E4M3)
+    for h in (orc.rans_encode(sym, sc, 1, chunk, streams, run),
+              eq.codec.rans_encode(sym, sc, 1, chunk, streams, run)):
+        nchunks = (h.rows * h.cols + (chunk or h.cols) - 1) // (chunk or h.cols)
+        t = eq.DeviceRans(h.rows, h.cols, h.symfmt, h.prob_bits, h.chunk_symbols, h.streams,
+                          h.run, nchunks, *[_FakeDev(1) for _ in range(5)])
+        assert len(h.word_off) == nchunks * (streams // 32) + 1
+        d = t.desc()
+        out = (C.c_void_p * 1)(1 << 24)
+        assert eq.lib().eq_decode(C.byref(d), 1, out, C.c_void_p(1 << 24), None) == 4
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="launches would run on fake pointers; host-only check")
+def test_binding_gemv_and_huff_descriptors_pass_host_validation(eq, orc):
+    import synth
+    wl = synth.WORKLOADS["mlp_13b"]
+    w = synth.normal(8, 5120, 0.02, 4)
+    sym, sc = orc.quantize(w, orc.E4M3)
+    h = eq.codec.rans_encode(sym, sc, 1, wl.chunk_rows * 5120, wl.streams, wl.run)
+    t = eq.DeviceRans(h.rows, h.cols, 1, 12, h.chunk_symbols, h.streams, h.run, 2,
+                      *[_FakeDev(1) for _ in range(5)])
+    d = t.desc()
+    fake = C.c_void_p(1 << 24)
+    assert eq.lib().eq_decode_gemv(C.byref(d), fake, 4, fake, fake, None) == 4
+    hb = eq.codec.huff_encode(synth.bf16_normal(4, 4096, 0.015, 5))
+    th = eq.DeviceHuff(hb.n, hb.total_bits, 8, hb.threads_per_block,
+                       *[_FakeDev(1) for _ in range(5)])
+    dh = th.desc()
+    assert eq.lib().eq_huff_bf16_decode(C.byref(dh), fake, fake, None) == 4

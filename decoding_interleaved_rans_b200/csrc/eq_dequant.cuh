@@ -33,33 +33,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&b);
 }
 
-// E4M3 NaN codes (0x7F, 0xFF) -> bf16 quiet NaN keeping the sign.  `four` holds 4 symbols,
-// `lo`/`hi` the two packed bf16 pairs computed for them.
-__device__ __forceinline__ void fix_e4m3_nan(uint32_t four, uint32_t &lo, uint32_t &hi) {
-  uint32_t r[2] = {lo, hi};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t b = (four >> (8 * i)) & 0xFFu;
-    if ((b & 0x7Fu) == 0x7Fu) {
-      uint32_t nan = 0x7FC0u | ((b & 0x80u) << 8);
-      uint32_t sh = 16 * (i & 1);
-      r[i >> 1] = (r[i >> 1] & ~(0xFFFFu << sh)) | (nan << sh);
-    }
-  }
-  lo = r[0];
-  hi = r[1];
-}
-
-// four symbols (low byte first) scaled -> four bf16 in two 32-bit words
+// two symbols (16-bit pair, first in the low byte) scaled -> two bf16 in one 32-bit word.
+// E4M3 NaN codes (0x7F, 0xFF) become the bf16 quiet NaN with the code's sign when nan_codes.
 template <int FMT>
-__device__ __forceinline__ uint2 dequant4(uint32_t four, float scale, bool nan_codes) {
-  float2 a = sym2_value<FMT>(four & 0xFFFFu);
-  float2 b = sym2_value<FMT>(four >> 16);
-  uint2 o;
-  o.x = pack_bf16x2(a.x * scale, a.y * scale);
-  o.y = pack_bf16x2(b.x * scale, b.y * scale);
+__device__ __forceinline__ uint32_t dequant2(uint32_t pair, float scale, bool nan_codes) {
+  const float2 v = sym2_value<FMT>(pair);
+  uint32_t o = pack_bf16x2(v.x * scale, v.y * scale);
   if constexpr (FMT == EQ_SYM_E4M3) {
-    if (nan_codes) fix_e4m3_nan(four, o.x, o.y);
+    if (nan_codes) {
+      if ((pair & 0x7Fu) == 0x7Fu) o = (o & 0xFFFF0000u) | 0x7FC0u | ((pair & 0x80u) << 8);
+      if ((pair & 0x7F00u) == 0x7F00u)
+        o = (o & 0x0000FFFFu) | ((0x7FC0u | (pair & 0x8000u)) << 16);
+    }
   }
   return o;
 }

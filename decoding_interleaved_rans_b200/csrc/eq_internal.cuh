@@ -13,9 +13,11 @@ namespace eq {
 // ------------------------------------------------------------------------------------------------
 
 // rANS: 16-byte header, then one 32-bit entry per slot of the 4096-slot probability space:
-//   bits 31..24 symbol, bits 23..12 frequency (1..4095), bits 11..0 slot - cum[symbol].
-// A table whose single symbol owns all 4096 slots cannot store its frequency in 12 bits; the
-// header flags it instead and the decoders take a separate path.
+//   bits 31..20 frequency f (1..4095), bits 19..12 symbol, bits 11..0 slot - cum[symbol].
+// With f in the top bits, f * floor(x / 4096) is the high word of (e & 0xFFF00000) *
+// (x & 0xFFFFF000), one multiply-high.  A table whose single symbol owns all 4096 slots cannot
+// store its frequency in 12 bits; the header flags it instead and the decoders take a separate
+// path.
 constexpr uint32_t kRansProbBits = 12;
 constexpr uint32_t kRansSlots = 1u << kRansProbBits;
 constexpr uint32_t kRansL = 1u << 16;

@@ -21,6 +21,7 @@ constexpr uint32_t kRoundWords = 32 * 8;  // words a group reads at most per rou
 // ------------------------------------------------------------------------------------------------
 struct WordRing {
   unsigned char *buf;
+  uint32_t ring_off;  // buf - shared-memory base (a multiple of kRingBytes)
   uint64_t *bar;
   const unsigned char *A;
   uint32_t off0;    // bytes from A to the first word
@@ -90,33 +91,53 @@ struct WordRing {
 
 // ------------------------------------------------------------------------------------------------
 // One decode step of the lane's state x.  q is the byte offset (from the ring's A) of the group's
-// next unread word; it advances by 2 bytes per word the warp reads.  Slot-table entry: symbol in
-// bits 31..24, frequency in 23..12, slot - cum in 11..0.  A ballot finds the lanes whose state
-// fell below 2^16; each takes the word at its rank among them, so words go out in stream order.
+// next unread word; it advances by 2 bytes per word the warp reads.  Slot-table entry e: f in bits
+// 31..20, symbol in 19..12, slot - cum in 11..0, so f * floor(x / 4096) + (slot - cum) is one
+// multiply-high-add: hi32((e & 0xFFF00000) * (x & 0xFFFFF000)) + (e & 0xFFF).  A ballot finds
+// the lanes whose state fell below 2^16; each takes the word at its rank among them, so words go
+// out in stream order.  ring_off: shared-memory offset of this warp's ring (a multiple of its
+// size), so the word address is one mask-and-or.
 // ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 template <bool FULL>
 __device__ __forceinline__ uint32_t rans_step(uint32_t &x, bool act, const uint32_t *lut,
-                                              const WordRing &R, uint32_t &q, uint32_t lt) {
+                                              const unsigned char *smem, uint32_t ring_off,
+                                              uint32_t &q, uint32_t lt) {
   const uint32_t e = lut[x & (kRansSlots - 1)];
-  const uint32_t nx = ((e >> 12) & 0xFFFu) * (x >> kRansProbBits) + (e & 0xFFFu);
+  const uint32_t nx = mad_hi(e & 0xFFF00000u, x & 0xFFFFF000u, e & 0xFFFu);
   const bool on = FULL || act;
   if (on) x = nx;
   const bool need = on && x < kRansL;
   const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-  if (need) x = (x << 16) | R.word_at(q + 2 * __popc(m & lt));
-  q += 2 * __popc(m);
+  if (need) {
+    const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (kRingBytes - 1)) | ring_off;
+    x = mad_lo(x, 65536u, *reinterpret_cast<const uint16_t *>(smem + a));
+  }
+  q = mad_lo(__popc(m), 2u, q);
   return e;
 }
 
-// byte 3 of `e` into byte p of `acc`
-__device__ __forceinline__ uint32_t put_sym(uint32_t acc, uint32_t e, int p) {
-  return __byte_perm(acc, e, (0x3210u & ~(0xFu << (4 * p))) | (0x7u << (4 * p)));
+// symbols of two slot-table entries as one 16-bit pair (first in the low byte)
+__device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {
+  return ((e0 >> 12) & 0xFFu) | ((e1 >> 4) & 0xFF00u);
 }
 
 // Init the rings' mbarriers (lane 0 of each warp) -- call before the block-wide sync.
-__device__ __forceinline__ void ring_init(WordRing &R, unsigned char *rings, uint64_t *bars,
-                                          uint32_t warp, uint32_t lane) {
+__device__ __forceinline__ void ring_init(WordRing &R, unsigned char *smem, unsigned char *rings,
+                                          uint64_t *bars, uint32_t warp, uint32_t lane) {
   R.buf = rings + warp * kRingBytes;
+  R.ring_off = uint32_t(R.buf - smem);
   R.bar = bars + warp * kNumSeg;
   if (lane == 0) {
     for (uint32_t s = 0; s < kNumSeg; ++s) mbar_init(&R.bar[s], 1);

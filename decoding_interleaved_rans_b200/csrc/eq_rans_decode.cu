@@ -53,30 +53,32 @@ struct RansDecodeParams {
 // ------------------------------------------------------------------------------------------------
 template <bool FULL, int G, int FMT>
 __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
-                                             const uint32_t *lut, const WordRing &R, uint32_t &q,
-                                             uint32_t lt, uint64_t jrun, bool nan_codes) {
-  uint32_t sym[(G + 3) / 4] = {};
+                                             const uint32_t *lut, const unsigned char *smem,
+                                             const WordRing &R, uint32_t &q, uint32_t lt,
+                                             uint64_t jrun, bool nan_codes) {
+  uint32_t e[G];
 #pragma unroll
-  for (int p = 0; p < G; ++p) {
-    const uint32_t e = rans_step<FULL>(x, act, lut, R, q, lt);
-    sym[p >> 2] = put_sym(sym[p >> 2], e, p & 3);
-  }
+  for (int p = 0; p < G; ++p) e[p] = rans_step<FULL>(x, act, lut, smem, R.ring_off, q, lt);
   if (FULL || act) {
     const float sc = bf16_bits_to_float(D.scales[div_by_magic(jrun, D.row_magic)]);
     if constexpr (G == 8) {
-      const uint2 a = dequant4<FMT>(sym[0], sc, nan_codes);
-      const uint2 b = dequant4<FMT>(sym[1], sc, nan_codes);
-      *reinterpret_cast<uint4 *>(D.out + jrun) = make_uint4(a.x, a.y, b.x, b.y);
+      uint4 o;
+      o.x = dequant2<FMT>(sym_pair(e[0], e[1]), sc, nan_codes);
+      o.y = dequant2<FMT>(sym_pair(e[2], e[3]), sc, nan_codes);
+      o.z = dequant2<FMT>(sym_pair(e[4], e[5]), sc, nan_codes);
+      o.w = dequant2<FMT>(sym_pair(e[6], e[7]), sc, nan_codes);
+      *reinterpret_cast<uint4 *>(D.out + jrun) = o;
     } else {
-      D.out[jrun] = dequant1<FMT>(sym[0], sc);
+      D.out[jrun] = dequant1<FMT>((e[0] >> 12) & 0xFFu, sc);
     }
   }
 }
 
 template <int G, int FMT>
 __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32_t *lut,
-                                                 uint32_t flags, uint32_t single_sym, WordRing &R,
-                                                 uint64_t unit, uint32_t lane) {
+                                                 const unsigned char *smem, uint32_t flags,
+                                                 uint32_t single_sym, WordRing &R, uint64_t unit,
+                                                 uint32_t lane) {
   const uint64_t chunk = unit / D.groups;
   const uint32_t g = uint32_t(unit - chunk * D.groups);
   const uint32_t S = 32 * D.groups, s = 32 * g + lane;
@@ -117,8 +119,8 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
     }
     const uint32_t run = r * S + s;
     const uint64_t jrun = j0 + uint64_t(run) * G;
-    if (r < full) decode_round<true, G, FMT>(D, x, true, lut, R, q, lt, jrun, nan_codes);
-    else decode_round<false, G, FMT>(D, x, run < runs, lut, R, q, lt, jrun, nan_codes);
+    if (r < full) decode_round<true, G, FMT>(D, x, true, lut, smem, R, q, lt, jrun, nan_codes);
+    else decode_round<false, G, FMT>(D, x, run < runs, lut, smem, R, q, lt, jrun, nan_codes);
     if (q - R.off0 > 2 * nwords) {
       status |= EQ_DEV_OVERRUN;
       break;
@@ -153,14 +155,14 @@ __global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant_
   for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
     reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
   WordRing R;
-  ring_init(R, rings, bars, warp, lane);
+  ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
   const uint64_t unit = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
   if (unit >= D.units) return;
   uint32_t status = 0;
   if (hdr.magic != kRansMagic) status = EQ_DEV_CORRUPT_STATE;
-  else status = decode_group<G, FMT>(D, lut, hdr.flags, hdr.single_sym, R, unit, lane);
+  else status = decode_group<G, FMT>(D, lut, smem, hdr.flags, hdr.single_sym, R, unit, lane);
   if (lane == 0) report(P.status, status);
 }
 

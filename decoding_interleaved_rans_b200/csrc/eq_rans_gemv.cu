@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
   for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
     reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
   WordRing R;
-  ring_init(R, rings, bars, warp, lane);
+  ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
   const uint64_t chunk = uint64_t(blockIdx.x) * P.warps + warp;
@@ -113,19 +113,19 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
 
   for (uint32_t r = 0; r < rounds; ++r) {
     const bool act = r * S + lane < runs;
-    uint32_t sym[2] = {0u, 0u};
+    uint32_t pr[4];  // the round's 8 symbols as 4 pairs
     if (single) {
-      sym[0] = sym[1] = hdr.single_sym * 0x01010101u;
+      pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
     } else {
       if (!R.wait_below(q + 2 * kRoundWords)) {
         status |= EQ_DEV_TIMEOUT;
         break;
       }
+      uint32_t e[8];
 #pragma unroll
-      for (int p = 0; p < 8; ++p) {
-        const uint32_t e = rans_step<false>(x, act, lut, R, q, lt);
-        sym[p >> 2] = put_sym(sym[p >> 2], e, p & 3);
-      }
+      for (int p = 0; p < 8; ++p) e[p] = rans_step<false>(x, act, lut, smem, R.ring_off, q, lt);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pr[k] = sym_pair(e[2 * k], e[2 * k + 1]);
       if (q - R.off0 > 2 * nwords) {
         status |= EQ_DEV_OVERRUN;
         break;
@@ -134,8 +134,9 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
     }
     if (act) {  // the weights exactly as eq_decode writes them, times the activations
       const uint32_t col = (r * S + lane) * 8 - row_local * P.cols;
-      fma_run<BMAX>(acc, dequant4<FMT>(sym[0], sc, nan_codes), dequant4<FMT>(sym[1], sc, nan_codes),
-                    P.x, P.cols, col, batch);
+      const uint2 wa = make_uint2(dequant2<FMT>(pr[0], sc, nan_codes), dequant2<FMT>(pr[1], sc, nan_codes));
+      const uint2 wb = make_uint2(dequant2<FMT>(pr[2], sc, nan_codes), dequant2<FMT>(pr[3], sc, nan_codes));
+      fma_run<BMAX>(acc, wa, wb, P.x, P.cols, col, batch);
     }
     // end of a weight row: reduce across the warp and write y
     const bool row_end = (r + 1 == rounds) || (P.rows_per_chunk > 1 && (r + 1) % P.rounds_per_row == 0);

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
     }
     uint32_t f = a.freq[lo];
     uint32_t fe = (f >= kRansSlots) ? 0u : f;  // a one-symbol table is handled by the flag
-    lut[slot] = (uint32_t(lo) << 24) | (fe << 12) | (slot - cum[lo]);
+    lut[slot] = (fe << 20) | (uint32_t(lo) << 12) | (slot - cum[lo]);
   }
 }
 

@@ -215,7 +215,7 @@ WORKLOADS = {
                                     TensorSpec("up", 13824, 5120, "normal", 4, 1),
                                     TensorSpec("down", 5120, 13824, "normal", 4, 2)),
                         symfmt="e4m3", chunk_symbols=0, streams=32, run=8, batches=(1, 4, 16),
-                        chunk_rows=4),
+                        chunk_rows=1),
     "df11_8k": Workload("df11_8k", (TensorSpec("w", 8192, 28672, "bf16_normal", 5, 0,
                                                std=0.015),), symfmt="bf16"),
 }

@@ -55,7 +55,7 @@ def test_all_exponents_and_long_codes(eq, orc):
     rng.shuffle(e)
     w = ((rng.integers(0, 2, e.size) << 15) | (e << 7) | rng.integers(0, 128, e.size)).astype(np.uint16)
     h = orc.huff_encode_bf16(w)
-    assert h.lengths.max() >= 20
+    assert h.lengths.max() >= 12  # three table levels
     out, st = run(eq, h)
     assert st == 0 and np.array_equal(out, w)
     fibc = np.zeros(256, np.uint64)

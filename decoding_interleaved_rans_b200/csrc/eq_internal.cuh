@@ -33,21 +33,31 @@ constexpr uint32_t kRansFlagNaNFF = 2u;       // frequency of byte 0xFF is nonze
 constexpr uint32_t kRansFlagSingle = 4u;      // one symbol owns every slot
 constexpr size_t kRansTableBytes = sizeof(RansTableHeader) + kRansSlots * 4;
 
-// Huffman (DFloat11 exponent): 16-byte header, then up to kHuffMaxTables tables of 256 uint16
-// entries.  Table 0 is indexed by the next 8 code bits; an entry is either
-//   a leaf   (bit 15 clear): bits 7..0 exponent value, bits 11..8 bits used at this level (1..8)
-//   a pointer (bit 15 set):  bits 7..0 index of the child table, which reads the next 8 bits
-//   0xFFFF: no code starts with this bit pattern.
+// Huffman (DFloat11 exponent): 16-byte header, then
+//   a window table W: 4096 x uint64, indexed by the next 12 code bits, listing the codes that lie
+//   wholly inside those 12 bits (up to 4): bits 8i..8i+7 value of code i, bits 32+4i..35+4i its
+//   length, bits 48..51 their total length, bits 52..54 how many (0 = no code fits, which is a
+//   bad pattern unless bit 63 says the first code is longer than 12 bits);
+//   then up to kHuffMaxTables hierarchical tables of 256 uint16 entries for codes of any length:
+//   table 0 is indexed by the next 8 code bits; an entry is
+//     a leaf    (bit 15 clear): bits 7..0 exponent value, bits 11..8 bits used at this level (1..8)
+//     a pointer (bit 15 set):   bits 7..0 index of the child table, which reads the next 8 bits
+//     0xFFFF: no code starts with this bit pattern.
 constexpr uint32_t kHuffMaxTables = 32;
+constexpr uint32_t kHuffWindowBits = 12;
+constexpr uint32_t kHuffWindow = 1u << kHuffWindowBits;
+constexpr uint64_t kHuffLong = 1ull << 63;
 struct HuffTableHeader {
   uint32_t magic;        // kHuffMagic
-  uint32_t num_tables;
+  uint32_t num_tables;   // hierarchical tables in use
   uint32_t max_len;
   uint32_t reserved;
 };
-constexpr uint32_t kHuffMagic = 0x48554646u;  // "HUFF"
+constexpr uint32_t kHuffMagic = 0x48554647u;  // "HUFG"
 constexpr uint16_t kHuffInvalid = 0xFFFFu;
-constexpr size_t kHuffTableBytes = sizeof(HuffTableHeader) + kHuffMaxTables * 256 * 2;
+constexpr size_t kHuffWindowOffset = sizeof(HuffTableHeader);
+constexpr size_t kHuffTreeOffset = kHuffWindowOffset + kHuffWindow * 8;
+constexpr size_t kHuffTableBytes = kHuffTreeOffset + kHuffMaxTables * 256 * 2;
 
 // ------------------------------------------------------------------------------------------------
 // host helpers

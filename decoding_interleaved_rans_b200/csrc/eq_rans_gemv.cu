@@ -162,6 +162,179 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
   if (lane == 0) report(P.status, status);
 }
 
+// ------------------------------------------------------------------------------------------------
+// Batch >= 8: the product goes to the tensor cores.  A CTA of 16 warps decodes 16 chunks in
+// lock-step, one round (256 weights of one row per warp) at a time; each warp writes its
+// dequantised bf16 weights into a shared 16 x 256 tile, and after a barrier the 16 warps multiply
+// the tile by the matching 256 x batch slice of x with mma.m16n8k16 (bf16 in, fp32 accumulate),
+// one 16-column k-step each.  At the end of a weight row the 16 warps' partial products are
+// summed in a fixed order through shared memory and written to y.  The weights are the ones
+// eq_decode returns and every product is exact in fp32, as in the CUDA-core path.
+// ------------------------------------------------------------------------------------------------
+constexpr uint32_t kTcWarps = 16;
+constexpr uint32_t kTcRowBytes = 256 * 2 + 16;  // one tile row, padded against bank conflicts
+constexpr uint32_t kTcTileBytes = kTcWarps * kTcRowBytes;
+
+__host__ __device__ constexpr size_t gemv_tc_smem_bytes() {
+  return rans_smem_bytes(kTcWarps) + 2 * kTcTileBytes + kTcWarps * 16 * 16 * 4;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __grid_constant__ GemvParams P) {
+  constexpr uint32_t S = 32;
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
+  unsigned char *rings = smem + kRansSlots * 4;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + kTcWarps * kRingBytes);
+  unsigned char *tiles = smem + rans_smem_bytes(kTcWarps);          // 2 x [16][264] bf16
+  float *red = reinterpret_cast<float *>(tiles + 2 * kTcTileBytes);  // [16 warps][16 rows][16 b]
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t grp = lane >> 2, tig = lane & 3;
+
+  const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
+  const uint4 *src = reinterpret_cast<const uint4 *>(P.table + sizeof(RansTableHeader) / 4);
+  for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
+    reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+  WordRing R;
+  ring_init(R, smem, rings, bars, warp, lane);
+  __syncthreads();
+
+  // every warp runs the same number of rounds (a full chunk's), so the barriers line up;
+  // a warp without a chunk, or whose chunk failed, feeds zeros
+  const uint64_t chunk = uint64_t(blockIdx.x) * kTcWarps + warp;
+  const bool have = chunk < P.num_chunks;
+  uint32_t status = have && hdr.magic != kRansMagic ? EQ_DEV_CORRUPT_STATE : 0u;
+  const bool single = hdr.flags & kRansFlagSingle;
+  const bool nan_codes = (FMT == EQ_SYM_E4M3) && (hdr.flags & (kRansFlagNaN7F | kRansFlagNaNFF));
+  uint32_t x = kRansL, nwords = 0, q = 0, n = 0;
+  bool started = false;
+  if (have && !status) {
+    const uint64_t j0 = chunk * uint64_t(P.chunk_symbols);
+    n = uint32_t(P.numel - j0 < P.chunk_symbols ? P.numel - j0 : P.chunk_symbols);
+    const uint64_t w0 = P.word_off[chunk], w1 = P.word_off[chunk + 1];
+    if (w1 < w0 || w1 - w0 >= (1ull << 30)) status |= EQ_DEV_OVERRUN;
+    nwords = status ? 0u : uint32_t(w1 - w0);
+    x = P.states[chunk * S + lane];
+    if (!status && !single) {
+      R.start(P.words, w0, nwords, lane);
+      q = R.off0;
+      started = true;
+    }
+  }
+  bool live = have && !status && !single;  // decoding from the stream
+  const uint32_t lt = lanemask_lt();
+  const uint32_t runs = n / 8;
+  const uint32_t rounds = P.chunk_symbols / 256;  // the same for every warp of the launch
+  const uint32_t rpr = P.rows_per_chunk > 1 ? P.rounds_per_row : rounds;
+  const uint32_t row0 = uint32_t(chunk * P.rows_per_chunk);
+  const uint32_t ntiles = (P.batch + 7) / 8;
+  float c[2][4] = {};
+  uint32_t row_local = 0;
+  float sc = have && !status ? bf16_bits_to_float(P.scales[row0]) : 0.0f;
+  const uint32_t tiles_addr = smem_addr(tiles);
+
+  for (uint32_t r = 0; r < rounds; ++r) {
+    const bool act = have && !status && r * S + lane < runs;
+    uint32_t pr[4] = {0u, 0u, 0u, 0u};
+    if (live) {
+      if (!R.wait_below(q + 2 * kRoundWords)) {
+        status |= EQ_DEV_TIMEOUT;
+        live = false;
+      } else {
+        uint32_t e[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) e[p] = rans_step<false>(x, act, lut, smem, R.ring_off, q, lt);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) pr[k] = sym_pair(e[2 * k], e[2 * k + 1]);
+        if (q - R.off0 > 2 * nwords) {
+          status |= EQ_DEV_OVERRUN;
+          live = false;
+        } else {
+          R.refill(q, lane);
+        }
+      }
+    } else if (single) {
+      pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
+    }
+    // this warp's 256 weights of the round -> tile row `warp`
+    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
+    if (act && !status) {
+      wv.x = dequant2<FMT>(pr[0], sc, nan_codes);
+      wv.y = dequant2<FMT>(pr[1], sc, nan_codes);
+      wv.z = dequant2<FMT>(pr[2], sc, nan_codes);
+      wv.w = dequant2<FMT>(pr[3], sc, nan_codes);
+    }
+    unsigned char *tile = tiles + (r & 1) * kTcTileBytes;
+    *reinterpret_cast<uint4 *>(tile + warp * kTcRowBytes + lane * 16) = wv;
+    __syncthreads();
+    // warp w multiplies tile columns [16 w, 16 w + 16) by x[:, col0 + 16 w ...]
+    {
+      uint32_t a[4];
+      const uint32_t arow = lane & 15, acol = (lane >> 4) * 8 + warp * 16;
+      ldmatrix_x4(a, tiles_addr + (r & 1) * kTcTileBytes + arow * kTcRowBytes + acol * 2);
+      const uint32_t col0 = (r % rpr) * 256 + warp * 16 + 2 * tig;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        if (uint32_t(nt) < ntiles) {
+          const uint32_t b = nt * 8 + grp;
+          uint32_t b0 = 0, b1 = 0;
+          if (b < P.batch) {
+            const uint16_t *xr = P.x + size_t(b) * P.cols + col0;
+            b0 = __ldg(reinterpret_cast<const uint32_t *>(xr));
+            b1 = __ldg(reinterpret_cast<const uint32_t *>(xr + 8));
+          }
+          mma_bf16_16816(c[nt], a, b0, b1);
+        }
+      }
+    }
+    // end of a weight row: sum the 16 warps' partial products in a fixed order
+    if ((r + 1) % rpr == 0) {
+      float *mine = red + warp * 256;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        mine[grp * 16 + nt * 8 + 2 * tig] = c[nt][0];
+        mine[grp * 16 + nt * 8 + 2 * tig + 1] = c[nt][1];
+        mine[(grp + 8) * 16 + nt * 8 + 2 * tig] = c[nt][2];
+        mine[(grp + 8) * 16 + nt * 8 + 2 * tig + 1] = c[nt][3];
+        c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.0f;
+      }
+      __syncthreads();
+      if (threadIdx.x < 256) {
+        const uint32_t wr = threadIdx.x >> 4, b = threadIdx.x & 15;  // tile row = warp wr
+        float v = 0.0f;
+        for (uint32_t w = 0; w < kTcWarps; ++w) v += red[w * 256 + wr * 16 + b];
+        const uint64_t ch = uint64_t(blockIdx.x) * kTcWarps + wr;
+        const uint64_t row = ch * P.rows_per_chunk + (r / rpr);
+        if (ch < P.num_chunks && b < P.batch && row < P.rows) P.y[size_t(b) * P.rows + row] = v;
+      }
+      ++row_local;
+      if (have && !status && row_local < P.rows_per_chunk)
+        sc = bf16_bits_to_float(P.scales[row0 + row_local]);
+    }
+  }
+  if (have && !status) {
+    const bool ok = single ? (nwords == 0 && x == kRansL) : (q - R.off0 == 2 * nwords && x == kRansL);
+    if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
+  }
+  if (started) status |= R.drain();
+  if (lane == 0) report(P.status, status);
+}
+
 using GemvFn = void (*)(GemvParams);
 
 template <int FMT>
@@ -173,7 +346,7 @@ static GemvFn pick_b(uint32_t batch) {
   return rans_gemv_kernel<FMT, 16>;
 }
 
-static bool g_gemv_attr[64][2][5];
+static bool g_gemv_attr[64][2][6];
 
 }  // namespace eq
 
@@ -190,19 +363,23 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   if (t->run != 8 || t->streams != 32 || t->chunk_symbols % t->cols) return EQ_ERR_UNSUPPORTED;
   const uint32_t rpc = t->chunk_symbols / t->cols;
   if (rpc > 1 && t->cols % (t->streams * 8)) return EQ_ERR_UNSUPPORTED;
-  GemvFn fn = t->symfmt == EQ_SYM_E4M3 ? pick_b<EQ_SYM_E4M3>(batch) : pick_b<EQ_SYM_INT8>(batch);
+  // batch >= 8 on the tensor cores when a round never straddles a chunk's 256-column tiles
+  const bool tc = batch >= 8 && t->chunk_symbols % 256 == 0;
+  GemvFn fn = tc ? (t->symfmt == EQ_SYM_E4M3 ? rans_gemv_tc_kernel<EQ_SYM_E4M3> : rans_gemv_tc_kernel<EQ_SYM_INT8>)
+                 : (t->symfmt == EQ_SYM_E4M3 ? pick_b<EQ_SYM_E4M3>(batch) : pick_b<EQ_SYM_INT8>(batch));
   const uint64_t sms = uint64_t(device_sm_count());
   uint32_t warps = 16;
-  while (warps > 1 && (t->num_chunks + warps - 1) / warps < 4 * sms) warps >>= 1;
+  if (!tc)
+    while (warps > 1 && (t->num_chunks + warps - 1) / warps < 4 * sms) warps >>= 1;
   const uint64_t ctas = (t->num_chunks + warps - 1) / warps;
   if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  const int bi = batch <= 1 ? 0 : batch <= 2 ? 1 : batch <= 4 ? 2 : batch <= 8 ? 3 : 4;
+  const int bi = tc ? 5 : batch <= 1 ? 0 : batch <= 2 ? 1 : batch <= 4 ? 2 : 3;
   bool &attr = g_gemv_attr[dev][t->symfmt - 1][bi];
   if (!attr) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(rans_smem_bytes(16))) != cudaSuccess)
+                             int(tc ? gemv_tc_smem_bytes() : rans_smem_bytes(16))) != cudaSuccess)
       return EQ_ERR_CUDA;
     attr = true;
   }
@@ -224,6 +401,7 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   P.rounds_per_row = rpc > 1 ? t->cols / (t->streams * 8) : 0;
   P.batch = batch;
   P.warps = warps;
-  fn<<<uint32_t(ctas), 32 * warps, rans_smem_bytes(warps), static_cast<cudaStream_t>(stream)>>>(P);
+  fn<<<uint32_t(ctas), 32 * warps, tc ? gemv_tc_smem_bytes() : rans_smem_bytes(warps),
+       static_cast<cudaStream_t>(stream)>>>(P);
   return cuda_status(cudaGetLastError());
 }

@@ -55,11 +55,59 @@ struct HuffBuildArgs {
   uint16_t t[kHuffMaxTables][256];
 };
 
+// One code from the hierarchical tables, reading the 32 bits of w from the top.  Returns the
+// length (0 for a bad pattern) and the value in *sym.
+__device__ __forceinline__ uint32_t huff_tree_decode(const uint16_t *tree, uint32_t ntab, uint32_t w,
+                                                     uint32_t *sym) {
+  uint32_t e = tree[w >> 24], used = 0;
+  while ((e & 0x8000u) && e != kHuffInvalid) {
+    const uint32_t tab = e & 0xFFu;
+    used += 8;
+    if (tab >= ntab || used > 24) return 0;
+    e = tree[tab * 256 + ((w >> (24 - used)) & 0xFFu)];
+  }
+  const uint32_t rem = (e >> 8) & 0xFu;
+  if (e == kHuffInvalid || rem == 0 || rem > 8) return 0;
+  *sym = e & 0xFFu;
+  return used + rem;
+}
+
+// Copies the hierarchical tables and derives the 12-bit window table from them: window v lists
+// the codes that a greedy decode of the 12 bits v finds wholly inside them (at most 4).
 __global__ void __launch_bounds__(256) huff_build_kernel(const __grid_constant__ HuffBuildArgs a) {
+  __shared__ uint16_t tree[kHuffMaxTables * 256];
+  const uint32_t ntab = a.h.num_tables;
+  unsigned char *base = reinterpret_cast<unsigned char *>(a.dst);
+  uint16_t *gtree = reinterpret_cast<uint16_t *>(base + kHuffTreeOffset);
+  for (uint32_t i = threadIdx.x; i < ntab * 256; i += blockDim.x) {
+    tree[i] = a.t[i / 256][i % 256];
+    gtree[i] = tree[i];
+  }
   if (threadIdx.x == 0) *reinterpret_cast<HuffTableHeader *>(a.dst) = a.h;
-  uint16_t *out = reinterpret_cast<uint16_t *>(a.dst + sizeof(HuffTableHeader) / 4);
-  const uint16_t *src = &a.t[0][0];
-  for (uint32_t i = threadIdx.x; i < a.h.num_tables * 256; i += blockDim.x) out[i] = src[i];
+  __syncthreads();
+  uint64_t *win = reinterpret_cast<uint64_t *>(base + kHuffWindowOffset);
+  for (uint32_t v = threadIdx.x; v < kHuffWindow; v += blockDim.x) {
+    uint64_t entry = 0;
+    uint32_t pos = 0, n = 0;
+    while (n < 4) {
+      uint32_t sym = 0;
+      const uint32_t w = (v << (32 - kHuffWindowBits)) << pos;  // zeros past the window
+      const uint32_t len = huff_tree_decode(tree, ntab, w, &sym);
+      if (len == 0 || pos + len > kHuffWindowBits) {
+        // the first code needs bits past the window (or the pattern is bad, which the full
+        // decode on the real bits reports): the decoder takes the hierarchical path
+        if (n == 0) entry |= kHuffLong;
+        break;
+      }
+      entry |= uint64_t(sym) << (8 * n);
+      entry |= uint64_t(len) << (32 + 4 * n);
+      pos += len;
+      ++n;
+    }
+    entry |= uint64_t(pos) << 48;
+    entry |= uint64_t(n) << 52;
+    win[v] = entry;
+  }
 }
 
 // Hierarchical tables of a canonical code given by its lengths.  Returns EQ_OK and fills `a`.

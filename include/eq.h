@@ -112,7 +112,7 @@ typedef struct {
   uint64_t n;                  /* number of bf16 weights                                      */
   uint64_t total_bits;         /* length of the code stream in bits                           */
   uint32_t bytes_per_thread;   /* 8                                                           */
-  uint32_t threads_per_block;  /* 256                                                         */
+  uint32_t threads_per_block;  /* 32..512, a multiple of 32 (256 is the usual choice)          */
   const uint8_t *enc_exp;      /* EncodedExponent, threads * 8 bytes + 16 zero bytes           */
   const uint8_t *sign_mant;    /* PackedSignMantissa [n]                                      */
   const uint8_t *gaps;         /* ceil(5 threads / 8) bytes + 8 zero bytes                    */
@@ -132,9 +132,11 @@ size_t eq_table_bytes(eq_table_kind kind);
  *     and slot - cum[symbol].
  *   EQ_TABLE_HUFF: host_in[256] = code length of each exponent value (0 = absent), prob_bits
  *     ignored.  Builds the hierarchical lookup tables of the DFloat11 page ("Decodificacion
- *     basada en LUT jerarquicas"): the code tree is cut into height-8 subtrees, each a 256-entry
- *     table.  EQ_ERR_FORMAT if a length exceeds 32 or the lengths violate the Kraft inequality;
- *     EQ_ERR_UNSUPPORTED if more than 32 subtables would be needed.
+ *     basada en LUT jerarquicas": the code tree cut into height-8 subtrees, each a 256-entry
+ *     table) and, from them, a 4096-entry window table that returns every code lying wholly in
+ *     the next 12 bits (up to four) with one lookup.  EQ_ERR_FORMAT if a length exceeds 32 or the
+ *     lengths violate the Kraft inequality; EQ_ERR_UNSUPPORTED if more than 32 subtables would
+ *     be needed.
  */
 eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in, uint32_t prob_bits,
                           void *d_tables, void *stream);
@@ -155,7 +157,9 @@ eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uint16_t *cons
  * and never written to memory ("Float8@2bits" summary, closing section: fused decompression
  * kernels are the next step; the decoded values are consumed where they are produced).  W is
  * taken exactly as eq_decode would return it (bf16 of value * scale), products and sums in fp32.
- * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].  batch 1..16.
+ * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].  batch 1..16; for batch >= 8
+ * (and chunk_symbols % 256 == 0) the product of each 16-row x 256-column decoded tile with x runs
+ * on the tensor cores (mma, bf16 in, fp32 accumulate).
  * Requires run == 8, streams == 32 (one warp owns a chunk, so its sums never leave the warp)
  * and whole rows per chunk (chunk_symbols a multiple of cols); a chunk of several rows also needs
  * cols % 256 == 0, so that one decode round never straddles two rows.  Otherwise

@@ -127,7 +127,8 @@ def test_binding_gemv_and_huff_descriptors_pass_host_validation(eq, orc):
     w = synth.normal(8, 5120, 0.02, 4)
     sym, sc = orc.quantize(w, orc.E4M3)
     h = eq.codec.rans_encode(sym, sc, 1, wl.chunk_rows * 5120, wl.streams, wl.run)
-    t = eq.DeviceRans(h.rows, h.cols, 1, 12, h.chunk_symbols, h.streams, h.run, 2,
+    nchunks = (h.rows * h.cols) // h.chunk_symbols
+    t = eq.DeviceRans(h.rows, h.cols, 1, 12, h.chunk_symbols, h.streams, h.run, nchunks,
                       *[_FakeDev(1) for _ in range(5)])
     d = t.desc()
     fake = C.c_void_p(1 << 24)

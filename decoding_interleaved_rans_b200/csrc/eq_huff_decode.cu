@@ -8,12 +8,13 @@
 // buffer; the block then merges them with PackedSignMantissa and writes its span once, coalesced.
 //
 // Different from the page's kernel, for B200:
-//   * codes are read through a 12-bit window table that returns up to four whole codes per
-//     lookup (the common exponent codes are 2-3 bits long); codes longer than 12 bits fall back
-//     to the page's hierarchical 8-bit tables ("Decodificacion basada en LUT jerarquicas"), with
-//     16-bit entries so no exponent value has to be given up as a pointer;
-//   * blocks are persistent: each CTA loads the 32 KiB window table once and walks over many
-//     blocks of the stream;
+//   * codes are read through an 11-bit window table (16 KiB in shared memory) that returns up to
+//     four whole codes per lookup (the common exponent codes are 2-3 bits long); the rare codes
+//     longer than 11 bits fall back to the page's hierarchical 8-bit tables ("Decodificacion
+//     basada en LUT jerarquicas"), read through L1, with 16-bit entries so no exponent value has
+//     to be given up as a pointer;
+//   * blocks are persistent: each CTA loads the window table once and walks over many blocks of
+//     the stream, fetching the next block's bits while it merges the current one;
 //   * the block scan is a warp-shuffle scan rather than Blelloch's tree.
 #include <algorithm>
 
@@ -35,10 +36,8 @@ struct HuffParams {
   uint64_t blocks;
 };
 
-constexpr size_t kHuffTreeBytes = kHuffMaxTables * 256 * 2;
-
 __host__ __device__ constexpr size_t huff_smem_bytes(uint32_t tpb) {
-  return kHuffWindow * 8 + kHuffTreeBytes + size_t(tpb) * 64 + 16 + 66 * 4;
+  return kHuffWindow * 8 + size_t(tpb) * 64 + 16 + 66 * 4;
 }
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t v) { return __byte_perm(v, 0, 0x0123); }
@@ -50,12 +49,12 @@ __device__ __forceinline__ uint32_t bits32(uint32_t r0, uint32_t r1, uint32_t r2
 
 __device__ __forceinline__ uint32_t tree_decode(const uint16_t *tree, uint32_t ntab, uint32_t w,
                                                 uint32_t *sym) {
-  uint32_t e = tree[w >> 24], used = 0;
+  uint32_t e = __ldg(tree + (w >> 24)), used = 0;
   while ((e & 0x8000u) && e != kHuffInvalid) {
     const uint32_t tab = e & 0xFFu;
     used += 8;
     if (tab >= ntab || used > 24) return 0;
-    e = tree[tab * 256 + ((w >> (24 - used)) & 0xFFu)];
+    e = __ldg(tree + tab * 256 + ((w >> (24 - used)) & 0xFFu));
   }
   const uint32_t rem = (e >> 8) & 0xFu;
   if (e == kHuffInvalid || rem == 0 || rem > 8) return 0;
@@ -129,9 +128,9 @@ __global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant_
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t T = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t *win = reinterpret_cast<uint64_t *>(smem);
-  uint16_t *tree = reinterpret_cast<uint16_t *>(smem + kHuffWindow * 8);
-  uint8_t *ebuf = smem + kHuffWindow * 8 + kHuffTreeBytes;
+  uint8_t *ebuf = smem + kHuffWindow * 8;
   uint32_t *wsum = reinterpret_cast<uint32_t *>(ebuf + T * 64 + 16);
+  const uint16_t *tree = reinterpret_cast<const uint16_t *>(P.table + kHuffTreeOffset);
 
   const HuffTableHeader hdr = *reinterpret_cast<const HuffTableHeader *>(P.table);
   if (hdr.magic != kHuffMagic || hdr.num_tables == 0 || hdr.num_tables > kHuffMaxTables) {
@@ -142,28 +141,35 @@ __global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant_
   {
     const uint4 *w4 = reinterpret_cast<const uint4 *>(P.table + kHuffWindowOffset);
     for (uint32_t i = tid; i < kHuffWindow / 2; i += T) reinterpret_cast<uint4 *>(win)[i] = __ldg(w4 + i);
-    const uint4 *t4 = reinterpret_cast<const uint4 *>(P.table + kHuffTreeOffset);
-    for (uint32_t i = tid; i < ntab * 32; i += T) reinterpret_cast<uint4 *>(tree)[i] = __ldg(t4 + i);
   }
   __syncthreads();
 
-  uint32_t err = 0;
-  for (uint64_t b = blockIdx.x; b < P.blocks; b += gridDim.x) {
-    // ---- this thread's 64-bit segment plus the 32 bits after it ----
+  // a thread's 64-bit segment plus the 32 bits after it, and its Gap
+  auto fetch = [&](uint64_t b, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &g) {
     const uint64_t t = b * T + tid;
-    uint32_t r0 = 0, r1 = 0, r2 = 0, pos = 0, end = 0;
-    if (t < P.threads) {
+    r0 = r1 = r2 = g = 0;
+    if (b < P.blocks && t < P.threads) {
       const uint32_t *src = reinterpret_cast<const uint32_t *>(P.enc + 8 * t);
-      r0 = bswap32(__ldg(src));
-      r1 = bswap32(__ldg(src + 1));
-      r2 = bswap32(__ldg(src + 2));
+      r0 = __ldg(src);
+      r1 = __ldg(src + 1);
+      r2 = __ldg(src + 2);
       const uint64_t gbit = 5 * t;
-      const uint32_t g2 = uint32_t(__ldg(P.gaps + (gbit >> 3))) |
-                          (uint32_t(__ldg(P.gaps + (gbit >> 3) + 1)) << 8);
-      pos = (g2 >> (gbit & 7)) & 31u;
+      g = (uint32_t(__ldg(P.gaps + (gbit >> 3))) | (uint32_t(__ldg(P.gaps + (gbit >> 3) + 1)) << 8)) >>
+          (gbit & 7);
+    }
+  };
+  uint32_t err = 0;
+  uint32_t n0, n1, n2, ng;
+  fetch(blockIdx.x, n0, n1, n2, ng);
+  for (uint64_t b = blockIdx.x; b < P.blocks; b += gridDim.x) {
+    const uint64_t t = b * T + tid;
+    const uint32_t r0 = bswap32(n0), r1 = bswap32(n1), r2 = bswap32(n2);
+    uint32_t pos = ng & 31u, end = 0;
+    if (t < P.threads) {
       const uint64_t left = P.total_bits - 64 * t;
       end = left < 64 ? uint32_t(left) : 64u;
     }
+    fetch(b + gridDim.x, n0, n1, n2, ng);  // next block's bits, in flight during this one
     // ---- stage 1: count ----
     uint32_t bad = 0;
     const uint32_t cnt = segment<false>(win, tree, ntab, r0, r1, r2, pos, end, nullptr, &bad);

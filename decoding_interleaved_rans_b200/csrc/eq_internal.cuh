@@ -34,8 +34,8 @@ constexpr uint32_t kRansFlagSingle = 4u;      // one symbol owns every slot
 constexpr size_t kRansTableBytes = sizeof(RansTableHeader) + kRansSlots * 4;
 
 // Huffman (DFloat11 exponent): 16-byte header, then
-//   a window table W: 4096 x uint64, indexed by the next 12 code bits, listing the codes that lie
-//   wholly inside those 12 bits (up to 4): bits 8i..8i+7 value of code i, bits 32+4i..35+4i its
+//   a window table W: 2048 x uint64, indexed by the next 11 code bits, listing the codes that lie
+//   wholly inside those 11 bits (up to 4): bits 8i..8i+7 value of code i, bits 32+4i..35+4i its
 //   length, bits 48..51 their total length, bits 52..54 how many (0 = no code fits, which is a
 //   bad pattern unless bit 63 says the first code is longer than 12 bits);
 //   then up to kHuffMaxTables hierarchical tables of 256 uint16 entries for codes of any length:
@@ -44,7 +44,7 @@ constexpr size_t kRansTableBytes = sizeof(RansTableHeader) + kRansSlots * 4;
 //     a pointer (bit 15 set):   bits 7..0 index of the child table, which reads the next 8 bits
 //     0xFFFF: no code starts with this bit pattern.
 constexpr uint32_t kHuffMaxTables = 32;
-constexpr uint32_t kHuffWindowBits = 12;
+constexpr uint32_t kHuffWindowBits = 11;
 constexpr uint32_t kHuffWindow = 1u << kHuffWindowBits;
 constexpr uint64_t kHuffLong = 1ull << 63;
 struct HuffTableHeader {

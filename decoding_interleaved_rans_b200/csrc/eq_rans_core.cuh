@@ -29,6 +29,8 @@ struct WordRing {
   uint32_t nseg;
   uint32_t issued;  // segments handed to the copy engine
   uint32_t ready;   // segments waited for
+  uint32_t ready_end;  // offsets below this have landed (ready segments)
+  uint32_t refill_at;  // once q reaches this offset a slot can be refilled
 
   __device__ __forceinline__ void issue(uint32_t lane) {
     if (lane == 0) {
@@ -39,6 +41,7 @@ struct WordRing {
       bulk_g2s(buf + slot * kSegBytes, A + size_t(s) * kSegBytes, bytes, &bar[slot]);
     }
     ++issued;
+    refill_at = issued < nseg ? (issued - kNumSeg + 1) * kSegBytes : 0xFFFFFFFFu;
   }
 
   // point the ring at words [w0, w0 + nwords) and start the first copies
@@ -51,6 +54,8 @@ struct WordRing {
     nseg = (span + kSegBytes - 1) / kSegBytes;
     issued = 0;
     ready = 0;
+    ready_end = 0;
+    refill_at = 0xFFFFFFFFu;
     while (issued < min(nseg, kNumSeg)) issue(lane);
   }
 
@@ -62,7 +67,17 @@ struct WordRing {
       if (!mbar_wait_bounded(&bar[ready % kNumSeg], (ready / kNumSeg) & 1u)) return false;
       ++ready;
     }
+    ready_end = ready * kSegBytes;
     return true;
+  }
+
+  // the per-round checks: wait only when the round may read past the landed bytes, refill only
+  // when a slot has been used up
+  __device__ __forceinline__ bool round_wait(uint32_t q) {
+    return (q + 2 * kRoundWords <= ready_end || ready >= nseg) ? true : wait_below(q + 2 * kRoundWords);
+  }
+  __device__ __forceinline__ void round_refill(uint32_t q, uint32_t lane) {
+    if (q >= refill_at) refill(q, lane);
   }
 
   // hand out the slots of segments lying wholly below offset q

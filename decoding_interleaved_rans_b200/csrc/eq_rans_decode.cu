@@ -35,6 +35,7 @@ struct RansDesc {
   uint64_t numel;
   uint64_t units;         // num_chunks * groups: one warp each
   uint64_t row_magic;     // floor(j / cols) = __umul64hi(j, row_magic) (0: cols == 1)
+  uint32_t rows, cols;
   uint32_t chunk_symbols;
   uint32_t groups;        // streams / 32
   uint32_t cta_begin;     // first CTA of this tensor in the launch
@@ -55,22 +56,13 @@ template <bool FULL, int G, int FMT>
 __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
                                              const uint32_t *lut, const unsigned char *smem,
                                              const WordRing &R, uint32_t &q, uint32_t lt,
-                                             uint64_t jrun, bool nan_codes) {
+                                             uint16_t *out, float sc, bool nan_codes) {
   uint32_t e[G];
 #pragma unroll
   for (int p = 0; p < G; ++p) e[p] = rans_step<FULL>(x, act, lut, smem, R.ring_off, q, lt);
   if (FULL || act) {
-    const float sc = bf16_bits_to_float(D.scales[div_by_magic(jrun, D.row_magic)]);
-    if constexpr (G == 8) {
-      uint4 o;
-      o.x = dequant2<FMT>(sym_pair(e[0], e[1]), sc, nan_codes);
-      o.y = dequant2<FMT>(sym_pair(e[2], e[3]), sc, nan_codes);
-      o.z = dequant2<FMT>(sym_pair(e[4], e[5]), sc, nan_codes);
-      o.w = dequant2<FMT>(sym_pair(e[6], e[7]), sc, nan_codes);
-      *reinterpret_cast<uint4 *>(D.out + jrun) = o;
-    } else {
-      D.out[jrun] = dequant1<FMT>((e[0] >> 12) & 0xFFu, sc);
-    }
+    if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT>(e, sc, nan_codes);
+    else *out = dequant1<FMT>((e[0] >> 12) & 0xFFu, sc);
   }
 }
 
@@ -112,20 +104,34 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   // rounds in which all 32 lanes of this group hold a run
   const uint32_t full = runs >= 32 * g + 32 ? (runs - 32 * g - 32) / S + 1 : 0;
   uint32_t q = R.off0;
+  // the lane's first output and its row; both advance by S runs per round
+  uint64_t jrun = j0 + uint64_t(s) * G;
+  const uint32_t step = S * G, cols = D.cols;
+  uint64_t row = div_by_magic(jrun, D.row_magic);
+  uint32_t col = uint32_t(jrun - row * cols);
+  float sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+  uint16_t *out = D.out + jrun;
   for (uint32_t r = 0; r < rounds; ++r) {
-    if (!R.wait_below(q + 2 * kRoundWords)) {
+    if (!R.round_wait(q)) {
       status |= EQ_DEV_TIMEOUT;
       break;
     }
-    const uint32_t run = r * S + s;
-    const uint64_t jrun = j0 + uint64_t(run) * G;
-    if (r < full) decode_round<true, G, FMT>(D, x, true, lut, smem, R, q, lt, jrun, nan_codes);
-    else decode_round<false, G, FMT>(D, x, run < runs, lut, smem, R, q, lt, jrun, nan_codes);
+    if (r < full) decode_round<true, G, FMT>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
+    else decode_round<false, G, FMT>(D, x, r * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
     if (q - R.off0 > 2 * nwords) {
       status |= EQ_DEV_OVERRUN;
       break;
     }
-    R.refill(q, lane);
+    R.round_refill(q, lane);
+    out += step;
+    col += step;
+    if (col >= cols) {
+      do {
+        col -= cols;
+        ++row;
+      } while (col >= cols);
+      if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
+    }
   }
   if (!status && !__all_sync(0xFFFFFFFFu, q - R.off0 == 2 * nwords && x == kRansL))
     status |= EQ_DEV_CORRUPT_STATE;
@@ -243,6 +249,8 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
       D.groups = t.streams / 32;
       D.units = t.num_chunks * D.groups;
       D.row_magic = div_magic(t.cols);
+      D.rows = t.rows;
+      D.cols = t.cols;
       D.chunk_symbols = t.chunk_symbols;
       D.cta_begin = uint32_t(ctas);
       D.pad = 0;

@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
     if (single) {
       pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
     } else {
-      if (!R.wait_below(q + 2 * kRoundWords)) {
+      if (!R.round_wait(q)) {
         status |= EQ_DEV_TIMEOUT;
         break;
       }
@@ -130,7 +130,7 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
         status |= EQ_DEV_OVERRUN;
         break;
       }
-      R.refill(q, lane);
+      R.round_refill(q, lane);
     }
     if (act) {  // the weights exactly as eq_decode writes them, times the activations
       const uint32_t col = (r * S + lane) * 8 - row_local * P.cols;
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __gri
     const bool act = have && !status && r * S + lane < runs;
     uint32_t pr[4] = {0u, 0u, 0u, 0u};
     if (live) {
-      if (!R.wait_below(q + 2 * kRoundWords)) {
+      if (!R.round_wait(q)) {
         status |= EQ_DEV_TIMEOUT;
         live = false;
       } else {
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __gri
           status |= EQ_DEV_OVERRUN;
           live = false;
         } else {
-          R.refill(q, lane);
+          R.round_refill(q, lane);
         }
       }
     } else if (single) {

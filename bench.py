@@ -34,6 +34,35 @@ WORKLOAD = "int8_8k"
 METRIC = "decoded params/s (rANS decode to bf16)"
 
 
+KERNEL_SOURCES = {
+    "rans_decode_kernel": ["eq_rans_decode.cu", "eq_rans_core.cuh", "eq_dequant.cuh",
+                           "eq_internal.cuh"],
+    "huff_decode_kernel": ["eq_huff_decode.cu", "eq_internal.cuh"],
+    "rans_gemv_kernel": ["eq_rans_gemv.cu", "eq_rans_core.cuh", "eq_dequant.cuh",
+                         "eq_internal.cuh"],
+}
+
+
+def kernel_sources_sha(kernel: str) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "decoding_interleaved_rans_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, units: int):
+    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json), scaled to
+    `units` weights; None when the kernel's sources changed since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(kernel)
+    if not rec or rec.get("sources_sha256") != kernel_sources_sha(kernel):
+        return None
+    return rec["dram_bytes_per_launch"] * units / rec["weights_per_launch"]
+
+
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -122,35 +151,23 @@ class ClockSampler:
 
 def dist_setup():
     import torch
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
 
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+    from decoding_interleaved_rans_b200 import dist
+    world, rank, local = dist.env_rank()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init("nccl", timeout_s=120, device=torch.device("cuda", local))
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    from decoding_interleaved_rans_b200 import dist
+    dist.barrier()
 
 
 def max_over_ranks(world, v: float) -> float:
-    if world == 1:
-        return v
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from decoding_interleaved_rans_b200 import dist
+    return dist.max_over_ranks(v, device="cuda")
 
 
 def prepare_rans(eq, wl_name: str):
@@ -263,8 +280,9 @@ def run_ours(args):
                    "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{world}"},
         "gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "peak_src": peaks["src"], "kernel": "rans_decode_kernel<4,8,INT8>",
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": measured_traffic("rans_decode_kernel", numel),
+                     "peak_src": peaks["src"], "kernel": "rans_decode_kernel<run 8, Int8>",
                      "alg_bytes_per_launch": alg_bytes},
         "e2e": {"value": numel * world / e2e_s, "unit": "params/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
@@ -453,9 +471,8 @@ def main():
     else:
         run_ours(args)
     if int(os.environ.get("WORLD_SIZE", "1")) > 1:
-        import torch.distributed as dist
-        if dist.is_initialized():
-            dist.destroy_process_group()
+        from decoding_interleaved_rans_b200 import dist
+        dist.shutdown()
 
 
 if __name__ == "__main__":

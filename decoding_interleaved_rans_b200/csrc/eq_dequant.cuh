@@ -49,25 +49,6 @@ __device__ __forceinline__ uint32_t dequant2(uint32_t pair, float scale, bool na
   return o;
 }
 
-// Int8 scale prepared once per row for the exact magic-number product below:
-//   s12 = scale * 2^-12 (exact: a bf16 scale has 8 significant bits and is >= 2^-133) and
-//   c = -(2^11 + 2^7) * scale (exact: at most 13 significant bits).  plain: rows whose scale is
-//   not positive (a zero product must keep the sign the plain product gives) or so large that c
-//   would overflow take the plain conversion.
-struct Int8Scale {
-  float s, s12, c;
-  bool big;
-};
-
-__device__ __forceinline__ Int8Scale int8_scale(float s) {
-  Int8Scale r;
-  r.s = s;
-  r.s12 = s * 0.000244140625f;
-  r.c = -2176.0f * s;
-  r.big = !(s > 0.0f && s < 1.0e30f);
-  return r;
-}
-
 // the eight symbols of a round, taken from their slot-table entries (symbol in bits 19..12),
 // scaled -> eight bf16 (one 16-byte store)
 template <int FMT>
@@ -84,22 +65,6 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, b
       const uint32_t pair = ((e[2 * k] >> 12) & 0xFFu) | ((e[2 * k + 1] >> 4) & 0xFF00u);
       o[k] = dequant2<FMT>(pair, scale, nan_codes);
     }
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-// Int8 without a conversion instruction: with u = byte ^ 0x80 = v + 128, the float whose bits are
-// 0x4B000000 | u << 12 is 2^23 + 4096 (v + 128); times s12 plus c that is exactly v * scale (the
-// fused multiply-add rounds once and the true result has at most 15 significant bits), then one
-// rounding to bf16.  The entry's symbol already sits at bits 19..12.
-__device__ __forceinline__ uint4 dequant8_int8(const uint32_t (&e)[8], const Int8Scale &sc) {
-  if (sc.big) return dequant8<EQ_SYM_INT8>(e, sc.s, false);
-  uint32_t o[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float f0 = __uint_as_float((e[2 * k] & 0xFF000u) ^ 0x4B080000u);
-    const float f1 = __uint_as_float((e[2 * k + 1] & 0xFF000u) ^ 0x4B080000u);
-    o[k] = pack_bf16x2(fmaf(f0, sc.s12, sc.c), fmaf(f1, sc.s12, sc.c));
   }
   return make_uint4(o[0], o[1], o[2], o[3]);
 }

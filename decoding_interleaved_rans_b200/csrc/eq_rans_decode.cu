@@ -56,17 +56,13 @@ template <bool FULL, int G, int FMT>
 __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
                                              const uint32_t *lut, const unsigned char *smem,
                                              const WordRing &R, uint32_t &q, uint32_t lt,
-                                             uint16_t *out, const Int8Scale &sc, bool nan_codes) {
+                                             uint16_t *out, float sc, bool nan_codes) {
   uint32_t e[G];
 #pragma unroll
   for (int p = 0; p < G; ++p) e[p] = rans_step<FULL>(x, act, lut, smem, R.ring_off, q, lt);
   if (FULL || act) {
-    if constexpr (G == 8) {
-      if constexpr (FMT == EQ_SYM_INT8) *reinterpret_cast<uint4 *>(out) = dequant8_int8(e, sc);
-      else *reinterpret_cast<uint4 *>(out) = dequant8<FMT>(e, sc.s, nan_codes);
-    } else {
-      *out = dequant1<FMT>((e[0] >> 12) & 0xFFu, sc.s);
-    }
+    if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT>(e, sc, nan_codes);
+    else *out = dequant1<FMT>((e[0] >> 12) & 0xFFu, sc);
   }
 }
 
@@ -113,7 +109,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   const uint32_t step = S * G, cols = D.cols;
   uint64_t row = div_by_magic(jrun, D.row_magic);
   uint32_t col = uint32_t(jrun - row * cols);
-  Int8Scale sc = int8_scale(bf16_bits_to_float(D.scales[row < D.rows ? row : 0]));
+  float sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
   uint16_t *out = D.out + jrun;
   for (uint32_t r = 0; r < rounds; ++r) {
     if (!R.round_wait(q)) {
@@ -134,7 +130,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
         col -= cols;
         ++row;
       } while (col >= cols);
-      if (row < D.rows) sc = int8_scale(bf16_bits_to_float(D.scales[row]));
+      if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
     }
   }
   if (!status && !__all_sync(0xFFFFFFFFu, q - R.off0 == 2 * nwords && x == kRansL))

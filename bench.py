@@ -318,6 +318,27 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                 "bits_per_param": 8 * dh.compressed_bytes / dh.n,
                 "kernel": "huff_decode_kernel"})
     del dh, ob
+    # GPU compressor: fp32 weights in HBM -> quantise, histogram, frequency table (host), rANS
+    # plan + encode; wall clock around the whole call (it reads the word total back once)
+    wl = synth.WORKLOADS["int8_8k"]
+    wdev = torch.from_numpy(wl.tensors[0].generate()).to(dev)
+    times_c = []
+    for it in range(4):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        sym, sc = eq.quantize_device(wdev, eq.EQ_SYM_INT8, wl.int8_div)
+        tc = eq.rans_encode_device(sym, sc, eq.EQ_SYM_INT8, wl.chunk_symbols, wl.streams, wl.run)
+        torch.cuda.synchronize()
+        if it:
+            times_c.append(time.perf_counter() - t0)
+    sec = statistics.mean(times_c)
+    n_c = wdev.numel()
+    out.append({"what": "GPU compression (quantise + histogram + rANS plan + encode), Int8 8192x8192",
+                "params": n_c, "ms": sec * 1e3, "params_per_s": n_c / sec,
+                "projected_70B_s": 70e9 / (n_c / sec),
+                "pages_claim": "70B compressed in < 10 min (summaries) / < 30 min (abstract)",
+                "kernel": "quantize_kernel + histogram_kernel + rans_encode_kernel x2"})
+    del wdev, sym, sc, tc
     # fused decode + GEMV over the three 13B MLP weights (gate, up 13824x5120; down 5120x13824);
     # algorithmic bytes = the coded weights read (+ x and y)
     wl = synth.WORKLOADS["mlp_13b"]

@@ -22,7 +22,9 @@ EQ_ABI_VERSION = 1
 EXPORTS = ("eq_table_bytes", "eq_build_tables", "eq_decode", "eq_decode_gemv",
            "eq_huff_bf16_decode", "eq_status_string", "eq_abi_version", "eq_quantize_host",
            "eq_rans_freqs_host", "eq_rans_encode_host", "eq_huff_lengths_host",
-           "eq_huff_plan_host", "eq_huff_encode_host", "eq_free_host")
+           "eq_huff_plan_host", "eq_huff_encode_host", "eq_free_host", "eq_rans_normalize_host",
+           "eq_quantize_device",
+           "eq_histogram_device", "eq_rans_plan_device", "eq_rans_encode_device")
 
 
 class EqError(RuntimeError):
@@ -80,6 +82,11 @@ def lib() -> C.CDLL:
                 "eq_huff_plan_host": (i32, [p, u64, p, C.POINTER(C.c_uint64)]),
                 "eq_huff_encode_host": (i32, [p, u64, p, u32, u64, p, p, p, p]),
                 "eq_free_host": (None, [p]),
+                "eq_rans_normalize_host": (i32, [p, u32, p]),
+                "eq_quantize_device": (i32, [p, u32, u32, u32, C.c_float, p, p, p]),
+                "eq_histogram_device": (i32, [p, u64, p, p]),
+                "eq_rans_plan_device": (i32, [p, u32, u32, p, u32, u32, u32, p, p, p, p]),
+                "eq_rans_encode_device": (i32, [p, u32, u32, p, u32, u32, u32, p, p, p, p]),
             }
             for name, (res, args) in sig.items():
                 f = getattr(L, name)

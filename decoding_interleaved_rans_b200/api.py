@@ -194,3 +194,67 @@ def huff_bf16_decode(h: DeviceHuff, out=None, status=None, stream=None):
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Raw uint16 patterns of a bf16 tensor (device or host)."""
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU compressor (include/eq_encode.h, *_device calls)
+# ------------------------------------------------------------------------------------------------
+
+def quantize_device(w: torch.Tensor, symfmt: int, int8_div: float = 0.0, stream=None):
+    """Per-row AbsMax quantisation on the GPU: fp32 [rows, cols] -> (uint8 symbols, bf16 scales
+    as int16 bits)."""
+    assert w.dtype == torch.float32 and w.is_cuda and w.is_contiguous() and w.dim() == 2
+    rows, cols = w.shape
+    sym = torch.empty(rows, cols, dtype=torch.uint8, device=w.device)
+    sc = torch.empty(rows, dtype=torch.int16, device=w.device)
+    L.check(L.lib().eq_quantize_device(_ptr(w), rows, cols, symfmt, float(int8_div), _ptr(sym),
+                                       _ptr(sc), _stream(stream)), "eq_quantize_device")
+    return sym, sc
+
+
+def histogram_device(sym: torch.Tensor, stream=None) -> torch.Tensor:
+    counts = torch.zeros(256, dtype=torch.int32, device=sym.device)
+    L.check(L.lib().eq_histogram_device(_ptr(sym), sym.numel(), _ptr(counts), _stream(stream)),
+            "eq_histogram_device")
+    return counts
+
+
+def normalize_freqs(counts, prob_bits: int = 12) -> np.ndarray:
+    c = np.ascontiguousarray(np.asarray(counts).astype(np.uint64))
+    f = np.zeros(256, np.uint32)
+    L.check(L.lib().eq_rans_normalize_host(c.ctypes.data, prob_bits, f.ctypes.data),
+            "eq_rans_normalize_host")
+    return f
+
+
+def rans_encode_device(sym: torch.Tensor, scales: torch.Tensor, symfmt: int, chunk_symbols: int,
+                       streams: int, run: int, freqs=None, status=None,
+                       stream=None) -> "DeviceRans":
+    """Encode a device symbol matrix on the GPU into a DeviceRans (plan, offsets, encode)."""
+    assert sym.dtype == torch.uint8 and sym.is_cuda and sym.is_contiguous() and sym.dim() == 2
+    rows, cols = sym.shape
+    dev = sym.device
+    if freqs is None:
+        freqs = normalize_freqs(histogram_device(sym, stream).cpu().numpy())
+    f = (C.c_uint32 * 256)(*[int(v) for v in np.asarray(freqs).ravel()[:256]])
+    chunk = chunk_symbols if chunk_symbols else cols
+    nchunks = (rows * cols + chunk - 1) // chunk
+    units = nchunks * (streams // 32)
+    states = torch.empty(max(1, nchunks * streams), dtype=torch.int32, device=dev)
+    word_off = torch.empty(units + 1, dtype=torch.int64, device=dev)
+    if status is None:
+        status = new_status(dev)
+    L.check(L.lib().eq_rans_plan_device(_ptr(sym), rows, cols, f, chunk_symbols, streams, run,
+                                        _ptr(states), _ptr(word_off), _ptr(status),
+                                        _stream(stream)), "eq_rans_plan_device")
+    total = int(word_off[-1].item())
+    words = torch.zeros(max(8, (total + 7) // 8 * 8), dtype=torch.int16, device=dev)
+    L.check(L.lib().eq_rans_encode_device(_ptr(sym), rows, cols, f, chunk_symbols, streams, run,
+                                          _ptr(word_off), _ptr(words), _ptr(status),
+                                          _stream(stream)), "eq_rans_encode_device")
+    t = DeviceRans(rows, cols, symfmt, 12, chunk_symbols, streams, run, nchunks,
+                   states[:nchunks * streams] if nchunks else states, word_off, words,
+                   scales, torch.empty(table_bytes(L.EQ_TABLE_RANS), dtype=torch.uint8,
+                                       device=dev))
+    build_tables(L.EQ_TABLE_RANS, freqs, 12, t.tables, stream)
+    return t

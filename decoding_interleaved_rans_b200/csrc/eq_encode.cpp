@@ -101,12 +101,12 @@ extern "C" eq_status eq_quantize_host(const float *w, uint32_t rows, uint32_t co
   return EQ_OK;
 }
 
-extern "C" eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t prob_bits,
-                                        uint32_t *freqs) {
-  if (!freqs || (n && !sym) || prob_bits < 8 || prob_bits > 15) return EQ_ERR_ARG;
+extern "C" eq_status eq_rans_normalize_host(const uint64_t *counts, uint32_t prob_bits,
+                                            uint32_t *freqs) {
+  if (!counts || !freqs || prob_bits < 8 || prob_bits > 15) return EQ_ERR_ARG;
   const uint64_t M = 1ull << prob_bits;
-  uint64_t cnt[256] = {0};
-  for (uint64_t i = 0; i < n; ++i) ++cnt[sym[i]];
+  uint64_t n = 0;
+  for (int s = 0; s < 256; ++s) n += counts[s];
   std::fill(freqs, freqs + 256, 0u);
   if (n == 0) {
     freqs[0] = uint32_t(M);
@@ -115,9 +115,9 @@ extern "C" eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t
   int top = 0;
   uint64_t total = 0;
   for (int s = 0; s < 256; ++s) {
-    if (cnt[s] > cnt[top]) top = s;
-    if (!cnt[s]) continue;
-    const uint64_t f = std::max<uint64_t>(1, uint64_t((static_cast<unsigned __int128>(cnt[s]) * M) / n));
+    if (counts[s] > counts[top]) top = s;
+    if (!counts[s]) continue;
+    const uint64_t f = std::max<uint64_t>(1, uint64_t((static_cast<unsigned __int128>(counts[s]) * M) / n));
     freqs[s] = uint32_t(f);
     total += f;
   }
@@ -129,6 +129,14 @@ extern "C" eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t
     --freqs[big];
   }
   return EQ_OK;
+}
+
+extern "C" eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t prob_bits,
+                                        uint32_t *freqs) {
+  if (!freqs || (n && !sym)) return EQ_ERR_ARG;
+  uint64_t cnt[256] = {0};
+  for (uint64_t i = 0; i < n; ++i) ++cnt[sym[i]];
+  return eq_rans_normalize_host(cnt, prob_bits, freqs);
 }
 
 extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint32_t cols,

@@ -4,9 +4,10 @@
  *
  * The pages compress once, offline, then keep the weights coded in GPU memory ("Float8@2bits"
  * summary, "Codificacion de Pesos": per-channel AbsMax scales, Float8/Int8 symbols, ANS over the
- * flattened stream; DFloat11 page, "Formato DFloat11": Huffman-coded bf16 exponents).  These calls
- * run on the host CPU with worker threads; none of them touches the GPU.  The formats are the ones
- * defined in eq.h.  Arrays are host memory owned by the caller unless stated otherwise.
+ * flattened stream; DFloat11 page, "Formato DFloat11": Huffman-coded bf16 exponents).  The *_host
+ * calls run on the host CPU with worker threads and touch no GPU; the *_device calls at the end
+ * run the rANS side on the GPU.  The formats are the ones defined in eq.h.  Arrays of the host
+ * calls are host memory owned by the caller unless stated otherwise.
  */
 #ifndef EQ_ENCODE_H
 #define EQ_ENCODE_H
@@ -38,6 +39,9 @@ eq_status eq_quantize_host(const float *w, uint32_t rows, uint32_t cols, uint32_
  */
 eq_status eq_rans_freqs_host(const uint8_t *sym, uint64_t n, uint32_t prob_bits, uint32_t *freqs);
 
+/* The same normalisation from 256 symbol counts (e.g. those of eq_histogram_device). */
+eq_status eq_rans_normalize_host(const uint64_t *counts, uint32_t prob_bits, uint32_t *freqs);
+
 /*
  * Interleaved-rANS encoding of a symbol matrix sym[rows][cols] in the format of eq_rans_tensor.
  * chunk_symbols = 0 means one row per chunk.  states: [num_chunks * streams]; word_off:
@@ -68,6 +72,35 @@ eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const uint32_t *len
 
 /* Release a buffer returned by eq_rans_encode_host. */
 void eq_free_host(void *p);
+
+/*
+ * The same compressor on the GPU: every pointer below is device memory owned by the caller,
+ * every call is asynchronous on `stream` and allocates nothing.  The results are bit-identical
+ * to the host calls above.
+ *
+ * eq_quantize_device: as eq_quantize_host (one CTA per row).
+ * eq_histogram_device: d_counts[256] += the number of each byte value among d_sym[0 .. n)
+ *   (zero d_counts first).
+ * eq_rans_plan_device: encodes every chunk once to learn the final states (d_states,
+ *   [num_chunks * streams]) and each substream's word count, then turns the counts into the
+ *   offsets d_word_off ([num_chunks * streams / 32 + 1]; d_word_off[last] = total words).
+ * eq_rans_encode_device: encodes again and writes the words at those offsets into d_words (room
+ *   for d_word_off[last] words, rounded up to a multiple of 8 and zero-filled by the caller).
+ * host_freqs: the frequency table (host memory, 256 entries summing to 4096).  A symbol without
+ * frequency sets EQ_DEV_BAD_CODE in *d_status; a word count that does not match the plan sets
+ * EQ_DEV_COUNT_MISMATCH.
+ */
+eq_status eq_quantize_device(const float *d_w, uint32_t rows, uint32_t cols, uint32_t symfmt,
+                             float int8_div, uint8_t *d_sym, uint16_t *d_scales, void *stream);
+eq_status eq_histogram_device(const uint8_t *d_sym, uint64_t n, uint32_t *d_counts, void *stream);
+eq_status eq_rans_plan_device(const uint8_t *d_sym, uint32_t rows, uint32_t cols,
+                              const uint32_t *host_freqs, uint32_t chunk_symbols, uint32_t streams,
+                              uint32_t run, uint32_t *d_states, uint64_t *d_word_off,
+                              uint32_t *d_status, void *stream);
+eq_status eq_rans_encode_device(const uint8_t *d_sym, uint32_t rows, uint32_t cols,
+                                const uint32_t *host_freqs, uint32_t chunk_symbols,
+                                uint32_t streams, uint32_t run, const uint64_t *d_word_off,
+                                uint16_t *d_words, uint32_t *d_status, void *stream);
 
 #ifdef __cplusplus
 }

@@ -84,3 +84,14 @@ def test_huff_lengths_optimal_and_capped(eq, orc):
     a = eq.codec.huff_lengths(counts, 32)
     b = orc.huff_lengths(counts, 32)
     assert a.max() <= 32 and np.array_equal(a, b.astype(np.uint32))
+
+
+def test_normalize_from_counts_matches_oracle(eq, orc):
+    rng = np.random.default_rng(3)
+    for _ in range(50):
+        counts = np.zeros(256, np.uint64)
+        k = int(rng.integers(1, 257))
+        counts[rng.choice(256, k, replace=False)] = rng.integers(1, 10 ** 7, k).astype(np.uint64)
+        f = np.zeros(256, np.uint32)
+        assert orc.lib().orc_rans_normalize(counts.ctypes.data, 12, f.ctypes.data) == 0
+        assert np.array_equal(eq.normalize_freqs(counts), f)

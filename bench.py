@@ -339,6 +339,43 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                 "pages_claim": "70B compressed in < 10 min (summaries) / < 30 min (abstract)",
                 "kernel": "quantize_kernel + histogram_kernel + rans_encode_kernel x2"})
     del wdev, sym, sc, tc
+    # block-by-block decode overlapped with the block's forward GEMMs (4 LLaMA-2-7B-shaped layers,
+    # coded on the GPU): compute alone on resident bf16 weights, decode then compute, overlapped
+    from decoding_interleaved_rans_b200.pipeline import BlockPipeline
+    wl7 = synth.scaled(synth.WORKLOADS["llama2_7b"], layers=4)
+    blocks, resident = [], []
+    for layer in range(4):
+        hs, rs = [], []
+        for spec in [t for t in wl7.tensors if t.name.startswith(f"layers.{layer}.")]:
+            wt = torch.from_numpy(spec.generate()).to(dev)
+            sym, sc = eq.quantize_device(wt, eq.EQ_SYM_E4M3)
+            hs.append(eq.rans_encode_device(sym, sc, eq.EQ_SYM_E4M3, wl7.chunk_symbols,
+                                            wl7.streams, wl7.run))
+            rs.append(wt.to(torch.bfloat16))
+            del wt, sym, sc
+        blocks.append(hs)
+        resident.append(rs)
+    pipe = BlockPipeline(blocks)
+    lparams = sum(t.numel for b in blocks for t in b)
+    for tokens in (1, 512):
+        xt = torch.randn(tokens, 11008, device=dev).to(torch.bfloat16)
+
+        def fwd(i, ws):
+            for w in ws:
+                torch.matmul(xt[:, :w.shape[1]], w.t())
+        ts_c = time_steps(lambda: [fwd(i, resident[i]) for i in range(4)], steps, 3, flush, stream)
+        ts_s = time_steps(lambda: pipe.run(fwd, overlap=False), steps, 3, flush, stream)
+        ts_o = time_steps(lambda: pipe.run(fwd, overlap=True), steps, 3, flush, stream)
+        assert int(pipe.status.item()) == 0
+        c, sq, ov = (statistics.mean(v) for v in (ts_c, ts_s, ts_o))
+        out.append({"what": f"4 LLaMA-2-7B layers, {tokens} token(s): forward GEMMs on resident "
+                            f"bf16 vs decode-then-compute vs overlapped",
+                    "params": lparams, "compute_ms": c * 1e3, "sequential_ms": sq * 1e3,
+                    "overlapped_ms": ov * 1e3, "slowdown_sequential": sq / c,
+                    "slowdown_overlapped": ov / c,
+                    "pages_claim": "1.5-2x slower than bf16 (EntQuant), 2-3x (DFloat11 forum)",
+                    "kernel": "rans_decode_kernel + cuBLAS bf16 GEMM"})
+    del pipe, blocks, resident
     # fused decode + GEMV over the three 13B MLP weights (gate, up 13824x5120; down 5120x13824);
     # algorithmic bytes = the coded weights read (+ x and y)
     wl = synth.WORKLOADS["mlp_13b"]

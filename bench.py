@@ -404,6 +404,20 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                     "gbs": alg / sec / 1e9, "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"],
                     "bits_per_param": 8 * coded / params, "kernel": "rans_gemv_kernel",
                     "launches_per_step": len(mats)})
+        # the whole MLP block: gate and up products, SiLU gate to bf16, down product
+        byname = {spec.name: m for spec, m in zip(wl.tensors, mats)}
+        g, u, d = byname["gate"], byname["up"], byname["down"]
+        xb = xs[[spec.name for spec in wl.tensors].index("gate")]
+        yb = torch.empty(batch, d.rows, dtype=torch.float32, device=dev)
+        scratch = torch.empty(eq.mlp_scratch_bytes(g.rows, batch), dtype=torch.uint8, device=dev)
+        ts = time_steps(lambda: eq.mlp_decode(g, u, d, xb, yb, scratch, st, stream), steps, 3,
+                        flush, stream)
+        assert int(st.item()) == 0
+        sec = statistics.mean(ts)
+        out.append({"what": f"MLP block from coded weights (13B: gate, up, SiLU gate, down), "
+                            f"batch {batch}",
+                    "params": params, "ms": sec * 1e3, "params_per_s": params / sec,
+                    "kernel": "rans_gemv_kernel x3 + silu_mul_kernel", "launches_per_step": 4})
     return out
 
 

@@ -11,6 +11,7 @@ from ._lib import (EQ_DEV_BAD_CODE, EQ_DEV_CORRUPT_STATE, EQ_DEV_COUNT_MISMATCH,
                    EQ_DEV_OVERRUN, EQ_DEV_TIMEOUT, EQ_SYM_E4M3, EQ_SYM_INT8, EQ_TABLE_HUFF,
                    EQ_TABLE_RANS, EXPORTS, EqError, lib)
 from .api import (DeviceHuff, DeviceRans, bf16_bits, build_tables, decode,  # noqa: F401
-                  decode_gemv, histogram_device, huff_bf16_decode, new_status, normalize_freqs,
+                  decode_gemv, histogram_device, huff_bf16_decode, mlp_decode,
+                  mlp_scratch_bytes, new_status, normalize_freqs,
                   quantize_device, rans_encode_device, table_bytes)
 from . import codec  # noqa: F401

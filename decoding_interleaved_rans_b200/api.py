@@ -178,6 +178,29 @@ def decode_gemv(t: DeviceRans, x: torch.Tensor, y=None, status=None, stream=None
     return y, status
 
 
+def mlp_scratch_bytes(inter: int, batch: int) -> int:
+    return int(L.lib().eq_mlp_scratch_bytes(inter, batch))
+
+
+def mlp_decode(gate: DeviceRans, up: DeviceRans, down: DeviceRans, x: torch.Tensor, y=None,
+               scratch=None, status=None, stream=None):
+    """eq_mlp_decode: y[b] = W_down(silu(W_gate x[b]) * (W_up x[b])) from coded weights."""
+    assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape[-1] == gate.cols
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty(batch, down.rows, dtype=torch.float32, device=x.device)
+    nbytes = mlp_scratch_bytes(gate.rows, batch)
+    if scratch is None:
+        scratch = torch.empty(nbytes, dtype=torch.uint8, device=x.device)
+    if status is None:
+        status = new_status(x.device)
+    dg, du, dd = gate.desc(), up.desc(), down.desc()
+    L.check(L.lib().eq_mlp_decode(C.byref(dg), C.byref(du), C.byref(dd), _ptr(x), batch, _ptr(y),
+                                  _ptr(scratch), scratch.numel() * scratch.element_size(),
+                                  _ptr(status), _stream(stream)), "eq_mlp_decode")
+    return y, status
+
+
 def huff_bf16_decode(h: DeviceHuff, out=None, status=None, stream=None):
     """eq_huff_bf16_decode: DFloat11 -> bf16 [n]."""
     dev = h.enc_exp.device

@@ -177,6 +177,22 @@ eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x, uint32_t 
 eq_status eq_huff_bf16_decode(const eq_huff_tensor *h, uint16_t *d_out, uint32_t *d_status,
                               void *stream);
 
+/*
+ * Beyond the four calls: a LLaMA-style MLP block straight from coded weights,
+ *   y[b] = W_down ( silu(W_gate x[b]) * (W_up x[b]) ),   silu(v) = v / (1 + e^-v),
+ * with gate, up: inter x hidden and down: hidden x inter, all in eq_decode_gemv's layout; the
+ * hidden activations are rounded to bf16 before the down projection.  The decoded weights never
+ * reach memory ("Float8@2bits" summary, closing section: fused decompression + compute kernels).
+ * d_x: bf16 [batch][hidden]; d_y: fp32 [batch][hidden]; batch 1..16; inter % 8 == 0.
+ * d_scratch: device memory of at least eq_mlp_scratch_bytes(inter, batch) bytes, 256-byte
+ * aligned, owned by the caller; it holds the two fp32 products and the bf16 hidden vector.
+ */
+size_t eq_mlp_scratch_bytes(uint32_t inter, uint32_t batch);
+eq_status eq_mlp_decode(const eq_rans_tensor *gate, const eq_rans_tensor *up,
+                        const eq_rans_tensor *down, const uint16_t *d_x, uint32_t batch,
+                        float *d_y, void *d_scratch, size_t scratch_bytes, uint32_t *d_status,
+                        void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *eq_status_string(eq_status s);
 

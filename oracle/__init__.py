@@ -368,6 +368,16 @@ def gemv_f64(w_bf16: np.ndarray, x_bf16: np.ndarray) -> np.ndarray:
     return y
 
 
+def mlp_f64(wg_bf16, wu_bf16, wd_bf16, x_bf16) -> np.ndarray:
+    """y[b] = W_down h[b], h = bf16( silu(W_gate x[b]) * (W_up x[b]) ), silu(v) = v / (1 + e^-v);
+    the products in binary64, h rounded once to bf16 (what the down projection reads)."""
+    g = gemv_f64(wg_bf16, x_bf16)
+    u = gemv_f64(wu_bf16, x_bf16)
+    hv = g / (1.0 + np.exp(-g)) * u
+    h = f64_to_bf16(hv.ravel()).reshape(hv.shape)
+    return gemv_f64(wd_bf16, h)
+
+
 # ----------------------------------------------------------------------------------------------
 # DFloat11 (Huffman-coded bf16 exponent)
 # ----------------------------------------------------------------------------------------------

@@ -26,3 +26,30 @@ def test_gemv_matches_numpy_float64(orc):
     y = orc.gemv_f64(w, x)
     ref = orc.bf16_to_f32(x).astype(np.float64) @ orc.bf16_to_f32(w).astype(np.float64).T
     assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+
+
+def _round_bf16_f64(v):
+    """bf16 round-to-nearest-even of binary64 values in bf16's normal range, written from the
+    format: 8 significant bits, ties to the even significand (numpy's round is half-to-even)."""
+    m, e = np.frexp(v)
+    return np.ldexp(np.round(m * 256.0) / 256.0, e)
+
+
+def test_mlp_chain_matches_numpy(orc):
+    """The oracle's MLP block (gate and up products, SiLU gate, hidden rounded once to bf16, down
+    product) against the same chain written here from its definition with numpy float64."""
+    rng = np.random.default_rng(5)
+    hidden, inter, batch = 48, 160, 3
+    wg = synth.bf16_bits(rng.standard_normal((inter, hidden)).astype(np.float32) * 0.2)
+    wu = synth.bf16_bits(rng.standard_normal((inter, hidden)).astype(np.float32) * 0.2)
+    wd = synth.bf16_bits(rng.standard_normal((hidden, inter)).astype(np.float32) * 0.2)
+    x = synth.bf16_bits(rng.standard_normal((batch, hidden)).astype(np.float32))
+    f = lambda b: orc.bf16_to_f32(b).astype(np.float64)  # noqa: E731
+    g, u = f(x) @ f(wg).T, f(x) @ f(wu).T
+    h = _round_bf16_f64(g * u / (1.0 + np.exp(-g)))
+    ref = h @ f(wd).T
+    y = orc.mlp_f64(wg, wu, wd, x)
+    assert np.max(np.abs(y - ref)) <= 1e-12 * np.max(np.abs(ref))
+    # SiLU(0) = 0: an all-zero gate makes the hidden vector, and so y, exactly zero
+    z = np.zeros_like(wg)
+    assert np.all(orc.mlp_f64(z, wu, wd, x) == 0.0)

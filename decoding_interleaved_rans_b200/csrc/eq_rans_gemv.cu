@@ -375,7 +375,8 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  const int bi = tc ? 5 : batch <= 1 ? 0 : batch <= 2 ? 1 : batch <= 4 ? 2 : 3;
+  // one flag per kernel instance that pick_b / the tensor-core choice can return
+  const int bi = tc ? 5 : batch <= 1 ? 0 : batch <= 2 ? 1 : batch <= 4 ? 2 : batch <= 8 ? 3 : 4;
   bool &attr = g_gemv_attr[dev][t->symfmt - 1][bi];
   if (!attr) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -98,3 +98,18 @@ def test_unsupported_layouts_rejected(eq, orc):
         t = eq.DeviceRans.upload(orc.rans_encode(sym, sc, orc.E4M3, chunk, S, G))
         with pytest.raises(eq.EqError):
             eq.decode_gemv(t, x)
+
+
+def test_every_batch_width_after_another_on_a_large_tensor(eq, orc):
+    """Each kernel instance opts into its own shared-memory size: on a tensor with enough chunks
+    for 16-warp CTAs (whose shared memory exceeds the default limit), every batch width runs
+    after the others, the CUDA-core batch 9..16 kernel included (chunks not a multiple of 256)."""
+    w = synth.normal(16384, 64, 0.02, 10)
+    sym, sc = orc.quantize(w, orc.E4M3)
+    h = orc.rans_encode(sym, sc, orc.E4M3, 64, 32, 8)
+    wbf = orc.dequant(sym, sc, orc.E4M3)
+    for batch in (8, 16, 5, 2, 1, 12):
+        x = synth.activations(batch, 64, 11, tensor=200 + batch)
+        y, st = gemv(eq, h, x)
+        assert st == 0, batch
+        assert rel_l2(y, orc.gemv_f64(wbf, x)) <= TIGHT, batch

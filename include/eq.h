@@ -193,6 +193,24 @@ eq_status eq_mlp_decode(const eq_rans_tensor *gate, const eq_rans_tensor *up,
                         float *d_y, void *d_scratch, size_t scratch_bytes, uint32_t *d_status,
                         void *stream);
 
+/*
+ * No counterpart in the pages: an addition for callers that cannot allocate device memory.
+ * eq_mlp_decode with the scratch inside the library, for callers that can pass no scratch
+ * buffer: an engine or framework that has reserved (nearly) all of HBM for its own allocator,
+ * so a cudaMalloc from here would fail or eat into its pool, and hot loops that must not pay
+ * for cudaMalloc / cudaFree, which can synchronise the device.  The scratch is one fixed device
+ * array per device (placed by the CUDA runtime when it loads the library's code on that device)
+ * sized for inter * batch <= EQ_MLP_NOALLOC_MAX_ELEMS (5 MiB); no allocating routine is called.
+ * Larger sizes return EQ_ERR_UNSUPPORTED without launching.  The array's address on the current
+ * device is looked up on the first call there.  Every call on a device shares the array, so
+ * calls whose work may overlap on the GPU (streams not ordered with one another) race: order
+ * them.  Nothing needs zeroing beforehand.  Arguments, layouts and other errors as eq_mlp_decode.
+ */
+#define EQ_MLP_NOALLOC_MAX_ELEMS 524288u
+eq_status eq_mlp_decode_noalloc(const eq_rans_tensor *gate, const eq_rans_tensor *up,
+                                const eq_rans_tensor *down, const uint16_t *d_x, uint32_t batch,
+                                float *d_y, uint32_t *d_status, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *eq_status_string(eq_status s);
 

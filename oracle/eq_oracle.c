@@ -230,14 +230,23 @@ int orc_rans_normalize(const uint64_t *counts, uint32_t prob_bits, uint32_t *fre
  * Streams form groups of 32 (group g = streams 32g .. 32g+31, the last group may be smaller);
  *   every group has its own word substream, holding the words its streams read, in the order
  *   they read them.  Groups never share words, so a chunk's groups decode independently.
- * Encoder: all S states start at L = 2^16; steps are taken in exactly the reverse order.  Before
- *   coding s with frequency f and cumulative frequency c, if x >= f * 2^(32 - prob_bits) the low 16
- *   bits of x are emitted onto its group's stack and x >>= 16; then x = floor(x / f) * M +
- *   (x mod f) + c.  Each group's stack, reversed, is its substream in decoder-forward order; the
- *   chunk's words are the substreams of groups 0, 1, ... one after the other.
+ * Renormalisation interval: with M = 2^prob_bits, a stream renormalises after every k-th of its
+ *   own steps and after its last step, k = floor(16 / prob_bits) (k = 1 for 12-bit tables, k = 2
+ *   for 8-bit ones).  M^k <= 2^16 = L makes one 16-bit word always enough: k steps shrink a state
+ *   >= L by at most a factor M^k, so it stays >= 1.  A stream's steps are counted t = 0, 1, ...
+ *   in decode order (step t is position t mod G of its (t div G)-th run); the steps between two
+ *   renormalisation points form a group of m <= k steps.
+ * Encoder: all S states start at L = 2^16; steps are taken in exactly the reverse order.  On the
+ *   last step of a group (the first the encoder meets), if x >= 2^(32 - m * prob_bits) times the
+ *   product of the group's m frequencies, the low 16 bits of x are emitted onto its group's stack
+ *   and x >>= 16 (that bound is the largest x from which the m coding steps stay below 2^32);
+ *   then, on every step, coding s with frequency f and cumulative frequency c is
+ *   x = floor(x / f) * M + (x mod f) + c.  Each group's stack, reversed, is its substream in
+ *   decoder-forward order; the chunk's words are the substreams of groups 0, 1, ... in turn.
  * Decoder: slot = x mod M; s is the symbol with c_s <= slot < c_s + f_s;
- *   x = f_s * floor(x / M) + slot - c_s; if x < L then x = x * 2^16 + next word of its group.
- *   At the end every x is L again and every group has read all of its words.
+ *   x = f_s * floor(x / M) + slot - c_s; at a renormalisation point, if x < L then
+ *   x = x * 2^16 + next word of its group.  At the end every x is L again and every group has
+ *   read all of its words.
  * ========================================================================================== */
 
 #define RANS_L 65536u
@@ -253,40 +262,70 @@ static void cum_of(const uint32_t *freqs, uint32_t *cum) {
 
 int64_t orc_rans_groups(uint32_t S) { return ((int64_t)S + RANS_GROUP - 1) / RANS_GROUP; }
 
+/* Steps of stream s in a chunk of n symbols: its runs are s, s + S, s + 2S, ... below the run
+ * count, all G long except the chunk's last run, which may be short. */
+static int64_t stream_steps(int64_t n, uint32_t S, uint32_t G, uint32_t s) {
+  const int64_t runs = (n + G - 1) / G;
+  if ((int64_t)s >= runs) return 0;
+  int64_t T = ((runs - 1 - (int64_t)s) / S + 1) * G;
+  if ((runs - 1) % S == (int64_t)s) T -= runs * (int64_t)G - n;
+  return T;
+}
+
+/* index in the chunk of step t of stream s */
+static int64_t step_symbol(int64_t t, uint32_t S, uint32_t G, uint32_t s) {
+  return ((t / G) * S + s) * G + t % G;
+}
+
+static uint32_t renorm_interval(uint32_t prob_bits) { return 16u / prob_bits; }
+
 /* Returns the number of words written to words_out (capacity must be >= n), or < 0.
  * group_count[g] receives the length of group g's substream (ceil(S / 32) entries). */
 int64_t orc_rans_encode_chunk(const uint8_t *sym, int64_t n, const uint32_t *freqs,
                               uint32_t prob_bits, uint32_t S, uint32_t G, uint32_t *states_out,
                               uint16_t *words_out, int64_t *group_count) {
-  if (S < 1 || G < 1 || n < 0) return ORC_ERR_ARG;
+  if (S < 1 || G < 1 || n < 0 || prob_bits < 1 || prob_bits > 16) return ORC_ERR_ARG;
   uint32_t cum[256];
   cum_of(freqs, cum);
   const int64_t ng = orc_rans_groups(S);
+  const int64_t k = renorm_interval(prob_bits);
   uint32_t *x = (uint32_t *)malloc(S * sizeof(uint32_t));
+  int64_t *T = (int64_t *)malloc(S * sizeof(int64_t));
   /* one stack per group, each with room for every symbol of the chunk */
   uint16_t *stack = (uint16_t *)malloc((size_t)(ng * (n > 0 ? n : 1)) * sizeof(uint16_t));
   int64_t *depth = (int64_t *)calloc((size_t)ng, sizeof(int64_t));
-  for (uint32_t s = 0; s < S; ++s) x[s] = RANS_L;
+  for (uint32_t s = 0; s < S; ++s) {
+    x[s] = RANS_L;
+    T[s] = stream_steps(n, S, G, s);
+  }
+  for (int64_t j = 0; j < n; ++j)
+    if (freqs[sym[j]] == 0) {
+      free(x);
+      free(T);
+      free(stack);
+      free(depth);
+      return ORC_ERR_SYMBOL;
+    }
   int64_t runs = (n + G - 1) / G, rounds = (runs + S - 1) / S;
   for (int64_t round = rounds - 1; round >= 0; --round)
     for (int64_t p = (int64_t)G - 1; p >= 0; --p)
       for (int64_t s = (int64_t)S - 1; s >= 0; --s) {
         int64_t j = (round * S + s) * G + p;
         if (j >= n) continue;
-        uint32_t f = freqs[sym[j]];
-        if (f == 0) {
-          free(x);
-          free(stack);
-          free(depth);
-          return ORC_ERR_SYMBOL;
-        }
-        uint64_t xmax = (uint64_t)f << (32 - prob_bits);
+        const int64_t t = round * G + p;
+        const int64_t g0 = t / k * k;
+        const int64_t g1 = g0 + k < T[s] ? g0 + k : T[s];
         uint32_t xs = x[s];
-        if ((uint64_t)xs >= xmax) {
-          int64_t g = s / RANS_GROUP;
-          stack[g * n + depth[g]++] = (uint16_t)(xs & 0xFFFFu);
-          xs >>= 16;
+        if (t == g1 - 1) { /* the group's last step: flush before its m coding steps */
+          uint64_t xmax = (uint64_t)1 << (32 - (g1 - g0) * prob_bits);
+          for (int64_t u = g0; u < g1; ++u) xmax *= freqs[sym[step_symbol(u, S, G, (uint32_t)s)]];
+          if ((uint64_t)xs >= xmax) {
+            int64_t g = s / RANS_GROUP;
+            stack[g * n + depth[g]++] = (uint16_t)(xs & 0xFFFFu);
+            xs >>= 16;
+          }
         }
+        uint32_t f = freqs[sym[j]];
         x[s] = ((xs / f) << prob_bits) + (xs % f) + cum[sym[j]];
       }
   int64_t nw = 0;
@@ -296,6 +335,7 @@ int64_t orc_rans_encode_chunk(const uint8_t *sym, int64_t n, const uint32_t *fre
   }
   memcpy(states_out, x, S * sizeof(uint32_t));
   free(x);
+  free(T);
   free(stack);
   free(depth);
   return nw;
@@ -305,9 +345,10 @@ int64_t orc_rans_encode_chunk(const uint8_t *sym, int64_t n, const uint32_t *fre
 int orc_rans_decode_chunk(const uint16_t *words, const int64_t *group_off, const uint32_t *states,
                           int64_t n, const uint32_t *freqs, uint32_t prob_bits, uint32_t S,
                           uint32_t G, uint8_t *sym_out) {
-  if (S < 1 || G < 1 || n < 0) return ORC_ERR_ARG;
+  if (S < 1 || G < 1 || n < 0 || prob_bits < 1 || prob_bits > 16) return ORC_ERR_ARG;
   const uint32_t M = 1u << prob_bits;
   const int64_t ng = orc_rans_groups(S);
+  const int64_t k = renorm_interval(prob_bits);
   uint32_t cum[256];
   cum_of(freqs, cum);
   uint8_t *slot_sym = (uint8_t *)malloc(M);
@@ -333,7 +374,9 @@ int orc_rans_decode_chunk(const uint16_t *words, const int64_t *group_off, const
         uint32_t slot = x[s] & (M - 1);
         uint8_t q = slot_sym[slot];
         x[s] = freqs[q] * (x[s] >> prob_bits) + slot - cum[q];
-        if (x[s] < RANS_L) {
+        const int64_t t = round * G + p;
+        const int renorm_point = (t + 1) % k == 0 || t + 1 == stream_steps(n, S, G, (uint32_t)s);
+        if (renorm_point && x[s] < RANS_L) {
           int64_t g = s / RANS_GROUP;
           if (ptr[g] >= group_off[g + 1]) {
             rc = ORC_ERR_OVERRUN;

@@ -4,13 +4,15 @@
     torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
 
 A step decodes the whole Int8 8192x8192 Laplace weight (H = 2.0 bits, 64 KiB chunks, 128
-interleaved streams, run 8) from its rANS stream in HBM into bf16 in HBM: one eq_decode launch.
+interleaved streams, run 8, 8-bit frequency table: one renormalisation per two steps) from its
+rANS stream in HBM into bf16 in HBM: one eq_decode launch.
 Every rank decodes its own copy (weak scaling; the decode has no exchange step).  Timing: CUDA
 events on the launching stream around each step, the L2 flushed between steps by writing a
 256 MiB buffer, max over ranks.  `e2e` repeats the step through the C ABI with host buffers:
 pinned host -> device copy of the coded arrays, decode, device -> host copy of the bf16 weight.
-Secondary lines under "also": the fused decode-GEMV on the 13B MLP (batch 1/4/16) and the DFloat11
-decode, each with its own roofline.
+Secondary lines under "also": the same weight with a 12-bit table, the fused decode-GEMV on the
+13B MLP (batch 1/4/16), the MLP block, the DFloat11 decode, the GPU compressor and the block
+pipeline, each with its own roofline or comparison.
 """
 from __future__ import annotations
 
@@ -170,7 +172,7 @@ def max_over_ranks(world, v: float) -> float:
     return dist.max_over_ranks(v, device="cuda")
 
 
-def prepare_rans(eq, wl_name: str):
+def prepare_rans(eq, wl_name: str, prob_bits: int | None = None):
     """Quantise + encode the workload with the library's own host compressor (no oracle)."""
     wl = synth.WORKLOADS[wl_name]
     spec = wl.tensors[0]
@@ -178,7 +180,8 @@ def prepare_rans(eq, wl_name: str):
     fmt = eq.EQ_SYM_E4M3 if wl.symfmt == "e4m3" else eq.EQ_SYM_INT8
     sym, sc = eq.codec.quantize(w, fmt, wl.int8_div)
     del w
-    h = eq.codec.rans_encode(sym, sc, fmt, wl.chunk_symbols, wl.streams, wl.run)
+    h = eq.codec.rans_encode(sym, sc, fmt, wl.chunk_symbols, wl.streams, wl.run,
+                             prob_bits=prob_bits or wl.prob_bits)
     return wl, h
 
 
@@ -263,7 +266,21 @@ def run_ours(args):
 
     also = []
     if not args.no_extra:
-        also = extra_measurements(eq, dev, stream, flush, peaks, args)
+        # the same weight with a 12-bit table (a renormalisation point after every step)
+        _, h12 = prepare_rans(eq, WORKLOAD, prob_bits=12)
+        t12 = eq.DeviceRans.upload(h12, dev)
+        ts12 = time_steps(lambda: eq.decode([t12], [out], status, stream), max(5, args.steps // 2),
+                          3, flush, stream)
+        assert int(status.item()) == 0
+        s12 = statistics.mean(ts12)
+        a12 = (t12.compressed_bytes + 2 * numel) / s12 / 1e9
+        also.append({"what": "same Int8 weight, 12-bit table (renormalisation every step)",
+                     "params": numel, "ms": s12 * 1e3, "params_per_s": numel / s12, "gbs": a12,
+                     "frac_of_peak": a12 / peaks["hbm_gbs"],
+                     "bits_per_param": 8 * t12.compressed_bytes / numel,
+                     "kernel": "rans_decode_kernel<run 8, Int8, 12-bit table>"})
+        del t12, h12
+        also += extra_measurements(eq, dev, stream, flush, peaks, args)
     barrier(world)
     if rank != 0:
         return
@@ -274,7 +291,7 @@ def run_ours(args):
         "ms_per_step": mean_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
         "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
-                               "chunks, 128 streams, run 8 -> bf16",
+                               "chunks, 128 streams, run 8, 8-bit table -> bf16",
                    "params_per_gpu": numel, "compressed_bytes": t.compressed_bytes,
                    "bits_per_param": 8 * t.compressed_bytes / numel,
                    "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{world}"},
@@ -282,7 +299,8 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": measured_traffic("rans_decode_kernel", numel),
-                     "peak_src": peaks["src"], "kernel": "rans_decode_kernel<run 8, Int8>",
+                     "peak_src": peaks["src"],
+                     "kernel": "rans_decode_kernel<run 8, Int8, 8-bit table>",
                      "alg_bytes_per_launch": alg_bytes},
         "e2e": {"value": numel * world / e2e_s, "unit": "params/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_s * 1e3},
@@ -327,7 +345,8 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         sym, sc = eq.quantize_device(wdev, eq.EQ_SYM_INT8, wl.int8_div)
-        tc = eq.rans_encode_device(sym, sc, eq.EQ_SYM_INT8, wl.chunk_symbols, wl.streams, wl.run)
+        tc = eq.rans_encode_device(sym, sc, eq.EQ_SYM_INT8, wl.chunk_symbols, wl.streams, wl.run,
+                                   prob_bits=wl.prob_bits)
         torch.cuda.synchronize()
         if it:
             times_c.append(time.perf_counter() - t0)
@@ -454,7 +473,8 @@ def run_reference(args):
     import oracle
     wl = synth.WORKLOADS[WORKLOAD]
     sym, sc = oracle.quantize(wl.tensors[0].generate(), oracle.INT8, wl.int8_div)
-    o = oracle.rans_encode(sym, sc, oracle.INT8, wl.chunk_symbols, wl.streams, wl.run)
+    o = oracle.rans_encode(sym, sc, oracle.INT8, wl.chunk_symbols, wl.streams, wl.run,
+                           prob_bits=wl.prob_bits)
     h = o
     cores = len(os.sched_getaffinity(0))
     take = min(o.num_chunks, max(cores * 4, 64))
@@ -475,7 +495,7 @@ def run_reference(args):
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
             "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
-                                   "chunks, 128 streams, run 8 -> bf16",
+                                   "chunks, 128 streams, run 8, 8-bit table -> bf16",
                        "sample_chunks": take, "parallelism": "host cores"},
             "cpu_baseline": {"value": v, "unit": "params/s", "cores": cores, "kind": "oracle",
                              "sample": f"{take} of {o.num_chunks} chunks per step"},

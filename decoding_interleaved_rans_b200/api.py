@@ -252,13 +252,14 @@ def normalize_freqs(counts, prob_bits: int = 12) -> np.ndarray:
 
 def rans_encode_device(sym: torch.Tensor, scales: torch.Tensor, symfmt: int, chunk_symbols: int,
                        streams: int, run: int, freqs=None, status=None,
-                       stream=None) -> "DeviceRans":
-    """Encode a device symbol matrix on the GPU into a DeviceRans (plan, offsets, encode)."""
+                       stream=None, prob_bits: int = 12) -> "DeviceRans":
+    """Encode a device symbol matrix on the GPU into a DeviceRans (plan, offsets, encode).
+    prob_bits 12, or 8 (needs run 8 and cols % 8 == 0)."""
     assert sym.dtype == torch.uint8 and sym.is_cuda and sym.is_contiguous() and sym.dim() == 2
     rows, cols = sym.shape
     dev = sym.device
     if freqs is None:
-        freqs = normalize_freqs(histogram_device(sym, stream).cpu().numpy())
+        freqs = normalize_freqs(histogram_device(sym, stream).cpu().numpy(), prob_bits)
     f = (C.c_uint32 * 256)(*[int(v) for v in np.asarray(freqs).ravel()[:256]])
     chunk = chunk_symbols if chunk_symbols else cols
     nchunks = (rows * cols + chunk - 1) // chunk
@@ -275,9 +276,9 @@ def rans_encode_device(sym: torch.Tensor, scales: torch.Tensor, symfmt: int, chu
     L.check(L.lib().eq_rans_encode_device(_ptr(sym), rows, cols, f, chunk_symbols, streams, run,
                                           _ptr(word_off), _ptr(words), _ptr(status),
                                           _stream(stream)), "eq_rans_encode_device")
-    t = DeviceRans(rows, cols, symfmt, 12, chunk_symbols, streams, run, nchunks,
+    t = DeviceRans(rows, cols, symfmt, prob_bits, chunk_symbols, streams, run, nchunks,
                    states[:nchunks * streams] if nchunks else states, word_off, words,
                    scales, torch.empty(table_bytes(L.EQ_TABLE_RANS), dtype=torch.uint8,
                                        device=dev))
-    build_tables(L.EQ_TABLE_RANS, freqs, 12, t.tables, stream)
+    build_tables(L.EQ_TABLE_RANS, freqs, prob_bits, t.tables, stream)
     return t

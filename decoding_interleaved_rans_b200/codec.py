@@ -70,12 +70,17 @@ def rans_freqs(sym: np.ndarray, prob_bits: int = 12) -> np.ndarray:
 
 
 def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols: int,
-                streams: int, run: int, freqs=None, threads: int = 0) -> HostRans:
+                streams: int, run: int, freqs=None, threads: int = 0,
+                prob_bits: int = 12) -> HostRans:
+    """prob_bits 12, or 8 (streams renormalise once per two steps; needs run 8).  Given freqs
+    must sum to 2^prob_bits."""
     sym = np.ascontiguousarray(sym, dtype=np.uint8)
     rows, cols = sym.shape
     if freqs is None:
-        freqs = rans_freqs(sym)
+        freqs = rans_freqs(sym, prob_bits)
     freqs = np.ascontiguousarray(freqs, dtype=np.uint32)
+    if int(freqs.sum()) != 1 << prob_bits:
+        raise ValueError("freqs do not sum to 2^prob_bits")
     chunk = chunk_symbols if chunk_symbols else cols
     nchunks = (rows * cols + chunk - 1) // chunk
     states = np.empty(max(1, nchunks * streams), np.uint32)
@@ -89,9 +94,26 @@ def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols:
         words = np.ctypeslib.as_array(C.cast(wp, C.POINTER(C.c_uint16)), (nw.value,)).copy()
     finally:
         L.lib().eq_free_host(wp)
-    return HostRans(rows, cols, symfmt, 12, chunk_symbols, streams, run, freqs,
+    return HostRans(rows, cols, symfmt, prob_bits, chunk_symbols, streams, run, freqs,
                     states[:nchunks * streams], word_off, words,
                     np.ascontiguousarray(scales, np.uint16))
+
+
+def choose_prob_bits(counts, max_loss: float = 0.005) -> int:
+    """8 when an 8-bit table codes these symbol counts within max_loss (relative) of the 12-bit
+    table's rate, else 12.  8-bit tables halve the decoder's renormalisation work; they suit
+    low-entropy alphabets (a few Int8 values), not the ~6.5-bit Float8 one."""
+    c = np.asarray(counts, dtype=np.float64).ravel()
+    if c.sum() == 0 or np.count_nonzero(c) > 256:
+        return 12
+    cu = np.ascontiguousarray(c, dtype=np.uint64)
+    rate = {}
+    for pb in (8, 12):
+        f = np.zeros(256, np.uint32)
+        L.check(L.lib().eq_rans_normalize_host(_p(cu), pb, _p(f)), "eq_rans_normalize_host")
+        m = c > 0
+        rate[pb] = float(-(c[m] * np.log2(f[m] / float(1 << pb))).sum() / c.sum())
+    return 8 if rate[8] <= rate[12] * (1 + max_loss) else 12
 
 
 def huff_lengths(counts: np.ndarray, max_len: int = 32) -> np.ndarray:

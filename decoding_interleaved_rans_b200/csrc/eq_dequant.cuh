@@ -49,21 +49,21 @@ __device__ __forceinline__ uint32_t dequant2(uint32_t pair, float scale, bool na
   return o;
 }
 
-// the eight symbols of a round, taken from their slot-table entries (symbol in bits 19..12),
-// scaled -> eight bf16 (one 16-byte store)
-template <int FMT>
+// the eight symbols of a round, taken from their PB-bit slot-table entries (symbol in bits
+// PB+7..PB), scaled -> eight bf16 (one 16-byte store)
+template <int FMT, uint32_t PB = 12>
 __device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, bool nan_codes) {
   uint32_t o[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     if constexpr (FMT == EQ_SYM_INT8) {
       // the symbol byte sign-extended straight out of the entry
-      const float v0 = float(int32_t(e[2 * k] << 12) >> 24);
-      const float v1 = float(int32_t(e[2 * k + 1] << 12) >> 24);
+      const float v0 = float(int32_t(e[2 * k] << (24 - PB)) >> 24);
+      const float v1 = float(int32_t(e[2 * k + 1] << (24 - PB)) >> 24);
       o[k] = pack_bf16x2(v0 * scale, v1 * scale);
     } else {
-      const uint32_t pair = ((e[2 * k] >> 12) & 0xFFu) | ((e[2 * k + 1] >> 4) & 0xFF00u);
-      o[k] = dequant2<FMT>(pair, scale, nan_codes);
+      if constexpr (PB == 8) o[k] = dequant2<FMT>(__byte_perm(e[2 * k], e[2 * k + 1], 0x0051u), scale, nan_codes);
+      else o[k] = dequant2<FMT>(((e[2 * k] >> PB) & 0xFFu) | ((e[2 * k + 1] >> (PB - 8)) & 0xFF00u), scale, nan_codes);
     }
   }
   return make_uint4(o[0], o[1], o[2], o[3]);

@@ -152,7 +152,9 @@ extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint
   uint32_t cum[257];
   cum[0] = 0;
   for (int s = 0; s < 256; ++s) cum[s + 1] = cum[s] + freqs[s];
-  if (cum[256] != 4096u) return EQ_ERR_FORMAT;
+  if (cum[256] != 256u && cum[256] != 4096u) return EQ_ERR_FORMAT;
+  // 8-bit tables renormalise after every second step of a stream, 12-bit ones after every step
+  const uint32_t pb = cum[256] == 256u ? 8u : 12u, k = 16u / pb;
   const uint64_t nchunks = (N + chunk - 1) / chunk;
   const uint32_t groups = (streams + 31) / 32;  // 32 streams share one word substream
   std::vector<std::vector<uint16_t>> pieces(nchunks * groups);
@@ -165,6 +167,16 @@ extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint
     std::vector<uint16_t> *out = &pieces[c * groups];  // encoder order, reversed at the end
     const uint64_t nruns = (n + run - 1) / run;
     const uint64_t nrounds = (nruns + streams - 1) / streams;
+    // steps of stream st: its runs st, st + S, ... are full except the chunk's last run
+    auto steps_of = [&](uint32_t st) -> uint64_t {
+      if (st >= nruns) return 0;
+      uint64_t t = ((nruns - 1 - st) / streams + 1) * run;
+      if ((nruns - 1) % streams == st) t -= nruns * run - n;
+      return t;
+    };
+    auto sym_of_step = [&](uint64_t t, uint32_t st) {
+      return s[((t / run) * streams + st) * run + t % run];
+    };
     for (uint64_t rr = nrounds; rr-- > 0;)
       for (uint32_t p = run; p-- > 0;)
         for (uint32_t st = streams; st-- > 0;) {
@@ -176,11 +188,18 @@ extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint
             return;
           }
           uint32_t v = x[st];
-          if (uint64_t(v) >= (uint64_t(f) << 20)) {
-            out[st / 32].push_back(uint16_t(v));
-            v >>= 16;
+          // flush on the last step of a renormalisation group, before its coding steps
+          const uint64_t t = rr * run + p, g0 = t / k * k;
+          const uint64_t g1 = k == 1 ? t + 1 : std::min<uint64_t>(g0 + k, steps_of(st));
+          if (t + 1 == g1) {
+            uint64_t xmax = 1ull << (32 - (g1 - g0) * pb);
+            for (uint64_t u = g0; u < g1; ++u) xmax *= freqs[sym_of_step(u, st)];
+            if (uint64_t(v) >= xmax) {
+              out[st / 32].push_back(uint16_t(v));
+              v >>= 16;
+            }
           }
-          x[st] = (v / f) * 4096u + v % f + cum[q];
+          x[st] = ((v / f) << pb) + v % f + cum[q];
         }
     for (uint32_t g = 0; g < groups; ++g) std::reverse(out[g].begin(), out[g].end());
     std::memcpy(states + c * streams, x.data(), streams * sizeof(uint32_t));

@@ -96,6 +96,7 @@ struct EncodeParams {
   uint64_t numel;
   uint64_t units;
   uint32_t chunk, streams, groups, run;
+  uint32_t prob_bits;  // 12, or 8: renormalise after every second step (then run == 8)
   uint16_t freq[256];
 };
 
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(256) rans_encode_kernel(const __grid_constant_
       const uint64_t j = uint64_t(run) * G + p;
       const bool on = run < runs && j < n;
       uint32_t f = 1, c = 0;
-      uint64_t m = 0;
+      uint64_t m = 0, xmax = 0;
       if (on) {
         const uint32_t q = src[j];
         f = fs[q];
@@ -142,8 +143,12 @@ __global__ void __launch_bounds__(256) rans_encode_kernel(const __grid_constant_
           bad = EQ_DEV_BAD_CODE;
           f = 1;
         }
+        // flush bound of the renormalisation group that ends at this step: one step (12-bit
+        // tables), or positions p - 1 and p of the run (8-bit tables, p odd)
+        if (P.prob_bits == 12) xmax = uint64_t(f) << 20;
+        else if (p & 1) xmax = (uint64_t(f) * max(fs[src[j - 1]], 1u)) << 16;
       }
-      const bool emit = on && uint64_t(x) >= (uint64_t(f) << 20);
+      const bool emit = on && xmax && uint64_t(x) >= xmax;
       const uint32_t em = __ballot_sync(0xFFFFFFFFu, emit);
       if (WRITE) {
         const uint32_t k = __popc(em);
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(256) rans_encode_kernel(const __grid_constant_
       if (emit) x >>= 16;
       if (on) {
         const uint32_t qt = f > 1 ? uint32_t(__umul64hi(uint64_t(x), m)) : x;
-        x = (qt << 12) + (x - qt * f) + c;
+        x = (qt << P.prob_bits) + (x - qt * f) + c;
       }
     }
   }
@@ -221,7 +226,10 @@ static eq_status check_encode_args(const uint8_t *d_sym, uint32_t rows, uint32_t
     sum += host_freqs[s];
     P.freq[s] = uint16_t(host_freqs[s]);
   }
-  if (sum != kRansSlots) return EQ_ERR_FORMAT;
+  if (sum != 256 && sum != kRansSlots) return EQ_ERR_FORMAT;
+  P.prob_bits = sum == 256 ? 8 : 12;
+  // pairs of steps stay inside runs only when every run is whole
+  if (P.prob_bits == 8 && (run != 8 || cols % 8)) return EQ_ERR_UNSUPPORTED;
   P.sym = d_sym;
   P.numel = numel;
   P.chunk = chunk;

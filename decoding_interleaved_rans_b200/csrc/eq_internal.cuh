@@ -12,20 +12,21 @@ namespace eq {
 // device decode-table layouts written by eq_build_tables
 // ------------------------------------------------------------------------------------------------
 
-// rANS: 16-byte header, then one 32-bit entry per slot of the 4096-slot probability space:
-//   bits 31..20 frequency f (1..4095), bits 19..12 symbol, bits 11..0 slot - cum[symbol].
-// With f in the top bits, f * floor(x / 4096) is the high word of (e & 0xFFF00000) *
-// (x & 0xFFFFF000), one multiply-high.  A table whose single symbol owns all 4096 slots cannot
-// store its frequency in 12 bits; the header flags it instead and the decoders take a separate
-// path.
-constexpr uint32_t kRansProbBits = 12;
-constexpr uint32_t kRansSlots = 1u << kRansProbBits;
+// rANS: 16-byte header, then one 32-bit entry per slot of the 2^pb-slot probability space
+// (pb = prob_bits, 12 or 8):
+//   the top pb bits frequency f (1 .. 2^pb - 1), bits pb+7..pb symbol, bits pb-1..0 slot - cum.
+// With f in the top bits, f * floor(x / 2^pb) is the high word of (e & top pb bits) *
+// (x & ~(2^pb - 1)), one multiply-high.  A table whose single symbol owns every slot cannot
+// store its frequency in pb bits; the header flags it instead and the decoders take a separate
+// path.  8-bit tables use the first 256 entries of the same 16 KiB allocation.
+constexpr uint32_t kRansProbBits = 12;                 // the larger table
+constexpr uint32_t kRansSlots = 1u << kRansProbBits;  // entries the table allocation holds
 constexpr uint32_t kRansL = 1u << 16;
 struct RansTableHeader {
   uint32_t magic;        // kRansMagic
   uint32_t flags;        // kRansFlag*
   uint32_t single_sym;   // symbol of a one-symbol table
-  uint32_t reserved;
+  uint32_t prob_bits;    // 12 or 8
 };
 constexpr uint32_t kRansMagic = 0x52414E53u;  // "RANS"
 constexpr uint32_t kRansFlagNaN7F = 1u;       // frequency of byte 0x7F is nonzero

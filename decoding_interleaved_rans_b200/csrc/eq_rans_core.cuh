@@ -72,9 +72,11 @@ struct WordRing {
   }
 
   // the per-round checks: wait only when the round may read past the landed bytes, refill only
-  // when a slot has been used up
+  // when a slot has been used up.  The wait covers one word beyond the round's last possible
+  // word: lanes that need no word still load the one after the warp's words (and drop it).
   __device__ __forceinline__ bool round_wait(uint32_t q) {
-    return (q + 2 * kRoundWords <= ready_end || ready >= nseg) ? true : wait_below(q + 2 * kRoundWords);
+    constexpr uint32_t kAhead = 2 * kRoundWords + 2;
+    return (q + kAhead <= ready_end || ready >= nseg) ? true : wait_below(q + kAhead);
   }
   __device__ __forceinline__ void round_refill(uint32_t q, uint32_t lane) {
     if (q >= refill_at) refill(q, lane);
@@ -105,13 +107,14 @@ struct WordRing {
 };
 
 // ------------------------------------------------------------------------------------------------
-// One decode step of the lane's state x.  q is the byte offset (from the ring's A) of the group's
-// next unread word; it advances by 2 bytes per word the warp reads.  Slot-table entry e: f in bits
-// 31..20, symbol in 19..12, slot - cum in 11..0, so f * floor(x / 4096) + (slot - cum) is one
-// multiply-high-add: hi32((e & 0xFFF00000) * (x & 0xFFFFF000)) + (e & 0xFFF).  A ballot finds
-// the lanes whose state fell below 2^16; each takes the word at its rank among them, so words go
-// out in stream order.  ring_off: shared-memory offset of this warp's ring (a multiple of its
-// size), so the word address is one mask-and-or.
+// Decode steps of the lane's state x.  q is the byte offset (from the ring's A) of the group's
+// next unread word; it advances by 2 bytes per word the warp reads.  Slot-table entry e of a
+// 12-bit table: f in bits 31..20, symbol in 19..12, slot - cum in 11..0, so f * floor(x / 4096) +
+// (slot - cum) is one multiply-high-add: hi32((e & 0xFFF00000) * (x & 0xFFFFF000)) + (e & 0xFFF)
+// (an 8-bit table: the same with 8-bit fields).  At a renormalisation point a ballot finds the
+// lanes whose state fell below 2^16; each takes the word at its rank among them, so words go out
+// in stream order.  ring_off: shared-memory offset of this warp's ring (a multiple of its size),
+// so the word address is one mask-and-or.
 // ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
@@ -125,27 +128,46 @@ __device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
+// The decoding half of a step with a PB-bit table (entry: f in the top PB bits, symbol above
+// the low PB bits, slot - cum in them); returns the entry.
+template <bool FULL, uint32_t PB>
+__device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, const uint32_t *lut) {
+  constexpr uint32_t kLow = (1u << PB) - 1;
+  const uint32_t e = lut[x & kLow];
+  const uint32_t nx = mad_hi(e & ~(0xFFFFFFFFu >> PB), x & ~kLow, e & kLow);
+  if (FULL || act) x = nx;
+  return e;
+}
+
+// A renormalisation point: every lane below 2^16 takes the group's next word, in lane order.
+// All lanes load (the others drop the word), which keeps the step free of branches; the load
+// stays inside the landed part of the ring (see round_wait).
+template <bool FULL>
+__device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigned char *smem,
+                                            uint32_t ring_off, uint32_t &q, uint32_t lt) {
+  const bool need = (FULL || act) && x < kRansL;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
+  const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (kRingBytes - 1)) | ring_off;
+  const uint32_t xr = mad_lo(x, 65536u, *reinterpret_cast<const uint16_t *>(smem + a));
+  x = need ? xr : x;
+  q = mad_lo(__popc(m), 2u, q);
+}
+
+// one full step of a 12-bit stream (a renormalisation point after every step)
 template <bool FULL>
 __device__ __forceinline__ uint32_t rans_step(uint32_t &x, bool act, const uint32_t *lut,
                                               const unsigned char *smem, uint32_t ring_off,
                                               uint32_t &q, uint32_t lt) {
-  const uint32_t e = lut[x & (kRansSlots - 1)];
-  const uint32_t nx = mad_hi(e & 0xFFF00000u, x & 0xFFFFF000u, e & 0xFFFu);
-  const bool on = FULL || act;
-  if (on) x = nx;
-  const bool need = on && x < kRansL;
-  const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-  if (need) {
-    const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (kRingBytes - 1)) | ring_off;
-    x = mad_lo(x, 65536u, *reinterpret_cast<const uint16_t *>(smem + a));
-  }
-  q = mad_lo(__popc(m), 2u, q);
+  const uint32_t e = rans_decode_step<FULL, 12>(x, act, lut);
+  rans_renorm<FULL>(x, act, smem, ring_off, q, lt);
   return e;
 }
 
-// symbols of two slot-table entries as one 16-bit pair (first in the low byte)
+// symbols of two PB-bit slot-table entries as one 16-bit pair (first in the low byte)
+template <uint32_t PB = 12>
 __device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {
-  return ((e0 >> 12) & 0xFFu) | ((e1 >> 4) & 0xFF00u);
+  if constexpr (PB == 8) return __byte_perm(e0, e1, 0x0051u);
+  else return ((e0 >> PB) & 0xFFu) | ((e1 >> (PB - 8)) & 0xFF00u);
 }
 
 // Init the rings' mbarriers (lane 0 of each warp) -- call before the block-wide sync.
@@ -162,8 +184,15 @@ __device__ __forceinline__ void ring_init(WordRing &R, unsigned char *smem, unsi
 
 #endif  // __CUDACC__
 
-__host__ __device__ constexpr size_t rans_smem_bytes(uint32_t warps) {
-  return kRansSlots * 4 + warps * (kRingBytes + kNumSeg * 8);
+// bytes before the first ring: the slot table (2^pb entries), padded so that every ring starts at
+// a multiple of its own size (the word address is formed with an OR)
+__host__ __device__ constexpr uint32_t rans_lut_bytes(uint32_t pb) {
+  return ((4u << pb) + kRingBytes - 1) / kRingBytes * kRingBytes;
+}
+
+// shared memory of a CTA: the slot table, then one ring per warp, then the rings' barriers
+__host__ __device__ constexpr size_t rans_smem_bytes(uint32_t warps, uint32_t pb = 12) {
+  return rans_lut_bytes(pb) + warps * (kRingBytes + kNumSeg * 8);
 }
 
 }  // namespace eq

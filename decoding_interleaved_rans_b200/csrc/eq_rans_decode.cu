@@ -50,23 +50,29 @@ struct RansDecodeParams {
 };
 
 // ------------------------------------------------------------------------------------------------
-// one round (G steps) of one group; FULL: every lane holds a run this round
+// one round (G steps) of one group; FULL: every lane holds a run this round.  A 12-bit stream
+// renormalises after every step; an 8-bit one (G = 8) after positions 1, 3, 5 and 7, i.e. after
+// every second of its own steps, since each round gives it one whole run.
 // ------------------------------------------------------------------------------------------------
-template <bool FULL, int G, int FMT>
+template <bool FULL, int G, int FMT, uint32_t PB>
 __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
                                              const uint32_t *lut, const unsigned char *smem,
                                              const WordRing &R, uint32_t &q, uint32_t lt,
                                              uint16_t *out, float sc, bool nan_codes) {
+  static_assert(PB == 12 || G == 8, "8-bit tables need whole runs of 8");
   uint32_t e[G];
 #pragma unroll
-  for (int p = 0; p < G; ++p) e[p] = rans_step<FULL>(x, act, lut, smem, R.ring_off, q, lt);
+  for (int p = 0; p < G; ++p) {
+    e[p] = rans_decode_step<FULL, PB>(x, act, lut);
+    if (PB == 12 || (p & 1)) rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
+  }
   if (FULL || act) {
-    if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT>(e, sc, nan_codes);
-    else *out = dequant1<FMT>((e[0] >> 12) & 0xFFu, sc);
+    if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
+    else *out = dequant1<FMT>((e[0] >> PB) & 0xFFu, sc);
   }
 }
 
-template <int G, int FMT>
+template <int G, int FMT, uint32_t PB>
 __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32_t *lut,
                                                  const unsigned char *smem, uint32_t flags,
                                                  uint32_t single_sym, WordRing &R, uint64_t unit,
@@ -116,8 +122,8 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
       status |= EQ_DEV_TIMEOUT;
       break;
     }
-    if (r < full) decode_round<true, G, FMT>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
-    else decode_round<false, G, FMT>(D, x, r * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
+    if (r < full) decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
+    else decode_round<false, G, FMT, PB>(D, x, r * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
     if (q - R.off0 > 2 * nwords) {
       status |= EQ_DEV_OVERRUN;
       break;
@@ -140,11 +146,11 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   return status;
 }
 
-template <int G, int FMT>
+template <int G, int FMT, uint32_t PB>
 __global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-  unsigned char *rings = smem + kRansSlots * 4;
+  unsigned char *rings = smem + rans_lut_bytes(PB);
   uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * kRingBytes);
 
   // tensor of this CTA: the last one whose first CTA is <= blockIdx.x
@@ -158,7 +164,7 @@ __global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant_
 
   const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(D.table);
   const uint4 *src = reinterpret_cast<const uint4 *>(D.table + sizeof(RansTableHeader) / 4);
-  for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
+  for (uint32_t i = threadIdx.x; i < (1u << PB) / 4; i += blockDim.x)
     reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
   WordRing R;
   ring_init(R, smem, rings, bars, warp, lane);
@@ -167,8 +173,8 @@ __global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant_
   const uint64_t unit = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
   if (unit >= D.units) return;
   uint32_t status = 0;
-  if (hdr.magic != kRansMagic) status = EQ_DEV_CORRUPT_STATE;
-  else status = decode_group<G, FMT>(D, lut, smem, hdr.flags, hdr.single_sym, R, unit, lane);
+  if (hdr.magic != kRansMagic || hdr.prob_bits != PB) status = EQ_DEV_CORRUPT_STATE;
+  else status = decode_group<G, FMT, PB>(D, lut, smem, hdr.flags, hdr.single_sym, R, unit, lane);
   if (lane == 0) report(P.status, status);
 }
 
@@ -177,11 +183,14 @@ __global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant_
 // ------------------------------------------------------------------------------------------------
 using KernelFn = void (*)(RansDecodeParams);
 
-static KernelFn pick_kernel(uint32_t symfmt, uint32_t run) {
-  if (run == 8)
-    return symfmt == EQ_SYM_E4M3 ? rans_decode_kernel<8, EQ_SYM_E4M3> : rans_decode_kernel<8, EQ_SYM_INT8>;
-  if (run == 1)
-    return symfmt == EQ_SYM_E4M3 ? rans_decode_kernel<1, EQ_SYM_E4M3> : rans_decode_kernel<1, EQ_SYM_INT8>;
+static KernelFn pick_kernel(uint32_t symfmt, uint32_t run, uint32_t pb) {
+  const bool e4 = symfmt == EQ_SYM_E4M3;
+  if (run == 8 && pb == 12)
+    return e4 ? rans_decode_kernel<8, EQ_SYM_E4M3, 12> : rans_decode_kernel<8, EQ_SYM_INT8, 12>;
+  if (run == 8 && pb == 8)
+    return e4 ? rans_decode_kernel<8, EQ_SYM_E4M3, 8> : rans_decode_kernel<8, EQ_SYM_INT8, 8>;
+  if (run == 1 && pb == 12)
+    return e4 ? rans_decode_kernel<1, EQ_SYM_E4M3, 12> : rans_decode_kernel<1, EQ_SYM_INT8, 12>;
   return nullptr;
 }
 
@@ -189,8 +198,9 @@ static KernelFn pick_kernel(uint32_t symfmt, uint32_t run) {
 eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   if (t.version != EQ_ABI_VERSION) return EQ_ERR_ARG;
   if (t.symfmt != EQ_SYM_E4M3 && t.symfmt != EQ_SYM_INT8) return EQ_ERR_ARG;
-  if (t.prob_bits != kRansProbBits) return EQ_ERR_UNSUPPORTED;
+  if (t.prob_bits != 12 && t.prob_bits != 8) return EQ_ERR_UNSUPPORTED;
   if (t.run != 1 && t.run != 8) return EQ_ERR_UNSUPPORTED;
+  if (t.prob_bits == 8 && t.run != 8) return EQ_ERR_UNSUPPORTED;  // pairs of steps inside runs
   if (t.streams == 0 || t.streams % 32 || t.streams > 1024) return EQ_ERR_UNSUPPORTED;
   const uint64_t numel = uint64_t(t.rows) * t.cols;
   if (numel >= (1ull << 40)) return EQ_ERR_UNSUPPORTED;
@@ -205,12 +215,12 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   return EQ_OK;
 }
 
-static bool g_attr_set[64][2][2];
+static bool g_attr_set[64][2][2][2];  // device, symfmt, run == 8, prob_bits == 8
 
 static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
                               uint16_t *const *d_out, uint32_t *d_status, cudaStream_t st) {
   const eq_rans_tensor &t0 = ts[idx[0]];
-  KernelFn fn = pick_kernel(t0.symfmt, t0.run);
+  KernelFn fn = pick_kernel(t0.symfmt, t0.run, t0.prob_bits);
   if (!fn) return EQ_ERR_UNSUPPORTED;
   uint64_t total_units = 0;
   for (uint32_t i : idx) total_units += ts[i].num_chunks * (ts[i].streams / 32);
@@ -218,13 +228,13 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
   const uint64_t sms = uint64_t(device_sm_count());
   uint32_t warps = 16;
   while (warps > 1 && (total_units + warps - 1) / warps < 4 * sms) warps >>= 1;
-  const size_t smem = rans_smem_bytes(warps);
+  const size_t smem = rans_smem_bytes(warps, t0.prob_bits);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8];
+  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8][t0.prob_bits == 8];
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(rans_smem_bytes(16)));
+                                         int(rans_smem_bytes(16, t0.prob_bits)));
     if (e != cudaSuccess) return EQ_ERR_CUDA;
     attr = true;
   }
@@ -280,10 +290,10 @@ extern "C" eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uin
     if (ts[i].num_chunks && (!d_out[i] || !aligned(d_out[i], ts[i].run == 8 ? 16 : 2)))
       return EQ_ERR_ARG;
   }
-  // one launch per kernel variant (symbol format x run length)
-  std::vector<std::vector<uint32_t>> groups(4);
+  // one launch per kernel variant (symbol format x run length x table size)
+  std::vector<std::vector<uint32_t>> groups(8);
   for (uint32_t i = 0; i < n_tensors; ++i)
-    groups[(ts[i].symfmt - 1) * 2 + (ts[i].run == 8)].push_back(i);
+    groups[(ts[i].symfmt - 1) * 4 + (ts[i].run == 8) * 2 + (ts[i].prob_bits == 8)].push_back(i);
   for (auto &g : groups) {
     if (g.empty()) continue;
     eq_status s = launch_group(ts, g, d_out, d_status, static_cast<cudaStream_t>(stream));

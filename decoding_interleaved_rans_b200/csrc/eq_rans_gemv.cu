@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
   constexpr uint32_t S = 32;
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-  unsigned char *rings = smem + kRansSlots * 4;
+  unsigned char *rings = smem + rans_lut_bytes(12);
   uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * kRingBytes);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
 
   const uint64_t chunk = uint64_t(blockIdx.x) * P.warps + warp;
   if (chunk >= P.num_chunks) return;
-  uint32_t status = hdr.magic == kRansMagic ? 0u : EQ_DEV_CORRUPT_STATE;
+  uint32_t status = hdr.magic == kRansMagic && hdr.prob_bits == 12 ? 0u : EQ_DEV_CORRUPT_STATE;
   const bool single = hdr.flags & kRansFlagSingle;
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (hdr.flags & (kRansFlagNaN7F | kRansFlagNaNFF));
   const uint64_t j0 = chunk * uint64_t(P.chunk_symbols);
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __gri
   constexpr uint32_t S = 32;
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-  unsigned char *rings = smem + kRansSlots * 4;
+  unsigned char *rings = smem + rans_lut_bytes(12);
   uint64_t *bars = reinterpret_cast<uint64_t *>(rings + kTcWarps * kRingBytes);
   unsigned char *tiles = smem + rans_smem_bytes(kTcWarps);          // 2 x [16][264] bf16
   float *red = reinterpret_cast<float *>(tiles + 2 * kTcTileBytes);  // [16 warps][16 rows][16 b]
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __gri
   // a warp without a chunk, or whose chunk failed, feeds zeros
   const uint64_t chunk = uint64_t(blockIdx.x) * kTcWarps + warp;
   const bool have = chunk < P.num_chunks;
-  uint32_t status = have && hdr.magic != kRansMagic ? EQ_DEV_CORRUPT_STATE : 0u;
+  uint32_t status = have && (hdr.magic != kRansMagic || hdr.prob_bits != 12) ? EQ_DEV_CORRUPT_STATE : 0u;
   const bool single = hdr.flags & kRansFlagSingle;
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (hdr.flags & (kRansFlagNaN7F | kRansFlagNaNFF));
   uint32_t x = kRansL, nwords = 0, q = 0, n = 0;
@@ -360,7 +360,8 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   if (batch < 1 || batch > 16) return EQ_ERR_ARG;
   if (t->rows == 0 || t->cols == 0) return EQ_OK;
   if (!d_x || !d_y || !aligned(d_x, 16) || !aligned(d_y, 4)) return EQ_ERR_ARG;
-  if (t->run != 8 || t->streams != 32 || t->chunk_symbols % t->cols) return EQ_ERR_UNSUPPORTED;
+  if (t->prob_bits != 12 || t->run != 8 || t->streams != 32 || t->chunk_symbols % t->cols)
+    return EQ_ERR_UNSUPPORTED;
   const uint32_t rpc = t->chunk_symbols / t->cols;
   if (rpc > 1 && t->cols % (t->streams * 8)) return EQ_ERR_UNSUPPORTED;
   // batch >= 8 on the tensor cores when a round never straddles a chunk's 256-column tiles

@@ -15,8 +15,9 @@
 namespace eq {
 
 struct RansBuildArgs {
-  uint32_t *dst;           // device table (header + 4096 entries)
+  uint32_t *dst;           // device table (header + 2^prob_bits entries)
   uint32_t flags, single;  // header fields
+  uint32_t prob_bits;
   uint16_t freq[256];
 };
 
@@ -31,12 +32,13 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
       c += a.freq[s];
     }
     cum[256] = c;
-    RansTableHeader h{kRansMagic, a.flags, a.single, 0u};
+    RansTableHeader h{kRansMagic, a.flags, a.single, a.prob_bits};
     *reinterpret_cast<RansTableHeader *>(a.dst) = h;
   }
   __syncthreads();
   uint32_t *lut = a.dst + sizeof(RansTableHeader) / 4;
-  for (uint32_t slot = t; slot < kRansSlots; slot += blockDim.x) {
+  const uint32_t pb = a.prob_bits, slots = 1u << pb;
+  for (uint32_t slot = t; slot < slots; slot += blockDim.x) {
     // largest s with cum[s] <= slot: that symbol owns the slot
     int lo = 0, hi = 255;
     while (lo < hi) {
@@ -44,8 +46,8 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
       if (cum[mid] <= slot) lo = mid; else hi = mid - 1;
     }
     uint32_t f = a.freq[lo];
-    uint32_t fe = (f >= kRansSlots) ? 0u : f;  // a one-symbol table is handled by the flag
-    lut[slot] = (fe << 20) | (uint32_t(lo) << 12) | (slot - cum[lo]);
+    uint32_t fe = (f >= slots) ? 0u : f;  // a one-symbol table is handled by the flag
+    lut[slot] = (fe << (32 - pb)) | (uint32_t(lo) << pb) | (slot - cum[lo]);
   }
 }
 
@@ -184,13 +186,15 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
   if (!host_in || !d_tables || !aligned(d_tables, 16)) return EQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (kind == EQ_TABLE_RANS) {
-    if (prob_bits != kRansProbBits) return EQ_ERR_UNSUPPORTED;
+    if (prob_bits != 12 && prob_bits != 8) return EQ_ERR_UNSUPPORTED;
+    const uint32_t slots = 1u << prob_bits;
     RansBuildArgs a;
     a.dst = static_cast<uint32_t *>(d_tables);
+    a.prob_bits = prob_bits;
     uint64_t sum = 0;
     uint32_t used = 0, single = 0;
     for (int s = 0; s < 256; ++s) {
-      if (host_in[s] > kRansSlots) return EQ_ERR_FORMAT;
+      if (host_in[s] > slots) return EQ_ERR_FORMAT;
       a.freq[s] = uint16_t(host_in[s]);
       sum += host_in[s];
       if (host_in[s]) {
@@ -198,7 +202,7 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
         single = uint32_t(s);
       }
     }
-    if (sum != kRansSlots) return EQ_ERR_FORMAT;
+    if (sum != slots) return EQ_ERR_FORMAT;
     a.flags = (host_in[0x7F] ? kRansFlagNaN7F : 0u) | (host_in[0xFF] ? kRansFlagNaNFF : 0u) |
               (used == 1 ? kRansFlagSingle : 0u);
     a.single = used == 1 ? single : 0u;

@@ -61,7 +61,7 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
  * output channel, are flattened into one symbol stream and ANS-coded; a parallel ANS decoder
  * restores them on the GPU before the layer runs).  The pages fix no rANS variant; this one is:
  *
- *   probabilities M = 2^prob_bits (prob_bits = 12), state x in [2^16, 2^32), 16-bit words.
+ *   probabilities M = 2^prob_bits (prob_bits = 12 or 8), state x in [2^16, 2^32), 16-bit words.
  *   The row-major symbol stream is cut into chunks of chunk_symbols symbols (the last one may be
  *   shorter); chunk c is coded on its own by `streams` interleaved rANS states.  Inside a chunk,
  *   symbol j belongs to run r = j / run, stream r % streams, round r / streams, position j % run;
@@ -69,9 +69,12 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
  *   no symbol at that step.  The streams form groups of 32 (group g = streams 32g .. 32g + 31);
  *   each group reads its own word substream, so the groups of a chunk decode independently.
  *   Decoding symbol s from x: slot = x mod M, s is the symbol with cum[s] <= slot < cum[s] +
- *   freq[s], x = freq[s] * (x / M) + slot - cum[s]; then, if x < 2^16, x = x * 2^16 + the next
- *   word of the stream's group.  A well-formed chunk ends with every state at 2^16 and every
- *   word read.
+ *   freq[s], x = freq[s] * (x / M) + slot - cum[s].  At a renormalisation point, if x < 2^16,
+ *   x = x * 2^16 + the next word of the stream's group.  A 12-bit stream has a renormalisation
+ *   point after each of its steps; an 8-bit stream after every second one of its own steps
+ *   (and after its last), which is exact because two 8-bit steps shrink the state by at most
+ *   2^16; it halves the renormalisation work.  A well-formed chunk ends with every state at
+ *   2^16 and every word read.
  *   Dequantisation: out = bf16_rne( value(s) * scale[row] ), value(s) being the E4M3 value of the
  *   byte (NaN codes 0x7F/0xFF give the bf16 quiet NaN 0x7FC0 / 0xFFC0) or the byte read as int8.
  */
@@ -79,7 +82,7 @@ typedef struct {
   uint32_t version;       /* EQ_ABI_VERSION                                                    */
   uint32_t symfmt;        /* eq_symfmt                                                         */
   uint32_t rows, cols;    /* W is rows x cols, row-major; rows*cols < 2^40                     */
-  uint32_t prob_bits;     /* 12                                                                */
+  uint32_t prob_bits;     /* 12, or 8 (then run must be 8)                                      */
   uint32_t chunk_symbols; /* symbols per chunk (>= 1); a multiple of `run`                     */
   uint32_t streams;       /* interleaved states per chunk: a multiple of 32, at most 1024      */
   uint32_t run;           /* consecutive symbols per stream visit: 1 or 8; 8 needs cols % 8 == 0 */
@@ -127,14 +130,15 @@ size_t eq_table_bytes(eq_table_kind kind);
  * Build the device decode tables of one tensor into d_tables (eq_table_bytes(kind) bytes,
  * 16-byte aligned, caller-owned).  The table contents travel as kernel arguments: no host
  * buffer outlives the call and no copy engine is used.
- *   EQ_TABLE_RANS: host_in[256] = symbol frequencies, summing to 2^prob_bits (prob_bits = 12).
+ *   EQ_TABLE_RANS: host_in[256] = symbol frequencies, summing to 2^prob_bits (prob_bits = 12
+ *     or 8).
  *     Builds the slot table: one 32-bit entry per slot holding the slot's symbol, its frequency
  *     and slot - cum[symbol].
  *   EQ_TABLE_HUFF: host_in[256] = code length of each exponent value (0 = absent), prob_bits
  *     ignored.  Builds the hierarchical lookup tables of the DFloat11 page ("Decodificacion
  *     basada en LUT jerarquicas": the code tree cut into height-8 subtrees, each a 256-entry
- *     table) and, from them, a 4096-entry window table that returns every code lying wholly in
- *     the next 12 bits (up to four) with one lookup.  EQ_ERR_FORMAT if a length exceeds 32 or the
+ *     table) and, from them, a 2048-entry window table that returns every code lying wholly in
+ *     the next 11 bits (up to four) with one lookup.  EQ_ERR_FORMAT if a length exceeds 32 or the
  *     lengths violate the Kraft inequality; EQ_ERR_UNSUPPORTED if more than 32 subtables would
  *     be needed.
  */
@@ -143,7 +147,7 @@ eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in, uint32_t 
 
 /*
  * Decode n_tensors rANS-coded weights to bf16 (one launch per group of tensors that share
- * symfmt, streams and run).  d_out[i] points to rows*cols bf16 values (16-byte aligned) for
+ * symfmt, run and prob_bits).  d_out[i] points to rows*cols bf16 values (16-byte aligned) for
  * tensor i; the array d_out itself is host memory.  Decoding all tensors of a transformer block
  * in one call follows the pages' block-wise decompression (DFloat11 page, "Descompresion por
  * bloque transformer"; "Float8@2bits" summary: decompression alternates with the forward
@@ -160,7 +164,8 @@ eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uint16_t *cons
  * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].  batch 1..16; for batch >= 8
  * (and chunk_symbols % 256 == 0) the product of each 16-row x 256-column decoded tile with x runs
  * on the tensor cores (mma, bf16 in, fp32 accumulate).
- * Requires run == 8, streams == 32 (one warp owns a chunk, so its sums never leave the warp)
+ * Requires prob_bits == 12, run == 8, streams == 32 (one warp owns a chunk, so its sums never
+ * leave the warp)
  * and whole rows per chunk (chunk_symbols a multiple of cols); a chunk of several rows also needs
  * cols % 256 == 0, so that one decode round never straddles two rows.  Otherwise
  * EQ_ERR_UNSUPPORTED.

@@ -50,7 +50,8 @@ def test_int8_8k_full_size(eq, orc):
     """The 8192x8192 Int8 workload in the bench's launch configuration, every element."""
     wl = synth.WORKLOADS["int8_8k"]
     sym, sc = quantized(orc, wl.tensors[0], orc.INT8, wl.int8_div)
-    h = orc.rans_encode(sym, sc, orc.INT8, wl.chunk_symbols, wl.streams, wl.run)
+    h = orc.rans_encode(sym, sc, orc.INT8, wl.chunk_symbols, wl.streams, wl.run,
+                        prob_bits=wl.prob_bits)
     (out,), st = run_decode(eq, [h])
     assert st == 0
     assert np.array_equal(out, expect(orc, sym, sc, orc.INT8))
@@ -134,7 +135,8 @@ def test_product_encoder_stream_decodes(eq, orc):
     wl = synth.WORKLOADS["int8_8k"]
     w = wl.tensors[0].generate(row_lo=0, row_hi=512)
     sym, sc = eq.codec.quantize(w, eq.EQ_SYM_INT8, wl.int8_div)
-    h = eq.codec.rans_encode(sym, sc, eq.EQ_SYM_INT8, wl.chunk_symbols, wl.streams, wl.run)
+    h = eq.codec.rans_encode(sym, sc, eq.EQ_SYM_INT8, wl.chunk_symbols, wl.streams, wl.run,
+                             prob_bits=wl.prob_bits)
     (out,), st = run_decode(eq, [h])
     osym, osc = orc.quantize(w, orc.INT8, wl.int8_div)
     assert st == 0 and np.array_equal(out, expect(orc, osym, osc, orc.INT8))

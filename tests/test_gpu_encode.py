@@ -73,15 +73,38 @@ def test_encode_matches_oracle(eq, orc, rows, cols, chunk, S, G):
     assert np.array_equal(eq.bf16_bits(out).ravel(), orc.dequant(osym, osc, orc.E4M3).ravel())
 
 
+@pytest.mark.parametrize("rows,cols,chunk,S", [
+    (64, 1024, 16384, 32), (256, 4096, 65536, 128), (37, 200, 1000, 64), (8, 512, 4096, 256),
+    (5, 104, 0, 96)])
+def test_encode_8bit_matches_oracle(eq, orc, rows, cols, chunk, S):
+    w = synth.laplace_clipped(rows, cols, 0.01, 0.06, rows + S)
+    osym, osc = orc.quantize(w, orc.INT8, synth.INT8_DIV_LAPLACE_8K)
+    h = orc.rans_encode(osym, osc, orc.INT8, chunk, S, 8, prob_bits=8)
+    t = eq.rans_encode_device(cuda(osym), cuda(osc.view(np.int16)), 2, chunk, S, 8, prob_bits=8)
+    torch.cuda.synchronize()
+    assert np.array_equal(t.word_off.cpu().numpy().view(np.uint64), h.word_off)
+    assert np.array_equal(t.states.cpu().numpy().view(np.uint32), h.states)
+    total = int(h.word_off[-1])
+    assert np.array_equal(t.words.cpu().numpy().view(np.uint16)[:total], h.words[:total])
+    (out,), st = eq.decode([t])
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(eq.bf16_bits(out).ravel(), orc.dequant(osym, osc, orc.INT8).ravel())
+
+
 def test_full_pipeline_int8_workload(eq, orc):
-    """fp32 weights on the GPU -> quantise -> histogram -> frequencies -> encode -> decode."""
+    """fp32 weights on the GPU -> quantise -> histogram -> frequencies -> encode -> decode, in the
+    workload's own table size."""
     wl = synth.WORKLOADS["int8_8k"]
     w = wl.tensors[0].generate(row_lo=0, row_hi=1024)
     sym, sc = eq.quantize_device(cuda(w), 2, wl.int8_div)
-    t = eq.rans_encode_device(sym, sc, 2, wl.chunk_symbols, wl.streams, wl.run)
+    t = eq.rans_encode_device(sym, sc, 2, wl.chunk_symbols, wl.streams, wl.run,
+                              prob_bits=wl.prob_bits)
     osym, osc = orc.quantize(w, orc.INT8, wl.int8_div)
-    h = orc.rans_encode(osym, osc, orc.INT8, wl.chunk_symbols, wl.streams, wl.run)
+    h = orc.rans_encode(osym, osc, orc.INT8, wl.chunk_symbols, wl.streams, wl.run,
+                        prob_bits=wl.prob_bits)
     assert np.array_equal(t.word_off.cpu().numpy().view(np.uint64), h.word_off)
+    assert np.array_equal(t.states.cpu().numpy().view(np.uint32), h.states)
     (out,), st = eq.decode([t])
     torch.cuda.synchronize()
     assert int(st.item()) == 0

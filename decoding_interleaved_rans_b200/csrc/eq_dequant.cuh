@@ -50,7 +50,7 @@ __device__ __forceinline__ uint32_t dequant2(uint32_t pair, float scale, bool na
 }
 
 // the eight symbols of a round, taken from their PB-bit slot-table entries (symbol in bits
-// PB+7..PB), scaled -> eight bf16 (one 16-byte store)
+// 19..12 of 12-bit entries, 23..16 of 8-bit ones), scaled -> eight bf16 (one 16-byte store)
 template <int FMT, uint32_t PB = 12>
 __device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, bool nan_codes) {
   uint32_t o[4];
@@ -58,11 +58,12 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, b
   for (int k = 0; k < 4; ++k) {
     if constexpr (FMT == EQ_SYM_INT8) {
       // the symbol byte sign-extended straight out of the entry
-      const float v0 = float(int32_t(e[2 * k] << (24 - PB)) >> 24);
-      const float v1 = float(int32_t(e[2 * k + 1] << (24 - PB)) >> 24);
+      constexpr int kUp = PB == 8 ? 8 : 24 - int(PB);
+      const float v0 = float(int32_t(e[2 * k] << kUp) >> 24);
+      const float v1 = float(int32_t(e[2 * k + 1] << kUp) >> 24);
       o[k] = pack_bf16x2(v0 * scale, v1 * scale);
     } else {
-      if constexpr (PB == 8) o[k] = dequant2<FMT>(__byte_perm(e[2 * k], e[2 * k + 1], 0x0051u), scale, nan_codes);
+      if constexpr (PB == 8) o[k] = dequant2<FMT>(__byte_perm(e[2 * k], e[2 * k + 1], 0x0062u), scale, nan_codes);
       else o[k] = dequant2<FMT>(((e[2 * k] >> PB) & 0xFFu) | ((e[2 * k + 1] >> (PB - 8)) & 0xFF00u), scale, nan_codes);
     }
   }

@@ -128,16 +128,29 @@ __device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
-// The decoding half of a step with a PB-bit table (entry: f in the top PB bits, symbol above
-// the low PB bits, slot - cum in them); returns the entry.
+// the low 16 bits of v, sign-extended (one byte permute that replicates byte 1's sign)
+__device__ __forceinline__ uint32_t sext16(uint32_t v) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, 0, 0x9910;" : "=r"(d) : "r"(v));
+  return d;
+}
+
+// The decoding half of a step with a PB-bit table (entry layouts in eq_internal.cuh); returns
+// the entry.
 template <bool FULL, uint32_t PB>
 __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, const uint32_t *lut) {
   constexpr uint32_t kLow = (1u << PB) - 1;
   const uint32_t e = lut[x & kLow];
-  const uint32_t nx = mad_hi(e & ~(0xFFFFFFFFu >> PB), x & ~kLow, e & kLow);
+  uint32_t nx;
+  if constexpr (PB == 8) nx = mad_hi(e & 0xFF000000u, x, sext16(e));
+  else nx = mad_hi(e & ~(0xFFFFFFFFu >> PB), x & ~kLow, e & kLow);
   if (FULL || act) x = nx;
   return e;
 }
+
+// the symbol byte of a PB-bit entry
+template <uint32_t PB>
+constexpr uint32_t kSymShift = PB == 8 ? 16 : PB;
 
 // A renormalisation point: every lane below 2^16 takes the group's next word, in lane order.
 // All lanes load (the others drop the word), which keeps the step free of branches; the load
@@ -166,7 +179,7 @@ __device__ __forceinline__ uint32_t rans_step(uint32_t &x, bool act, const uint3
 // symbols of two PB-bit slot-table entries as one 16-bit pair (first in the low byte)
 template <uint32_t PB = 12>
 __device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {
-  if constexpr (PB == 8) return __byte_perm(e0, e1, 0x0051u);
+  if constexpr (PB == 8) return __byte_perm(e0, e1, 0x0062u);
   else return ((e0 >> PB) & 0xFFu) | ((e1 >> (PB - 8)) & 0xFF00u);
 }
 

@@ -68,7 +68,7 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
   }
   if (FULL || act) {
     if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
-    else *out = dequant1<FMT>((e[0] >> PB) & 0xFFu, sc);
+    else *out = dequant1<FMT>((e[0] >> kSymShift<PB>) & 0xFFu, sc);
   }
 }
 
@@ -117,27 +117,35 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   uint32_t col = uint32_t(jrun - row * cols);
   float sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
   uint16_t *out = D.out + jrun;
-  for (uint32_t r = 0; r < rounds; ++r) {
+  // ring checks once per round (12-bit: up to 256 words a round), or once per two rounds
+  // (8-bit: up to 128 words a round); round_wait covers 256 words and one more
+  constexpr uint32_t kRoundsPerCheck = PB == 8 ? 2 : 1;
+  for (uint32_t r = 0; r < rounds; r += kRoundsPerCheck) {
     if (!R.round_wait(q)) {
       status |= EQ_DEV_TIMEOUT;
       break;
     }
-    if (r < full) decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
-    else decode_round<false, G, FMT, PB>(D, x, r * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
+#pragma unroll
+    for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
+      const uint32_t rk = r + k;
+      if (kRoundsPerCheck > 1 && rk >= rounds) break;
+      if (rk < full) decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
+      else decode_round<false, G, FMT, PB>(D, x, rk * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
+      out += step;
+      col += step;
+      if (col >= cols) {
+        do {
+          col -= cols;
+          ++row;
+        } while (col >= cols);
+        if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
+      }
+    }
     if (q - R.off0 > 2 * nwords) {
       status |= EQ_DEV_OVERRUN;
       break;
     }
     R.round_refill(q, lane);
-    out += step;
-    col += step;
-    if (col >= cols) {
-      do {
-        col -= cols;
-        ++row;
-      } while (col >= cols);
-      if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
-    }
   }
   if (!status && !__all_sync(0xFFFFFFFFu, q - R.off0 == 2 * nwords && x == kRansL))
     status |= EQ_DEV_CORRUPT_STATE;

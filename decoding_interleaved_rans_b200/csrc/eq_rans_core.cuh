@@ -128,22 +128,42 @@ __device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
-// the low 16 bits of v, sign-extended (one byte permute that replicates byte 1's sign)
-__device__ __forceinline__ uint32_t sext16(uint32_t v) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, 0, 0x9910;" : "=r"(d) : "r"(v));
-  return d;
-}
-
 // The decoding half of a step with a PB-bit table (entry layouts in eq_internal.cuh); returns
-// the entry.
+// the entry.  Written as one PTX block: slot = x mod 2^PB, its entry from the shared-memory
+// table, then the multiply-high-add (with ptxas left to pick the address arithmetic, the step
+// took about 1.5 more instructions).  Volatile, so it is never hoisted above the barrier that
+// publishes the table.
 template <bool FULL, uint32_t PB>
 __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, const uint32_t *lut) {
-  constexpr uint32_t kLow = (1u << PB) - 1;
-  const uint32_t e = lut[x & kLow];
-  uint32_t nx;
-  if constexpr (PB == 8) nx = mad_hi(e & 0xFF000000u, x, sext16(e));
-  else nx = mad_hi(e & ~(0xFFFFFFFFu >> PB), x & ~kLow, e & kLow);
+  const uint32_t base = uint32_t(__cvta_generic_to_shared(lut));
+  uint32_t e, nx;
+  if constexpr (PB == 8) {
+    asm volatile(
+        "{\n\t.reg .b32 a, f, d;\n\t"
+        "and.b32 a, %2, 255;\n\t"
+        "shl.b32 a, a, 2;\n\t"
+        "add.u32 a, a, %3;\n\t"
+        "ld.shared.u32 %1, [a];\n\t"
+        "and.b32 f, %1, 0xFF000000;\n\t"
+        "prmt.b32 d, %1, 0, 0x9910;\n\t"  // the signed correction, sign-extended
+        "mad.hi.u32 %0, f, %2, d;\n\t}"
+        : "=r"(nx), "=r"(e)
+        : "r"(x), "r"(base));
+  } else {
+    static_assert(PB == 12, "12- or 8-bit tables");
+    asm volatile(
+        "{\n\t.reg .b32 a, f, xm, b;\n\t"
+        "and.b32 a, %2, 4095;\n\t"
+        "shl.b32 a, a, 2;\n\t"
+        "add.u32 a, a, %3;\n\t"
+        "ld.shared.u32 %1, [a];\n\t"
+        "and.b32 f, %1, 0xFFF00000;\n\t"
+        "and.b32 xm, %2, 0xFFFFF000;\n\t"
+        "and.b32 b, %1, 4095;\n\t"
+        "mad.hi.u32 %0, f, xm, b;\n\t}"
+        : "=r"(nx), "=r"(e)
+        : "r"(x), "r"(base));
+  }
   if (FULL || act) x = nx;
   return e;
 }

@@ -15,7 +15,7 @@ import math
 import os
 import subprocess
 from concurrent.futures import ThreadPoolExecutor
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import numpy as np
 
@@ -61,6 +61,8 @@ def lib() -> C.CDLL:
             "orc_f32_to_e4m3": (C.c_uint8, [C.c_float]),
             "orc_quantize_e4m3": (None, [p, i64, i64, p, p]),
             "orc_quantize_int8": (None, [p, i64, i64, C.c_float, p, p]),
+            "orc_super_weights": (i64, [p, i64, i64, C.c_double, i64, p, p]),
+            "orc_quantize_excluding": (None, [p, i64, i64, i32, C.c_float, p, i64, p, p]),
             "orc_dequant_one": (C.c_uint16, [C.c_uint8, C.c_uint16, i32]),
             "orc_dequant": (None, [p, p, i64, i64, i32, p]),
             "orc_rans_normalize": (i32, [p, u32, p]),
@@ -201,6 +203,9 @@ class RansTensor:
     word_off: np.ndarray  # uint64[num_chunks * groups + 1]
     words: np.ndarray     # uint16
     scales: np.ndarray    # uint16[rows] (bf16 bits)
+    # super weights written back over the decoded values: flat indices (sorted) and bf16 bits
+    patch_idx: np.ndarray = field(default_factory=lambda: np.zeros(0, np.uint64))
+    patch_val: np.ndarray = field(default_factory=lambda: np.zeros(0, np.uint16))
 
     @property
     def numel(self) -> int:
@@ -221,9 +226,10 @@ class RansTensor:
 
     @property
     def compressed_bytes(self) -> int:
-        """Everything the decoder reads: words, states, offsets, scales, frequency table."""
+        """Everything the decoder reads: words, states, offsets, scales, frequency table and the
+        super-weight list."""
         return (self.payload_bytes + self.states.nbytes + self.word_off.nbytes
-                + self.scales.nbytes + 256 * 2)
+                + self.scales.nbytes + 256 * 2 + self.patch_idx.nbytes + self.patch_val.nbytes)
 
 
 def rans_freqs(sym: np.ndarray, prob_bits: int = PROB_BITS) -> np.ndarray:
@@ -313,7 +319,8 @@ def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols:
 
 
 def rans_decode_bf16(t: RansTensor, chunks=None, threads: int | None = 1):
-    """Decode chunks (default: all) and dequantise to bf16.  Returns (status, uint16 [rows*cols]).
+    """Decode chunks (default: all), dequantise to bf16 and write the super weights back.
+    Returns (status, uint16 [rows*cols]).
 
     Only the decoded chunks' spans of the output are written (the rest stays zero)."""
     out = np.zeros(t.numel, dtype=np.uint16)
@@ -336,7 +343,46 @@ def rans_decode_bf16(t: RansTensor, chunks=None, threads: int | None = 1):
         with ThreadPoolExecutor(nthr) as ex:
             rcs = list(ex.map(run, spans))
     rc = next((r for r in rcs if r), 0)
+    if t.patch_idx.size:
+        done = np.zeros(t.num_chunks, bool)
+        done[chunks] = True
+        mine = done[(t.patch_idx // chunk).astype(np.int64)]
+        out[t.patch_idx[mine].astype(np.int64)] = t.patch_val[mine]
     return rc, out
+
+
+def super_weights(w: np.ndarray, tau: float = 20.0):
+    """Super weights of a tensor: |w| > tau * rms(w).  Returns (flat indices uint64 sorted,
+    bf16 bits uint16)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    n = lib().orc_super_weights(_p(w), rows, cols, float(tau), 0, None, None)
+    if n < 0:
+        raise ValueError("bad arguments")
+    idx = np.zeros(max(1, n), np.uint64)
+    val = np.zeros(max(1, n), np.uint16)
+    lib().orc_super_weights(_p(w), rows, cols, float(tau), n, _p(idx), _p(val))
+    return idx[:n], val[:n]
+
+
+def quantize_excluding(w: np.ndarray, symfmt: int, int8_div: float, idx: np.ndarray):
+    """AbsMax quantisation with the listed positions left out of their rows' scales (symbol 0).
+    Returns (symbols uint8 [rows, cols], scales uint16 [rows])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    idx = np.ascontiguousarray(idx, dtype=np.uint64)
+    sym = np.empty((rows, cols), np.uint8)
+    sc = np.empty(rows, np.uint16)
+    lib().orc_quantize_excluding(_p(w), rows, cols, symfmt, float(int8_div),
+                                 _p(idx) if idx.size else None, idx.size, _p(sym), _p(sc))
+    return sym, sc
+
+
+def patch_bf16(out: np.ndarray, idx: np.ndarray, val: np.ndarray) -> np.ndarray:
+    """Decoded bf16 weights with the super weights written back (a copy)."""
+    o = np.array(out, dtype=np.uint16, copy=True)
+    o.reshape(-1)[np.asarray(idx, np.int64)] = val
+    return o
 
 
 # ----------------------------------------------------------------------------------------------

@@ -161,6 +161,53 @@ void orc_quantize_int8(const float *w, int64_t rows, int64_t cols, float div, ui
 }
 
 /* ============================================================================================
+ * Super-weight exclusion ("Float8@2bits" summary, section "Manejo de Pesos Superiores": for Int8
+ * bases, extreme outliers are detected and kept out of the entropy optimisation, so they do not
+ * crush the rest of their channel).  Reading: a weight is a super weight when
+ * |w| > tau * rms(w), rms over the whole tensor in binary64; super weights are stored exactly as
+ * bf16(w) in a list sorted by flat row-major index, their symbol is 0 and they take no part in
+ * their row's AbsMax scale; decoding writes them back over the decoded value.
+ * ========================================================================================== */
+
+/* Returns the number of super weights (writing at most max_out of them), or -1 on bad input. */
+int64_t orc_super_weights(const float *w, int64_t rows, int64_t cols, double tau, int64_t max_out,
+                          uint64_t *idx, uint16_t *val) {
+  if (rows < 0 || cols < 0 || tau <= 0.0) return -1;
+  const int64_t n = rows * cols;
+  double ss = 0.0;
+  for (int64_t j = 0; j < n; ++j) ss += (double)w[j] * (double)w[j];
+  const double limit = n ? tau * sqrt(ss / (double)n) : 0.0;
+  int64_t k = 0;
+  for (int64_t j = 0; j < n; ++j)
+    if (fabs((double)w[j]) > limit) {
+      if (k < max_out) {
+        idx[k] = (uint64_t)j;
+        val[k] = orc_f32_to_bf16(w[j]);
+      }
+      ++k;
+    }
+  return k;
+}
+
+/* AbsMax quantisation (symfmt 1 = E4M3, 2 = Int8) of w with the listed positions excluded: they
+ * take no part in their row's scale and get symbol 0.  idx sorted ascending, n entries. */
+void orc_quantize_excluding(const float *w, int64_t rows, int64_t cols, int symfmt, float div,
+                            const uint64_t *idx, int64_t n, uint8_t *sym, uint16_t *scale) {
+  uint8_t *skip = (uint8_t *)calloc((size_t)(rows * cols > 0 ? rows * cols : 1), 1);
+  for (int64_t i = 0; i < n; ++i) skip[idx[i]] = 1;
+  float *row = (float *)malloc((size_t)(cols > 0 ? cols : 1) * sizeof(float));
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) row[c] = skip[r * cols + c] ? 0.0f : w[r * cols + c];
+    if (symfmt == 1)
+      orc_quantize_e4m3(row, 1, cols, sym + r * cols, scale + r);
+    else
+      orc_quantize_int8(row, 1, cols, div, sym + r * cols, scale + r);
+  }
+  free(row);
+  free(skip);
+}
+
+/* ============================================================================================
  * Dequantisation: bf16( value(q) * scale[row] ); the product is exact in binary64
  * (at most 7 x 8 significant bits), so there is exactly one rounding.
  * symfmt: 1 = E4M3, 2 = Int8.

@@ -114,6 +114,20 @@ def activations(batch: int, cols: int, seed: int, tensor: int = 1000) -> np.ndar
     return bf16_normal(batch, cols, 1.0, seed, tensor)
 
 
+def plant_super_weights(w: np.ndarray, n: int, seed: int, lo: float = 0.5,
+                        hi: float = 2.0) -> list:
+    """Overwrite n seeded positions of w (in place, distinct rows) with super weights: magnitude
+    uniform in [lo, hi), random sign; LLaMA's super weights sit about 100x above the typical
+    weight.  Returns the flat indices, sorted."""
+    rows, cols = w.shape
+    g = _rng(seed, 0, 7)
+    rs = g.choice(rows, size=min(n, rows), replace=False)
+    cs = g.integers(0, cols, size=rs.size)
+    mags = g.uniform(lo, hi, size=rs.size) * np.where(g.integers(0, 2, size=rs.size) > 0, 1, -1)
+    w[rs, cs] = mags.astype(np.float32)
+    return sorted(int(r) * cols + int(c) for r, c in zip(rs, cs))
+
+
 def random_bytes(n: int, seed: int) -> np.ndarray:
     """Uniform random bytes (used by fault-injection tests)."""
     return _rng(seed, 0, 0).integers(0, 256, n, dtype=np.uint8)

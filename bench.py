@@ -336,6 +336,34 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                 "bits_per_param": 8 * dh.compressed_bytes / dh.n,
                 "kernel": "huff_decode_kernel"})
     del dh, ob
+    # super weights: the Int8 workload with 6 planted outliers (50-200x the typical weight), kept
+    # exactly in the patch list and out of their rows' scales; the decode writes them back
+    wl = synth.WORKLOADS["int8_8k"]
+    w = wl.tensors[0].generate()
+    synth.plant_super_weights(w, 6, 2)
+    pidx, pval = eq.codec.super_weights(w)
+    sym, sc = eq.codec.quantize_excluding(w, eq.EQ_SYM_INT8, wl.int8_div, pidx)
+    hs = eq.codec.rans_encode(sym, sc, eq.EQ_SYM_INT8, wl.chunk_symbols, wl.streams, wl.run,
+                              prob_bits=wl.prob_bits)
+    hs.patch_idx, hs.patch_val = pidx, pval
+    rows_sw = sorted({int(j) // w.shape[1] for j in pidx})
+    psym, psc = eq.codec.quantize(w[rows_sw], eq.EQ_SYM_INT8, wl.int8_div)
+    collapsed = float((psym == 0).mean())
+    del w, sym, sc, psym, psc
+    ts_ = eq.DeviceRans.upload(hs, dev)
+    osw = torch.empty(hs.rows, hs.cols, dtype=torch.bfloat16, device=dev)
+    st = eq.new_status(dev)
+    tsw = time_steps(lambda: eq.decode([ts_], [osw], st, stream), steps, 3, flush, stream)
+    assert int(st.item()) == 0
+    sec = statistics.mean(tsw)
+    alg = ts_.compressed_bytes + 2 * ts_.numel
+    out.append({"what": "Int8 8192x8192 with 6 super weights (patch list written back in the "
+                        "decode epilogue), 8-bit table", "params": ts_.numel, "ms": sec * 1e3,
+                "params_per_s": ts_.numel / sec, "gbs": alg / sec / 1e9,
+                "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"], "super_weights": int(pidx.size),
+                "zero_symbols_in_their_rows_without_exclusion": collapsed,
+                "kernel": "rans_decode_kernel<run 8, Int8, 8-bit table> + patch epilogue"})
+    del ts_, osw, hs
     # GPU compressor: fp32 weights in HBM -> quantise, histogram, frequency table (host), rANS
     # plan + encode; wall clock around the whole call (it reads the word total back once)
     wl = synth.WORKLOADS["int8_8k"]

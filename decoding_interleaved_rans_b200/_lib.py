@@ -16,13 +16,13 @@ EQ_DEV_CORRUPT_STATE, EQ_DEV_OVERRUN, EQ_DEV_BAD_CODE = 1, 2, 4
 EQ_DEV_COUNT_MISMATCH, EQ_DEV_TIMEOUT = 8, 16
 EQ_SYM_E4M3, EQ_SYM_INT8 = 1, 2
 EQ_TABLE_RANS, EQ_TABLE_HUFF = 1, 2
-EQ_ABI_VERSION = 1
+EQ_ABI_VERSION = 2
 
 # every exported function of include/eq.h and include/eq_encode.h
 EXPORTS = ("eq_table_bytes", "eq_build_tables", "eq_decode", "eq_decode_gemv",
            "eq_huff_bf16_decode", "eq_mlp_scratch_bytes", "eq_mlp_decode", "eq_mlp_decode_noalloc",
            "eq_status_string",
-           "eq_abi_version", "eq_quantize_host",
+           "eq_abi_version", "eq_quantize_host", "eq_super_weights_host", "eq_quantize_excluding_host",
            "eq_rans_freqs_host", "eq_rans_encode_host", "eq_huff_lengths_host",
            "eq_huff_plan_host", "eq_huff_encode_host", "eq_free_host", "eq_rans_normalize_host",
            "eq_quantize_device",
@@ -41,7 +41,8 @@ class RansTensorDesc(C.Structure):
                 ("cols", C.c_uint32), ("prob_bits", C.c_uint32), ("chunk_symbols", C.c_uint32),
                 ("streams", C.c_uint32), ("run", C.c_uint32), ("num_chunks", C.c_uint64),
                 ("states", C.c_void_p), ("word_off", C.c_void_p), ("words", C.c_void_p),
-                ("scales", C.c_void_p), ("tables", C.c_void_p)]
+                ("scales", C.c_void_p), ("tables", C.c_void_p), ("n_patch", C.c_uint64),
+                ("patch_idx", C.c_void_p), ("patch_val", C.c_void_p)]
 
 
 class HuffTensorDesc(C.Structure):
@@ -80,6 +81,10 @@ def lib() -> C.CDLL:
                 "eq_status_string": (C.c_char_p, [i32]),
                 "eq_abi_version": (u32, []),
                 "eq_quantize_host": (i32, [p, u32, u32, u32, C.c_float, p, p, u32]),
+                "eq_super_weights_host": (i32, [p, u32, u32, C.c_double, u64, p, p,
+                                                C.POINTER(C.c_uint64)]),
+                "eq_quantize_excluding_host": (i32, [p, u32, u32, u32, C.c_float, p, u64, p, p,
+                                                     u32]),
                 "eq_rans_freqs_host": (i32, [p, u64, u32, p]),
                 "eq_rans_encode_host": (i32, [p, u32, u32, p, u32, u32, u32, u32, p, p,
                                               C.POINTER(C.c_void_p), C.POINTER(C.c_uint64)]),

@@ -61,25 +61,35 @@ class DeviceRans:
     words: torch.Tensor
     scales: torch.Tensor
     tables: torch.Tensor
+    patch_idx: torch.Tensor | None = None  # super weights: int64 flat indices, sorted
+    patch_val: torch.Tensor | None = None  # their bf16 bits (int16)
 
     @property
     def numel(self) -> int:
         return self.rows * self.cols
 
     @property
+    def n_patch(self) -> int:
+        return 0 if self.patch_idx is None else int(self.patch_idx.numel())
+
+    @property
     def compressed_bytes(self) -> int:
-        """Bytes the decoder reads from memory: words in use, states, offsets, scales, table."""
+        """Bytes the decoder reads from memory: words in use, states, offsets, scales, table and
+        the super-weight list."""
         used_words = int(self.word_off[-1].item()) if self.num_chunks else 0
         return (2 * used_words + 4 * self.states.numel() + 8 * self.word_off.numel()
-                + 2 * self.scales.numel() + 256 * 2)
+                + 2 * self.scales.numel() + 256 * 2 + 10 * self.n_patch)
 
     def desc(self) -> L.RansTensorDesc:
         chunk = self.chunk_symbols if self.chunk_symbols else self.cols
+        npatch = self.n_patch
         return L.RansTensorDesc(L.EQ_ABI_VERSION, self.symfmt, self.rows, self.cols,
                                 self.prob_bits, chunk, self.streams, self.run, self.num_chunks,
                                 self.states.data_ptr(), self.word_off.data_ptr(),
                                 self.words.data_ptr(), self.scales.data_ptr(),
-                                self.tables.data_ptr())
+                                self.tables.data_ptr(), npatch,
+                                self.patch_idx.data_ptr() if npatch else None,
+                                self.patch_val.data_ptr() if npatch else None)
 
     @classmethod
     def upload(cls, h, device="cuda", stream=None) -> "DeviceRans":
@@ -101,6 +111,10 @@ class DeviceRans:
                 _dev(np.asarray(h.scales, np.uint16), device, np.int16),
                 torch.empty(table_bytes(L.EQ_TABLE_RANS), dtype=torch.uint8, device=device))
         build_tables(L.EQ_TABLE_RANS, h.freqs, t.prob_bits, t.tables, stream)
+        pidx = getattr(h, "patch_idx", None)
+        if pidx is not None and len(pidx):
+            t.patch_idx = _dev(np.asarray(pidx, np.uint64), device, np.int64)
+            t.patch_val = _dev(np.asarray(h.patch_val, np.uint16), device, np.int16)
         return t
 
 

@@ -6,7 +6,7 @@ containers hold exactly the arrays DeviceRans.upload / DeviceHuff.upload expect.
 from __future__ import annotations
 
 import ctypes as C
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import numpy as np
 
@@ -32,6 +32,9 @@ class HostRans:
     word_off: np.ndarray
     words: np.ndarray
     scales: np.ndarray
+    # super weights written back after decoding: flat indices (sorted), bf16 bits
+    patch_idx: np.ndarray = field(default_factory=lambda: np.zeros(0, np.uint64))
+    patch_val: np.ndarray = field(default_factory=lambda: np.zeros(0, np.uint16))
 
     @property
     def numel(self) -> int:
@@ -58,6 +61,35 @@ def quantize(w: np.ndarray, symfmt: int, int8_div: float = 0.0, threads: int = 0
     sc = np.empty(rows, np.uint16)
     L.check(L.lib().eq_quantize_host(_p(w), rows, cols, symfmt, float(int8_div), _p(sym), _p(sc),
                                      threads), "eq_quantize_host")
+    return sym, sc
+
+
+def super_weights(w: np.ndarray, tau: float = 20.0):
+    """Super weights (|w| > tau * rms(w)): (flat indices uint64 sorted, bf16 bits uint16)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    n = C.c_uint64()
+    L.check(L.lib().eq_super_weights_host(_p(w), rows, cols, float(tau), 0, None, None,
+                                          C.byref(n)), "eq_super_weights_host")
+    idx = np.zeros(max(1, n.value), np.uint64)
+    val = np.zeros(max(1, n.value), np.uint16)
+    L.check(L.lib().eq_super_weights_host(_p(w), rows, cols, float(tau), n.value, _p(idx),
+                                          _p(val), C.byref(n)), "eq_super_weights_host")
+    return idx[:n.value], val[:n.value]
+
+
+def quantize_excluding(w: np.ndarray, symfmt: int, int8_div: float, idx: np.ndarray,
+                       threads: int = 0):
+    """AbsMax quantisation with the listed positions (sorted flat indices) left out of their
+    rows' scales and coded as symbol 0."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    rows, cols = w.shape
+    idx = np.ascontiguousarray(idx, dtype=np.uint64)
+    sym = np.empty((rows, cols), np.uint8)
+    sc = np.empty(rows, np.uint16)
+    L.check(L.lib().eq_quantize_excluding_host(_p(w), rows, cols, symfmt, float(int8_div),
+                                               _p(idx) if idx.size else None, idx.size, _p(sym),
+                                               _p(sc), threads), "eq_quantize_excluding_host")
     return sym, sc
 
 

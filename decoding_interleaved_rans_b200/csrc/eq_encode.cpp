@@ -101,6 +101,59 @@ extern "C" eq_status eq_quantize_host(const float *w, uint32_t rows, uint32_t co
   return EQ_OK;
 }
 
+extern "C" eq_status eq_super_weights_host(const float *w, uint32_t rows, uint32_t cols,
+                                           double tau, uint64_t max_out, uint64_t *idx,
+                                           uint16_t *val, uint64_t *n_out) {
+  const uint64_t n = uint64_t(rows) * cols;
+  if (!n_out || (n && !w) || !(tau > 0.0) || (max_out && (!idx || !val))) return EQ_ERR_ARG;
+  std::vector<double> part(rows, 0.0);
+  parallel_for(rows, 0, [&](uint64_t r) {
+    double ss = 0.0;
+    for (uint32_t c = 0; c < cols; ++c) ss += double(w[r * cols + c]) * double(w[r * cols + c]);
+    part[r] = ss;
+  });
+  double ss = 0.0;
+  for (double v : part) ss += v;
+  const double limit = n ? tau * std::sqrt(ss / double(n)) : 0.0;
+  uint64_t k = 0;
+  for (uint64_t j = 0; j < n; ++j)
+    if (std::fabs(double(w[j])) > limit) {
+      if (k < max_out) {
+        idx[k] = j;
+        val[k] = to_bf16(w[j]);
+      }
+      ++k;
+    }
+  *n_out = k;
+  return EQ_OK;
+}
+
+extern "C" eq_status eq_quantize_excluding_host(const float *w, uint32_t rows, uint32_t cols,
+                                                uint32_t symfmt, float int8_div,
+                                                const uint64_t *idx, uint64_t n_idx, uint8_t *sym,
+                                                uint16_t *scales, uint32_t threads) {
+  if (n_idx && !idx) return EQ_ERR_ARG;
+  for (uint64_t i = 0; i < n_idx; ++i)
+    if (idx[i] >= uint64_t(rows) * cols || (i && idx[i] <= idx[i - 1])) return EQ_ERR_ARG;
+  if (n_idx == 0) return eq_quantize_host(w, rows, cols, symfmt, int8_div, sym, scales, threads);
+  if ((!w || !sym || !scales) && uint64_t(rows) * cols) return EQ_ERR_ARG;
+  if (symfmt != EQ_SYM_E4M3 && symfmt != EQ_SYM_INT8) return EQ_ERR_ARG;
+  if (symfmt == EQ_SYM_INT8 && !(int8_div > 0.0f)) return EQ_ERR_ARG;
+  const uint64_t *end = idx + n_idx;
+  std::atomic<int> bad{0};
+  parallel_for(rows, threads, [&](uint64_t r) {
+    // this row's excluded entries, zeroed in a copy of the row, then the ordinary quantiser
+    const uint64_t *lo = std::lower_bound(idx, end, r * cols);
+    const uint64_t *hi = std::lower_bound(lo, end, (r + 1) * cols);
+    std::vector<float> row(w + r * cols, w + (r + 1) * cols);
+    for (const uint64_t *p = lo; p < hi; ++p) row[*p - r * cols] = 0.0f;
+    if (eq_quantize_host(row.data(), 1, cols, symfmt, int8_div, sym + r * cols, scales + r, 1) !=
+        EQ_OK)
+      bad = 1;
+  });
+  return bad ? EQ_ERR_ARG : EQ_OK;
+}
+
 extern "C" eq_status eq_rans_normalize_host(const uint64_t *counts, uint32_t prob_bits,
                                             uint32_t *freqs) {
   if (!counts || !freqs || prob_bits < 8 || prob_bits > 15) return EQ_ERR_ARG;

@@ -196,6 +196,18 @@ __device__ __forceinline__ uint32_t rans_step(uint32_t &x, bool act, const uint3
   return e;
 }
 
+// first position of the sorted super-weight list idx[0, n) holding a value >= key
+__device__ __forceinline__ uint64_t patch_lower_bound(const uint64_t *idx, uint64_t n,
+                                                      uint64_t key) {
+  uint64_t lo = 0, hi = n;
+  while (lo < hi) {
+    const uint64_t mid = (lo + hi) >> 1;
+    if (__ldg(idx + mid) < key) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
 // symbols of two PB-bit slot-table entries as one 16-bit pair (first in the low byte)
 template <uint32_t PB = 12>
 __device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {

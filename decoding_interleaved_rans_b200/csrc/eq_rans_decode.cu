@@ -32,6 +32,9 @@ struct RansDesc {
   const uint16_t *scales;
   const uint32_t *table;  // RansTableHeader followed by the slot table
   uint16_t *out;
+  const uint64_t *patch_idx;  // super weights: sorted flat indices and bf16 values
+  const uint16_t *patch_val;
+  uint64_t n_patch;
   uint64_t numel;
   uint64_t units;         // num_chunks * groups: one warp each
   uint64_t row_magic;     // floor(j / cols) = __umul64hi(j, row_magic) (0: cols == 1)
@@ -48,6 +51,7 @@ struct RansDecodeParams {
   uint32_t warps;  // warps (= groups decoded) per CTA
   RansDesc d[kMaxDecodeTensors];
 };
+static_assert(sizeof(RansDecodeParams) <= 32764, "kernel parameters above the launch limit");
 
 // ------------------------------------------------------------------------------------------------
 // one round (G steps) of one group; FULL: every lane holds a run this round.  A 12-bit stream
@@ -70,6 +74,26 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
     if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
     else *out = dequant1<FMT>((e[0] >> kSymShift<PB>) & 0xFFu, sc);
   }
+}
+
+// Write the chunk's super weights that fall in this warp's group back over the decoded values
+// (after a warp barrier, so the lanes' own stores are ordered before).  A listed position must
+// have decoded to zero, and the list must increase; otherwise EQ_DEV_CORRUPT_STATE.
+template <int G>
+__device__ __forceinline__ uint32_t apply_patches(const RansDesc &D, uint64_t j0, uint32_t n,
+                                                  uint32_t g, uint32_t S, uint32_t lane) {
+  const uint64_t lo = patch_lower_bound(D.patch_idx, D.n_patch, j0);
+  const uint64_t hi = patch_lower_bound(D.patch_idx, D.n_patch, j0 + n);
+  uint32_t bad = 0;
+  __syncwarp();
+  for (uint64_t i = lo + lane; i < hi; i += 32) {
+    const uint64_t j = __ldg(D.patch_idx + i);
+    if (i + 1 < D.n_patch && __ldg(D.patch_idx + i + 1) <= j) bad = EQ_DEV_CORRUPT_STATE;
+    if (((uint32_t(j - j0) / G) % S) / 32 != g) continue;  // another group's run
+    if (D.out[j] & 0x7FFFu) bad = EQ_DEV_CORRUPT_STATE;
+    D.out[j] = __ldg(D.patch_val + i);
+  }
+  return __reduce_or_sync(0xFFFFFFFFu, bad);  // lane 0 reports the warp's status
 }
 
 template <int G, int FMT, uint32_t PB>
@@ -101,6 +125,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
         D.out[j] = dequant1<FMT>(single_sym, bf16_bits_to_float(D.scales[div_by_magic(j, D.row_magic)]));
       }
     }
+    if (D.n_patch && !status) status |= apply_patches<G>(D, j0, n, g, S, lane);
     return status;
   }
 
@@ -149,6 +174,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   }
   if (!status && !__all_sync(0xFFFFFFFFu, q - R.off0 == 2 * nwords && x == kRansL))
     status |= EQ_DEV_CORRUPT_STATE;
+  if (D.n_patch && !status) status |= apply_patches<G>(D, j0, n, g, S, lane);
   // every copy handed to the engine must land before the ring is reused or the CTA exits
   status |= R.drain();
   return status;
@@ -217,6 +243,9 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   if (t.run == 8 && t.cols % 8) return EQ_ERR_UNSUPPORTED;
   if (t.num_chunks != (numel + t.chunk_symbols - 1) / t.chunk_symbols) return EQ_ERR_ARG;
   if (!t.states || !t.word_off || !t.words || !t.scales || !t.tables) return EQ_ERR_ARG;
+  if (t.n_patch && (!t.patch_idx || !t.patch_val || !aligned(t.patch_idx, 8) ||
+                    t.n_patch > numel))
+    return EQ_ERR_ARG;
   if (!aligned(t.words, 16) || !aligned(t.tables, 16) || !aligned(t.states, 4) ||
       !aligned(t.word_off, 8) || !aligned(t.scales, 2))
     return EQ_ERR_ARG;
@@ -263,6 +292,9 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
       D.scales = t.scales;
       D.table = static_cast<const uint32_t *>(t.tables);
       D.out = d_out[idx[q]];
+      D.patch_idx = t.patch_idx;
+      D.patch_val = t.patch_val;
+      D.n_patch = t.n_patch;
       D.numel = uint64_t(t.rows) * t.cols;
       D.groups = t.streams / 32;
       D.units = t.num_chunks * D.groups;

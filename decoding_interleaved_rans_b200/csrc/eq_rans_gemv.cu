@@ -32,6 +32,9 @@ struct GemvParams {
   const uint16_t *x;
   float *y;
   uint32_t *status;
+  const uint64_t *patch_idx;  // super weights (sorted flat indices, bf16 values)
+  const uint16_t *patch_val;
+  uint64_t n_patch;
   uint64_t numel;
   uint64_t num_chunks;
   uint32_t rows, cols, chunk_symbols, rows_per_chunk, rounds_per_row, batch, warps;
@@ -138,9 +141,21 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
       const uint2 wb = make_uint2(dequant2<FMT>(pr[2], sc, nan_codes), dequant2<FMT>(pr[3], sc, nan_codes));
       fma_run<BMAX>(acc, wa, wb, P.x, P.cols, col, batch);
     }
-    // end of a weight row: reduce across the warp and write y
+    // end of a weight row: add its super weights' products, reduce across the warp, write y
     const bool row_end = (r + 1 == rounds) || (P.rows_per_chunk > 1 && (r + 1) % P.rounds_per_row == 0);
     if (row_end) {
+      if (P.n_patch) {
+        const uint64_t rs = uint64_t(row0 + row_local) * P.cols;
+        const uint64_t lo = patch_lower_bound(P.patch_idx, P.n_patch, rs);
+        const uint64_t hi = patch_lower_bound(P.patch_idx, P.n_patch, rs + P.cols);
+        for (uint64_t i = lo + lane; i < hi; i += 32) {
+          const uint32_t col = uint32_t(__ldg(P.patch_idx + i) - rs);
+          const float v = bf16_bits_to_float(__ldg(P.patch_val + i));
+#pragma unroll
+          for (int b = 0; b < BMAX; ++b)
+            if (b < int(batch)) acc[b] = fmaf(v, bf16_bits_to_float(P.x[size_t(b) * P.cols + col]), acc[b]);
+        }
+      }
 #pragma unroll
       for (int b = 0; b < BMAX; ++b) {
         float v = acc[b];
@@ -320,6 +335,13 @@ __global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __gri
         for (uint32_t w = 0; w < kTcWarps; ++w) v += red[w * 256 + wr * 16 + b];
         const uint64_t ch = uint64_t(blockIdx.x) * kTcWarps + wr;
         const uint64_t row = ch * P.rows_per_chunk + (r / rpr);
+        if (P.n_patch && ch < P.num_chunks && b < P.batch && row < P.rows) {  // super weights
+          const uint64_t rs = row * P.cols;
+          const uint64_t hi = patch_lower_bound(P.patch_idx, P.n_patch, rs + P.cols);
+          for (uint64_t i = patch_lower_bound(P.patch_idx, P.n_patch, rs); i < hi; ++i)
+            v = fmaf(bf16_bits_to_float(__ldg(P.patch_val + i)),
+                     bf16_bits_to_float(P.x[size_t(b) * P.cols + (__ldg(P.patch_idx + i) - rs)]), v);
+        }
         if (ch < P.num_chunks && b < P.batch && row < P.rows) P.y[size_t(b) * P.rows + row] = v;
       }
       ++row_local;
@@ -394,6 +416,9 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   P.x = d_x;
   P.y = d_y;
   P.status = d_status;
+  P.patch_idx = t->patch_idx;
+  P.patch_val = t->patch_val;
+  P.n_patch = t->n_patch;
   P.numel = uint64_t(t->rows) * t->cols;
   P.num_chunks = t->num_chunks;
   P.rows = t->rows;

@@ -34,7 +34,7 @@
 extern "C" {
 #endif
 
-#define EQ_ABI_VERSION 1u
+#define EQ_ABI_VERSION 2u
 
 typedef enum {
   EQ_OK = 0,
@@ -77,6 +77,11 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
  *   2^16 and every word read.
  *   Dequantisation: out = bf16_rne( value(s) * scale[row] ), value(s) being the E4M3 value of the
  *   byte (NaN codes 0x7F/0xFF give the bf16 quiet NaN 0x7FC0 / 0xFFC0) or the byte read as int8.
+ *   Super weights ("Float8@2bits" summary, "Manejo de Pesos Superiores": extreme outliers of Int8
+ *   weights kept out of the entropy coding): an optional sorted list of (flat index, bf16 value)
+ *   written over the decoded weight.  The coded symbol at a listed position must dequantise to
+ *   zero (the quantiser codes it as 0); eq_decode reports EQ_DEV_CORRUPT_STATE otherwise, and
+ *   eq_decode_gemv adds value * x for each listed weight.
  */
 typedef struct {
   uint32_t version;       /* EQ_ABI_VERSION                                                    */
@@ -95,6 +100,9 @@ typedef struct {
   const uint16_t *scales; /* [rows] bf16 per-output-channel scales                              */
   const void *tables;     /* eq_table_bytes(EQ_TABLE_RANS) bytes from eq_build_tables(RANS);
                              16-byte aligned                                                    */
+  uint64_t n_patch;       /* super weights in the list (0: none)                               */
+  const uint64_t *patch_idx; /* [n_patch] flat row-major indices, strictly increasing           */
+  const uint16_t *patch_val; /* [n_patch] their bf16 values                                     */
 } eq_rans_tensor;
 
 /*

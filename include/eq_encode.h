@@ -32,6 +32,24 @@ eq_status eq_quantize_host(const float *w, uint32_t rows, uint32_t cols, uint32_
                            float int8_div, uint8_t *sym, uint16_t *scales, uint32_t threads);
 
 /*
+ * Super weights ("Float8@2bits" summary, "Manejo de Pesos Superiores"): the weights with
+ * |w| > tau * rms(w) (rms over the whole tensor).  Writes up to max_out flat indices (increasing)
+ * and their bf16 values; *n_out = how many there are.  Call with max_out = 0 to count.
+ */
+eq_status eq_super_weights_host(const float *w, uint32_t rows, uint32_t cols, double tau,
+                                uint64_t max_out, uint64_t *idx, uint16_t *val, uint64_t *n_out);
+
+/*
+ * eq_quantize_host with the listed positions (flat indices, strictly increasing) left out of
+ * their rows' AbsMax scales; they are coded as symbol 0 (value zero), so the eq_rans_tensor
+ * patch list can carry them exactly.
+ */
+eq_status eq_quantize_excluding_host(const float *w, uint32_t rows, uint32_t cols,
+                                     uint32_t symfmt, float int8_div, const uint64_t *idx,
+                                     uint64_t n_idx, uint8_t *sym, uint16_t *scales,
+                                     uint32_t threads);
+
+/*
  * Frequency table for rANS, summing to 2^prob_bits: f = 0 for absent symbols, else
  * max(1, floor(count * 2^prob_bits / n)); the remainder goes to the most frequent symbol (lowest
  * byte on ties); an excess is taken back one unit at a time from the largest f > 1 (lowest byte

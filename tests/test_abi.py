@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(eq):
 
 def test_version_and_strings(eq):
     L = eq.lib()
-    assert L.eq_abi_version() == 1
+    assert L.eq_abi_version() == 2
     for code in range(5):
         assert L.eq_status_string(code)
     assert eq.table_bytes(1) >= 4096 * 4 and eq.table_bytes(2) > 0 and eq.table_bytes(7) == 0
@@ -60,24 +60,30 @@ def test_build_tables_rejects_bad_input_on_host(eq):
 
 def test_decode_rejects_bad_descriptors_on_host(eq):
     L = eq.lib()
-    d = eq._lib.RansTensorDesc(1, 1, 4, 64, 12, 256, 32, 8, 1, 1 << 20, 1 << 20, 1 << 20,
-                               1 << 20, 1 << 20)
+    d = eq._lib.RansTensorDesc(eq._lib.EQ_ABI_VERSION, 1, 4, 64, 12, 256, 32, 8, 1, 1 << 20,
+                               1 << 20, 1 << 20, 1 << 20, 1 << 20)
     out = (C.c_void_p * 1)(1 << 20)
     st = C.c_void_p(1 << 20)
     for field, val, code in [("version", 0, 1), ("symfmt", 3, 1), ("streams", 40, 3),
                              ("run", 2, 3), ("prob_bits", 10, 3), ("num_chunks", 2, 1),
-                             ("chunk_symbols", 100, 1), ("words", (1 << 20) + 2, 1)]:
+                             ("chunk_symbols", 100, 1), ("words", (1 << 20) + 2, 1),
+                             ("n_patch", 3, 1), ("n_patch", 1 << 40, 1), ("prob_bits", 8, 0)]:
         bad = eq._lib.RansTensorDesc.from_buffer_copy(d)
         setattr(bad, field, val)
+        if code == 0:
+            continue  # valid on the host; would launch
         assert L.eq_decode(C.byref(bad), 1, out, st, None) == code, field
+    bad = eq._lib.RansTensorDesc.from_buffer_copy(d)
+    bad.n_patch, bad.patch_idx, bad.patch_val = 2, (1 << 20) + 4, 1 << 20  # misaligned list
+    assert L.eq_decode(C.byref(bad), 1, out, st, None) == 1
     assert L.eq_decode(C.byref(d), 1, out, None, None) == 1
     assert L.eq_decode(None, 0, None, None, None) == 0
 
 
 def test_gemv_and_huff_reject_bad_input_on_host(eq):
     L = eq.lib()
-    d = eq._lib.RansTensorDesc(1, 1, 4, 64, 12, 100, 32, 8, 3, 1 << 20, 1 << 20, 1 << 20,
-                               1 << 20, 1 << 20)  # chunks do not hold whole rows
+    d = eq._lib.RansTensorDesc(eq._lib.EQ_ABI_VERSION, 1, 4, 64, 12, 100, 32, 8, 3, 1 << 20,
+                               1 << 20, 1 << 20, 1 << 20, 1 << 20)  # chunks do not hold whole rows
     assert L.eq_decode_gemv(C.byref(d), C.c_void_p(1 << 20), 1, C.c_void_p(1 << 20),
                             C.c_void_p(1 << 20), None) in (1, 3)
     h = eq._lib.HuffTensorDesc(10, 30, 8, 256, 1 << 20, 1 << 20, 1 << 20, 1 << 20, 1 << 20)

@@ -117,3 +117,17 @@ def test_normalize_from_counts_matches_oracle(eq, orc):
         f = np.zeros(256, np.uint32)
         assert orc.lib().orc_rans_normalize(counts.ctypes.data, 12, f.ctypes.data) == 0
         assert np.array_equal(eq.normalize_freqs(counts), f)
+
+
+def test_super_weights_and_excluding_quantiser_match_oracle(eq, orc):
+    w = synth.laplace_clipped(300, 1024, 0.01, 0.06, 8)
+    synth.plant_super_weights(w, 9, 8)
+    ia, va = eq.codec.super_weights(w)
+    ib, vb = orc.super_weights(w)
+    assert ia.size == 9 and np.array_equal(ia, ib) and np.array_equal(va, vb)
+    for fmt in (1, 2):
+        a = eq.codec.quantize_excluding(w, fmt, synth.INT8_DIV_LAPLACE_8K, ia)
+        b = orc.quantize_excluding(w, fmt, synth.INT8_DIV_LAPLACE_8K, ib)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    with pytest.raises(eq.EqError):  # the list must increase
+        eq.codec.quantize_excluding(w, 2, 4.0, ia[::-1].copy())

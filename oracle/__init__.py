@@ -73,6 +73,11 @@ def lib() -> C.CDLL:
                                            i64, i64, p]),
             "orc_gemv_f64": (None, [p, p, i64, i64, i64, p]),
             "orc_huff_lengths": (i32, [p, i32, p]),
+            "orc_intq_quantize": (i32, [p, i64, i32, i32, p, p, p]),
+            "orc_intq_dequant": (None, [p, i64, C.c_uint16, C.c_int32, p]),
+            "orc_huff_total_bits_sym": (u64, [p, i64, p]),
+            "orc_huff_encode_sym": (i32, [p, i64, p, p, u32, p, p, p, u64]),
+            "orc_huff_decode_sym": (i32, [p, u64, i64, p, p]),
             "orc_huff_canonical": (None, [p, p]),
             "orc_huff_total_bits": (u64, [p, i64, p]),
             "orc_huff_encode": (i32, [p, i64, p, p, u32, p, p, p, p, u64]),
@@ -506,6 +511,100 @@ def huff_decode_bf16(h: HuffTensor):
     sm = h.sign_mant if h.n else np.zeros(1, np.uint8)
     rc = lib().orc_huff_decode(_p(h.enc_exp), h.total_bits, _p(sm), h.n, _p(h.lengths), _p(out))
     return rc, out[:h.n]
+
+
+# ----------------------------------------------------------------------------------------------
+# EntroLLM-style integer weights, Huffman-coded in the DFloat11 layout
+# ----------------------------------------------------------------------------------------------
+
+INTQ_ASYM, INTQ_UNSIGNED = 0, 1
+
+
+def intq_quantize(w: np.ndarray, bits: int, scheme: int):
+    """Per-tensor b-bit codes: returns (codes uint8, same shape as w), bf16 scale bits, zero)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    sym = np.empty(w.shape, np.uint8)
+    sc, z = C.c_uint16(), C.c_int32()
+    rc = lib().orc_intq_quantize(_p(w), w.size, bits, scheme, _p(sym), C.byref(sc), C.byref(z))
+    if rc:
+        raise ValueError(ERRORS.get(rc, rc))
+    return sym, int(sc.value), int(z.value)
+
+
+def intq_dequant(sym: np.ndarray, scale: int, zero: int) -> np.ndarray:
+    """bf16( (q - z) * s ), one rounding.  Returns uint16 of sym's shape."""
+    sym = np.ascontiguousarray(sym, dtype=np.uint8)
+    out = np.empty(sym.shape, np.uint16)
+    lib().orc_intq_dequant(_p(sym), sym.size, int(scale), int(zero), _p(out))
+    return out
+
+
+def entrollm_quantize(w: np.ndarray, bits: int):
+    """EntroLLM's per-tensor choice between unsigned and asymmetric quantisation: the scheme
+    whose codes have the lower entropy (ties: asymmetric).  Returns (codes, scale, zero, scheme)."""
+    best = None
+    for scheme in (INTQ_ASYM, INTQ_UNSIGNED):
+        sym, sc, z = intq_quantize(w, bits, scheme)
+        h = entropy_bits(sym)
+        if best is None or h < best[0]:
+            best = (h, sym, sc, z, scheme)
+    return best[1], best[2], best[3], best[4]
+
+
+@dataclass
+class HuffSymTensor:
+    """Huffman-coded integer weights (format of the library's eq_huff_int_tensor)."""
+    n: int
+    bits: int
+    threads_per_block: int
+    total_bits: int
+    lengths: np.ndarray    # uint8[256] code length of each code byte (0 = unused)
+    enc: np.ndarray        # uint8[threads * 8 + 16]  the coded stream, MSB-first, zero padded
+    gaps: np.ndarray       # uint8[ceil(5 threads / 8) + 8]
+    block_out: np.ndarray  # uint64[blocks + 1]
+    scale: int             # bf16 bits
+    zero: int
+
+    @property
+    def threads(self) -> int:
+        return (self.total_bits + 63) // 64
+
+    @property
+    def compressed_bytes(self) -> int:
+        return self.threads * 8 + (5 * self.threads + 7) // 8 + self.block_out.nbytes + 256 + 8
+
+
+def huff_encode_sym(sym: np.ndarray, bits: int, scale: int, zero: int,
+                    threads_per_block: int = 256, max_len: int = 32) -> HuffSymTensor:
+    s = np.ascontiguousarray(sym, dtype=np.uint8).ravel()
+    n = s.size
+    lengths = huff_lengths(np.bincount(s, minlength=256).astype(np.uint64), max_len)
+    codes = huff_canonical(lengths)
+    total_bits = int(lib().orc_huff_total_bits_sym(_p(s) if n else None, n, _p(lengths)))
+    threads = (total_bits + 63) // 64
+    blocks = (threads + threads_per_block - 1) // threads_per_block
+    enc = np.zeros(threads * 8 + 16, dtype=np.uint8)
+    gaps = np.zeros((5 * threads + 7) // 8 + 8, dtype=np.uint8)
+    block_out = np.zeros(blocks + 1, dtype=np.uint64)
+    rc = lib().orc_huff_encode_sym(_p(s) if n else None, n, _p(lengths), _p(codes),
+                                   threads_per_block, _p(enc), _p(gaps), _p(block_out), threads)
+    if rc:
+        raise ValueError(ERRORS.get(rc, rc))
+    return HuffSymTensor(n, bits, threads_per_block, total_bits, lengths, enc, gaps, block_out,
+                         int(scale), int(zero))
+
+
+def huff_decode_sym(h: HuffSymTensor):
+    """Sequential canonical decode.  Returns (status, codes uint8[n])."""
+    out = np.zeros(max(1, h.n), dtype=np.uint8)
+    rc = lib().orc_huff_decode_sym(_p(h.enc), h.total_bits, h.n, _p(h.lengths), _p(out))
+    return rc, out[:h.n]
+
+
+def entrollm_decode_bf16(h: HuffSymTensor):
+    """Decode and dequantise: (status, bf16 bits uint16[n])."""
+    rc, sym = huff_decode_sym(h)
+    return rc, intq_dequant(sym, h.scale, h.zero)
 
 
 def gaps_unpack(gaps: np.ndarray, threads: int) -> np.ndarray:

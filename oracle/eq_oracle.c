@@ -473,6 +473,135 @@ int orc_rans_decode_bf16(const uint16_t *words, const uint64_t *word_off, const 
 }
 
 /* ============================================================================================
+ * EntroLLM-style integer weights (EntroLLM page, "Metodologia": per-tensor unsigned or
+ * asymmetric integer quantisation, the codes Huffman-coded and decoded in parallel).
+ * Reading: b-bit codes (b = 8 or 4, L = 2^b levels), one bf16 scale s and one integer zero point z
+ * per tensor, value = (q - z) * s rounded once to bf16.
+ *   scheme 0, asymmetric: s = bf16((max - min) / (L - 1)), z = clamp(rne(-min / s), 0, L - 1);
+ *   scheme 1, unsigned:   s = bf16(max|w| / (L/2 - 1)), z = L/2 (the symmetric grid, offset);
+ *   q = clamp(rne(w / s) + z, 0, L - 1), divisions in binary32.  s = 0 becomes 1.
+ * The codes are Huffman-coded in the DFloat11 layout (MSB-first stream, thread t owns bits
+ * [64t, 64t + 64), 5-bit Gaps, one output position per block of threads), with the code bytes
+ * in place of the exponents and no sign/mantissa stream.
+ * ========================================================================================== */
+
+int orc_intq_quantize(const float *w, int64_t n, int bits, int scheme, uint8_t *sym,
+                      uint16_t *scale_out, int32_t *zero_out) {
+  if ((bits != 8 && bits != 4) || (scheme != 0 && scheme != 1) || n < 0) return ORC_ERR_ARG;
+  const int L = 1 << bits;
+  float lo = 0.0f, hi = 0.0f, amax = 0.0f;
+  for (int64_t i = 0; i < n; ++i) {
+    if (i == 0 || w[i] < lo) lo = w[i];
+    if (i == 0 || w[i] > hi) hi = w[i];
+    if (fabsf(w[i]) > amax) amax = fabsf(w[i]);
+  }
+  uint16_t sb;
+  int32_t z;
+  if (scheme == 0) {
+    sb = orc_f32_to_bf16((hi - lo) / (float)(L - 1));
+    if (orc_bf16_to_f32(sb) == 0.0f) sb = 0x3F80u;
+    float zf = nearbyintf(-lo / orc_bf16_to_f32(sb));
+    if (zf < 0.0f) zf = 0.0f;
+    if (zf > (float)(L - 1)) zf = (float)(L - 1);
+    z = (int32_t)zf;
+  } else {
+    sb = orc_f32_to_bf16(amax / (float)(L / 2 - 1));
+    if (orc_bf16_to_f32(sb) == 0.0f) sb = 0x3F80u;
+    z = L / 2;
+  }
+  const float s = orc_bf16_to_f32(sb);
+  for (int64_t i = 0; i < n; ++i) {
+    float q = nearbyintf(w[i] / s) + (float)z;
+    if (q < 0.0f) q = 0.0f;
+    if (q > (float)(L - 1)) q = (float)(L - 1);
+    sym[i] = (uint8_t)q;
+  }
+  *scale_out = sb;
+  *zero_out = z;
+  return ORC_OK;
+}
+
+/* bf16( (q - z) * s ): |q - z| < 512 and s has 8 significant bits, so the binary64 product is
+ * exact and rounding it is the only rounding. */
+void orc_intq_dequant(const uint8_t *sym, int64_t n, uint16_t scale, int32_t zero, uint16_t *out) {
+  const double s = (double)orc_bf16_to_f32(scale);
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_f64_to_bf16((double)((int32_t)sym[i] - zero) * s);
+}
+
+uint64_t orc_huff_total_bits_sym(const uint8_t *sym, int64_t n, const uint8_t *len) {
+  uint64_t bits = 0;
+  for (int64_t i = 0; i < n; ++i) bits += len[sym[i]];
+  return bits;
+}
+
+/* The DFloat11 layout for byte symbols; buffers as for orc_huff_encode. */
+int orc_huff_encode_sym(const uint8_t *sym, int64_t n, const uint8_t *len, const uint32_t *codes,
+                        uint32_t threads_per_block, uint8_t *enc, uint8_t *gaps,
+                        uint64_t *block_out, uint64_t threads) {
+  uint64_t pos = 0, next_thread = 0, next_block = 0;
+  for (int64_t i = 0; i <= n; ++i) {
+    /* every thread whose segment starts at or before this code's start takes its Gap from it;
+     * after the last code (i == n) the remaining threads point at the end of the stream */
+    while (next_thread < threads && (i == n || 64 * next_thread <= pos)) {
+      if (pos < 64 * next_thread || pos - 64 * next_thread > 31) return ORC_ERR_ARG;
+      uint64_t g = pos - 64 * next_thread, bit = 5 * next_thread;
+      for (int k = 0; k < 5; ++k)
+        if ((g >> k) & 1) gaps[(bit + k) >> 3] |= (uint8_t)(1u << ((bit + k) & 7));
+      if (next_thread % threads_per_block == 0) block_out[next_block++] = (uint64_t)i;
+      ++next_thread;
+    }
+    if (i == n) break;
+    int l = len[sym[i]];
+    if (l == 0) return ORC_ERR_SYMBOL;
+    for (int k = l - 1; k >= 0; --k) {
+      if ((codes[sym[i]] >> k) & 1) enc[pos >> 3] |= (uint8_t)(0x80u >> (pos & 7));
+      ++pos;
+    }
+  }
+  block_out[next_block] = (uint64_t)n;
+  return ORC_OK;
+}
+
+/* Sequential canonical decode of n byte symbols, one bit at a time. */
+int orc_huff_decode_sym(const uint8_t *enc, uint64_t total_bits, int64_t n, const uint8_t *len,
+                        uint8_t *out) {
+  uint32_t count[33] = {0};
+  uint8_t sorted[256];
+  int ns = 0;
+  for (int l = 1; l <= 32; ++l)
+    for (int s = 0; s < 256; ++s)
+      if (len[s] == l) {
+        sorted[ns++] = (uint8_t)s;
+        count[l]++;
+      }
+  uint64_t first[33], index[33], code = 0;
+  int idx = 0;
+  for (int l = 1; l <= 32; ++l) {
+    first[l] = code;
+    index[l] = (uint64_t)idx;
+    code = (code + count[l]) << 1;
+    idx += (int)count[l];
+  }
+  uint64_t pos = 0;
+  for (int64_t i = 0; i < n; ++i) {
+    uint64_t c = 0;
+    int found = -1;
+    for (int l = 1; l <= 32; ++l) {
+      if (pos >= total_bits) return ORC_ERR_OVERRUN;
+      c = (c << 1) | ((enc[pos >> 3] >> (7 - (pos & 7))) & 1u);
+      ++pos;
+      if (count[l] && c >= first[l] && c - first[l] < count[l]) {
+        found = sorted[index[l] + (c - first[l])];
+        break;
+      }
+    }
+    if (found < 0) return ORC_ERR_CODE;
+    out[i] = (uint8_t)found;
+  }
+  return pos == total_bits ? ORC_OK : ORC_ERR_CORRUPT;
+}
+
+/* ============================================================================================
  * GEMV in binary64 over bf16 operands: y[b][r] = sum_c W[r][c] * x[b][c], summed in column order.
  * ========================================================================================== */
 

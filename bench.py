@@ -336,6 +336,27 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                 "bits_per_param": 8 * dh.compressed_bytes / dh.n,
                 "kernel": "huff_decode_kernel"})
     del dh, ob
+    # EntroLLM-style integer weights: a phi3-mini-shaped MLP weight (8192 x 3072, N(0, 0.02)),
+    # uint8 and uint4 codes Huffman-coded, decoded by the two-stage kernel
+    w = synth.normal(8192, 3072, 0.02, 6)
+    for bits in (8, 4):
+        hi_ = eq.codec.entrollm_encode(w, bits)
+        di = eq.DeviceHuffInt.upload(hi_, dev)
+        oi = torch.empty(di.n, dtype=torch.bfloat16, device=dev)
+        st = eq.new_status(dev)
+        ti = time_steps(lambda: eq.huff_int_decode(di, oi, st, stream), steps, 3, flush, stream)
+        assert int(st.item()) == 0
+        sec = statistics.mean(ti)
+        alg = di.compressed_bytes + 2 * di.n
+        out.append({"what": f"EntroLLM-style uint{bits} codes, Huffman-coded, 8192x3072 N(0,0.02)",
+                    "params": di.n, "ms": sec * 1e3, "params_per_s": di.n / sec,
+                    "gbs": alg / sec / 1e9, "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"],
+                    "bits_per_param": 8 * di.compressed_bytes / di.n,
+                    "pages_context": "EntroLLM: 5.58 bits/param from uint8 on phi3-mini (real "
+                                     "weights, Jetson)",
+                    "kernel": "huff_decode_kernel<integer codes>"})
+        del di, oi, hi_
+    del w
     # super weights: the Int8 workload with 6 planted outliers (50-200x the typical weight), kept
     # exactly in the patch list and out of their rows' scales; the decode writes them back
     wl = synth.WORKLOADS["int8_8k"]

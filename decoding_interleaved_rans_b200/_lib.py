@@ -20,12 +20,13 @@ EQ_ABI_VERSION = 2
 
 # every exported function of include/eq.h and include/eq_encode.h
 EXPORTS = ("eq_table_bytes", "eq_build_tables", "eq_decode", "eq_decode_gemv",
-           "eq_huff_bf16_decode", "eq_mlp_scratch_bytes", "eq_mlp_decode", "eq_mlp_decode_noalloc",
+           "eq_huff_bf16_decode", "eq_huff_int_decode", "eq_mlp_scratch_bytes", "eq_mlp_decode", "eq_mlp_decode_noalloc",
            "eq_status_string",
            "eq_abi_version", "eq_quantize_host", "eq_super_weights_host", "eq_quantize_excluding_host",
            "eq_rans_freqs_host", "eq_rans_encode_host", "eq_huff_lengths_host",
            "eq_huff_plan_host", "eq_huff_encode_host", "eq_free_host", "eq_rans_normalize_host",
-           "eq_quantize_device",
+           "eq_quantize_device", "eq_intq_quantize_host", "eq_huff_sym_plan_host",
+           "eq_huff_sym_encode_host",
            "eq_histogram_device", "eq_rans_plan_device", "eq_rans_encode_device")
 
 
@@ -53,6 +54,17 @@ class HuffTensorDesc(C.Structure):
                 ("tables", C.c_void_p)]
 
 
+class HuffIntTensorDesc(C.Structure):
+    """eq_huff_int_tensor"""
+    _fields_ = [("n", C.c_uint64), ("total_bits", C.c_uint64), ("bytes_per_thread", C.c_uint32),
+                ("threads_per_block", C.c_uint32), ("enc", C.c_void_p), ("gaps", C.c_void_p),
+                ("block_out", C.c_void_p), ("tables", C.c_void_p), ("bits", C.c_uint32),
+                ("zero", C.c_int32), ("scale", C.c_uint16), ("reserved16", C.c_uint16),
+                ("reserved32", C.c_uint32)]
+
+
+EQ_INTQ_ASYM, EQ_INTQ_UNSIGNED = 0, 1
+
 _lib = None
 _lock = threading.Lock()
 
@@ -75,6 +87,10 @@ def lib() -> C.CDLL:
                 "eq_decode": (i32, [p, u32, p, p, p]),
                 "eq_decode_gemv": (i32, [p, p, u32, p, p, p]),
                 "eq_huff_bf16_decode": (i32, [p, p, p, p]),
+                "eq_huff_int_decode": (i32, [p, p, p, p]),
+                "eq_intq_quantize_host": (i32, [p, u64, u32, u32, p, p, p]),
+                "eq_huff_sym_plan_host": (i32, [p, u64, p, C.POINTER(C.c_uint64)]),
+                "eq_huff_sym_encode_host": (i32, [p, u64, p, u32, u64, p, p, p]),
                 "eq_mlp_scratch_bytes": (C.c_size_t, [u32, u32]),
                 "eq_mlp_decode": (i32, [p, p, p, p, u32, p, p, C.c_size_t, p, p]),
                 "eq_mlp_decode_noalloc": (i32, [p, p, p, p, u32, p, p, p]),

@@ -163,6 +163,62 @@ class DeviceHuff:
         return t
 
 
+@dataclass
+class DeviceHuffInt:
+    """EntroLLM-style Huffman-coded integer weights resident in device memory
+    (eq_huff_int_tensor)."""
+    n: int
+    total_bits: int
+    threads_per_block: int
+    bits: int
+    zero: int
+    scale: int  # bf16 bits
+    enc: torch.Tensor
+    gaps: torch.Tensor
+    block_out: torch.Tensor
+    tables: torch.Tensor
+
+    @property
+    def threads(self) -> int:
+        return (self.total_bits + 63) // 64
+
+    @property
+    def compressed_bytes(self) -> int:
+        return (8 * self.threads + (5 * self.threads + 7) // 8 + 8 * self.block_out.numel()
+                + 256 + 8)
+
+    def desc(self) -> L.HuffIntTensorDesc:
+        return L.HuffIntTensorDesc(self.n, self.total_bits, 8, self.threads_per_block,
+                                   self.enc.data_ptr(), self.gaps.data_ptr(),
+                                   self.block_out.data_ptr(), self.tables.data_ptr(), self.bits,
+                                   self.zero, self.scale, 0, 0)
+
+    @classmethod
+    def upload(cls, h, device="cuda", stream=None) -> "DeviceHuffInt":
+        """Copy a host container (fields n, total_bits, threads_per_block, bits, zero, scale,
+        lengths, enc, gaps, block_out) to the device and build its tables."""
+        t = cls(int(h.n), int(h.total_bits), int(h.threads_per_block), int(h.bits), int(h.zero),
+                int(h.scale), _dev(np.asarray(h.enc, np.uint8), device, np.uint8),
+                _dev(np.asarray(h.gaps, np.uint8), device, np.uint8),
+                _dev(np.asarray(h.block_out, np.uint64), device, np.int64),
+                torch.empty(table_bytes(L.EQ_TABLE_HUFF), dtype=torch.uint8, device=device))
+        build_tables(L.EQ_TABLE_HUFF, h.lengths, 0, t.tables, stream)
+        return t
+
+
+def huff_int_decode(h: DeviceHuffInt, out=None, status=None, stream=None):
+    """eq_huff_int_decode: Huffman-coded integer codes -> bf16 [n]."""
+    dev = h.enc.device
+    if out is None:
+        out = torch.empty(max(h.n, 1), dtype=torch.bfloat16, device=dev)[:h.n]
+    if status is None:
+        status = new_status(dev)
+    d = h.desc()
+    L.check(L.lib().eq_huff_int_decode(C.byref(d), _ptr(out), _ptr(status), _stream(stream)),
+            "eq_huff_int_decode")
+    return out, status
+
+
 def decode(tensors, outs=None, status=None, stream=None):
     """eq_decode over a list of DeviceRans.  Returns (list of bf16 outputs, status tensor)."""
     tensors = list(tensors)

@@ -148,6 +148,68 @@ def choose_prob_bits(counts, max_loss: float = 0.005) -> int:
     return 8 if rate[8] <= rate[12] * (1 + max_loss) else 12
 
 
+@dataclass
+class HostHuffInt:
+    """EntroLLM-style integer weights, Huffman-coded (eq_huff_int_tensor's arrays)."""
+    n: int
+    bits: int
+    zero: int
+    scale: int  # bf16 bits
+    total_bits: int
+    threads_per_block: int
+    lengths: np.ndarray
+    enc: np.ndarray
+    gaps: np.ndarray
+    block_out: np.ndarray
+
+
+def intq_quantize(w: np.ndarray, bits: int, scheme: int):
+    """Per-tensor integer codes: (codes uint8 of w's shape, bf16 scale bits, zero point)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    sym = np.empty(w.shape, np.uint8)
+    sc, z = C.c_uint16(), C.c_int32()
+    L.check(L.lib().eq_intq_quantize_host(_p(w) if w.size else None, w.size, bits, scheme,
+                                          _p(sym) if w.size else None, C.byref(sc), C.byref(z)),
+            "eq_intq_quantize_host")
+    return sym, int(sc.value), int(z.value)
+
+
+def _entropy(sym: np.ndarray) -> float:
+    c = np.bincount(np.asarray(sym, np.uint8).ravel(), minlength=256).astype(np.float64)
+    p = c[c > 0] / max(1.0, c.sum())
+    return float(-(p * np.log2(p)).sum())
+
+
+def entrollm_encode(w: np.ndarray, bits: int, threads_per_block: int = 256,
+                    max_len: int = 32) -> HostHuffInt:
+    """EntroLLM's mixed per-tensor quantisation (of the unsigned and the asymmetric scheme, the
+    one whose codes have the lower entropy; ties: asymmetric), then the codes Huffman-coded."""
+    best = None
+    for scheme in (L.EQ_INTQ_ASYM, L.EQ_INTQ_UNSIGNED):
+        q = intq_quantize(w, bits, scheme)
+        h = _entropy(q[0])
+        if best is None or h < best[0]:
+            best = (h, q)
+    sym, scale, zero = best[1]
+    s = np.ascontiguousarray(sym, np.uint8).ravel()
+    n = s.size
+    lengths = huff_lengths(np.bincount(s, minlength=256).astype(np.uint64), max_len)
+    tb = C.c_uint64()
+    sp = _p(s) if n else None
+    L.check(L.lib().eq_huff_sym_plan_host(sp, n, _p(lengths), C.byref(tb)), "eq_huff_sym_plan_host")
+    total_bits = tb.value
+    threads = (total_bits + 63) // 64
+    blocks = (threads + threads_per_block - 1) // threads_per_block
+    enc = np.zeros(threads * 8 + 16, np.uint8)
+    gaps = np.zeros((5 * threads + 7) // 8 + 8, np.uint8)
+    block_out = np.zeros(blocks + 1, np.uint64)
+    L.check(L.lib().eq_huff_sym_encode_host(sp, n, _p(lengths), threads_per_block, total_bits,
+                                            _p(enc), _p(gaps), _p(block_out)),
+            "eq_huff_sym_encode_host")
+    return HostHuffInt(n, bits, zero, scale, total_bits, threads_per_block,
+                       lengths.astype(np.uint8), enc, gaps, block_out)
+
+
 def huff_lengths(counts: np.ndarray, max_len: int = 32) -> np.ndarray:
     counts = np.ascontiguousarray(counts, dtype=np.uint64)
     lens = np.zeros(256, np.uint32)

@@ -373,12 +373,14 @@ extern "C" eq_status eq_huff_lengths_host(const uint64_t *counts, uint32_t max_l
   return EQ_OK;
 }
 
-extern "C" eq_status eq_huff_plan_host(const uint16_t *w, uint64_t n, const uint32_t *lengths,
-                                       uint64_t *total_bits) {
-  if ((n && !w) || !lengths || !total_bits) return EQ_ERR_ARG;
+namespace {
+
+// Total code bits of n symbols; EQ_ERR_FORMAT if one has no code.
+template <class SymOf>
+eq_status huff_plan(uint64_t n, SymOf sym_of, const uint32_t *lengths, uint64_t *total_bits) {
   uint64_t bits = 0;
   for (uint64_t i = 0; i < n; ++i) {
-    const uint32_t l = lengths[(w[i] >> 7) & 0xFFu];
+    const uint32_t l = lengths[sym_of(i)];
     if (!l) return EQ_ERR_FORMAT;
     bits += l;
   }
@@ -386,13 +388,13 @@ extern "C" eq_status eq_huff_plan_host(const uint16_t *w, uint64_t n, const uint
   return EQ_OK;
 }
 
-extern "C" eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const uint32_t *lengths,
-                                         uint32_t threads_per_block, uint64_t total_bits,
-                                         uint8_t *enc_exp, uint8_t *sign_mant, uint8_t *gaps,
-                                         uint64_t *block_out) {
-  if ((n && (!w || !sign_mant)) || !lengths || !enc_exp || !gaps || !block_out ||
-      threads_per_block == 0)
-    return EQ_ERR_ARG;
+// The DFloat11 layout for any byte-symbol stream: canonical codes MSB-first into enc, a 5-bit Gap
+// per 64-bit thread segment and the first output index of every block of threads.  side(i) runs
+// once per symbol (DFloat11 stores the sign and mantissa there).
+template <class SymOf, class Side>
+eq_status huff_encode(uint64_t n, SymOf sym_of, Side side, const uint32_t *lengths,
+                      uint32_t threads_per_block, uint64_t total_bits, uint8_t *enc,
+                      uint8_t *gaps, uint64_t *block_out) {
   // canonical codes from the lengths
   uint32_t code[256] = {0};
   {
@@ -418,8 +420,7 @@ extern "C" eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const ui
     gaps[(bit >> 3) + 1] |= uint8_t(v >> 8);
   };
   for (uint64_t i = 0; i < n; ++i) {
-    const uint16_t b = w[i];
-    const uint32_t e = (b >> 7) & 0xFFu, l = lengths[e];
+    const uint32_t e = sym_of(i), l = lengths[e];
     if (!l) return EQ_ERR_FORMAT;
     for (; t < threads && 64 * t <= pos; ++t) {  // threads whose first code starts here
       if (pos - 64 * t > 31) return EQ_ERR_FORMAT;
@@ -429,14 +430,14 @@ extern "C" eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const ui
     acc |= uint64_t(code[e]) << (64 - nacc - l);
     nacc += l;
     while (nacc >= 8) {
-      enc_exp[byte++] = uint8_t(acc >> 56);
+      enc[byte++] = uint8_t(acc >> 56);
       acc <<= 8;
       nacc -= 8;
     }
     pos += l;
-    sign_mant[i] = uint8_t(((b >> 8) & 0x80u) | (b & 0x7Fu));
+    side(i);
   }
-  if (nacc) enc_exp[byte++] = uint8_t(acc >> 56);
+  if (nacc) enc[byte++] = uint8_t(acc >> 56);
   if (pos != total_bits) return EQ_ERR_ARG;
   for (; t < threads; ++t) {
     if (pos < 64 * t || pos - 64 * t > 31) return EQ_ERR_FORMAT;
@@ -444,5 +445,80 @@ extern "C" eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const ui
     if (t % threads_per_block == 0) block_out[blk++] = n;
   }
   block_out[blk] = n;
+  return EQ_OK;
+}
+
+}  // namespace
+
+extern "C" eq_status eq_huff_plan_host(const uint16_t *w, uint64_t n, const uint32_t *lengths,
+                                       uint64_t *total_bits) {
+  if ((n && !w) || !lengths || !total_bits) return EQ_ERR_ARG;
+  return huff_plan(n, [&](uint64_t i) { return (w[i] >> 7) & 0xFFu; }, lengths, total_bits);
+}
+
+extern "C" eq_status eq_huff_encode_host(const uint16_t *w, uint64_t n, const uint32_t *lengths,
+                                         uint32_t threads_per_block, uint64_t total_bits,
+                                         uint8_t *enc_exp, uint8_t *sign_mant, uint8_t *gaps,
+                                         uint64_t *block_out) {
+  if ((n && (!w || !sign_mant)) || !lengths || !enc_exp || !gaps || !block_out ||
+      threads_per_block == 0)
+    return EQ_ERR_ARG;
+  return huff_encode(
+      n, [&](uint64_t i) { return (w[i] >> 7) & 0xFFu; },
+      [&](uint64_t i) { sign_mant[i] = uint8_t(((w[i] >> 8) & 0x80u) | (w[i] & 0x7Fu)); },
+      lengths, threads_per_block, total_bits, enc_exp, gaps, block_out);
+}
+
+extern "C" eq_status eq_huff_sym_plan_host(const uint8_t *sym, uint64_t n,
+                                           const uint32_t *lengths, uint64_t *total_bits) {
+  if ((n && !sym) || !lengths || !total_bits) return EQ_ERR_ARG;
+  return huff_plan(n, [&](uint64_t i) { return uint32_t(sym[i]); }, lengths, total_bits);
+}
+
+extern "C" eq_status eq_huff_sym_encode_host(const uint8_t *sym, uint64_t n,
+                                             const uint32_t *lengths, uint32_t threads_per_block,
+                                             uint64_t total_bits, uint8_t *enc, uint8_t *gaps,
+                                             uint64_t *block_out) {
+  if ((n && !sym) || !lengths || !enc || !gaps || !block_out || threads_per_block == 0)
+    return EQ_ERR_ARG;
+  return huff_encode(
+      n, [&](uint64_t i) { return uint32_t(sym[i]); }, [](uint64_t) {}, lengths,
+      threads_per_block, total_bits, enc, gaps, block_out);
+}
+
+extern "C" eq_status eq_intq_quantize_host(const float *w, uint64_t n, uint32_t bits,
+                                           uint32_t scheme, uint8_t *sym, uint16_t *scale,
+                                           int32_t *zero) {
+  if ((n && (!w || !sym)) || !scale || !zero || (bits != 8 && bits != 4) ||
+      (scheme != EQ_INTQ_ASYM && scheme != EQ_INTQ_UNSIGNED))
+    return EQ_ERR_ARG;
+  const int32_t L = 1 << bits;
+  float lo = 0.0f, hi = 0.0f, amax = 0.0f;
+  for (uint64_t i = 0; i < n; ++i) {
+    if (i == 0 || w[i] < lo) lo = w[i];
+    if (i == 0 || w[i] > hi) hi = w[i];
+    amax = std::max(amax, std::fabs(w[i]));
+  }
+  uint16_t sb;
+  int32_t z;
+  if (scheme == EQ_INTQ_ASYM) {
+    sb = to_bf16((hi - lo) / float(L - 1));
+    if ((sb & 0x7FFFu) == 0) sb = 0x3F80u;
+    const float zf = std::nearbyintf(-lo / bits_f32(uint32_t(sb) << 16));
+    z = int32_t(std::min(float(L - 1), std::max(0.0f, zf)));
+  } else {
+    sb = to_bf16(amax / float(L / 2 - 1));
+    if ((sb & 0x7FFFu) == 0) sb = 0x3F80u;
+    z = L / 2;
+  }
+  const float s = bits_f32(uint32_t(sb) << 16);
+  parallel_for((n + 65535) / 65536, 0, [&](uint64_t b) {
+    for (uint64_t i = b * 65536; i < std::min(n, (b + 1) * 65536); ++i) {
+      const float q = std::nearbyintf(w[i] / s) + float(z);
+      sym[i] = uint8_t(std::min(float(L - 1), std::max(0.0f, q)));
+    }
+  });
+  *scale = sb;
+  *zero = z;
   return EQ_OK;
 }

@@ -18,13 +18,22 @@
 //   * the block scan is a warp-shuffle scan rather than Blelloch's tree.
 #include <algorithm>
 
-#include "eq_internal.cuh"
+#include <cstring>
+
+#include "eq_dequant.cuh"
 
 namespace eq {
 
+// What the decoded byte stream becomes: DFloat11 exponents merged with PackedSignMantissa, or
+// integer codes q turned into bf16((q - zero) * scale).
+constexpr int kHuffDf11 = 0, kHuffInt = 1;
+
 struct HuffParams {
   const uint8_t *enc;
-  const uint8_t *sign_mant;
+  const uint8_t *sign_mant;  // DFloat11 only
+  float scale;               // integer codes only
+  int32_t zero;
+  uint32_t code_limit;       // largest valid integer code
   const uint8_t *gaps;
   const uint64_t *block_out;
   const unsigned char *table;
@@ -124,6 +133,12 @@ __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t 
   return cnt;
 }
 
+// one integer code -> bf16 bits: (q - z) * s is exact in fp32, so the conversion is the rounding
+__device__ __forceinline__ uint32_t int_code_bf16(uint32_t q, float s, int32_t z) {
+  return pack_bf16x2(__int2float_rn(int32_t(q) - z) * s, 0.0f) & 0xFFFFu;
+}
+
+template <int MODE>
 __global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant__ HuffParams P) {
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t T = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -216,36 +231,97 @@ __global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant_
     // ---- merge with PackedSignMantissa and write the block's span ----
     const uint64_t ga = min((o0 + 7) & ~uint64_t(7), o0 + m);
     const uint64_t gb = max(ga, (o0 + m) & ~uint64_t(7));
-    for (uint64_t g = o0 + tid; g < ga; g += T) {  // unaligned head
-      const uint32_t s = P.sign_mant[g], x = ebuf[shift + (g - o0)];
-      P.out[g] = uint16_t(((s & 0x80u) << 8) | (x << 7) | (s & 0x7Fu));
-    }
+    auto one = [&](uint64_t g) {
+      const uint32_t x = ebuf[shift + (g - o0)];
+      if constexpr (MODE == kHuffDf11) {
+        const uint32_t s = P.sign_mant[g];
+        P.out[g] = uint16_t(((s & 0x80u) << 8) | (x << 7) | (s & 0x7Fu));
+      } else {
+        if (x > P.code_limit) err |= EQ_DEV_BAD_CODE;
+        P.out[g] = uint16_t(int_code_bf16(x, P.scale, P.zero));
+      }
+    };
+    for (uint64_t g = o0 + tid; g < ga; g += T) one(g);  // unaligned head
     for (uint64_t g = ga + 8 * uint64_t(tid); g < gb; g += 8 * uint64_t(T)) {
-      const uint2 s = __ldg(reinterpret_cast<const uint2 *>(P.sign_mant + g));
       const uint2 x = *reinterpret_cast<const uint2 *>(ebuf + shift + (g - o0));
       uint32_t w[4];
+      if constexpr (MODE == kHuffDf11) {
+        const uint2 s = __ldg(reinterpret_cast<const uint2 *>(P.sign_mant + g));
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t sw = h ? s.y : s.x, xw = h ? x.y : x.x;
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t sw = h ? s.y : s.x, xw = h ? x.y : x.x;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {  // bytes 2q, 2q+1 -> one bf16 pair
-          const uint32_t s2 = __byte_perm(sw, 0, q ? 0x4342u : 0x4140u);
-          const uint32_t x2 = __byte_perm(xw, 0, q ? 0x4342u : 0x4140u);
-          w[2 * h + q] = ((s2 & 0x00800080u) << 8) | (x2 << 7) | (s2 & 0x007F007Fu);
+          for (int q = 0; q < 2; ++q) {  // bytes 2q, 2q+1 -> one bf16 pair
+            const uint32_t s2 = __byte_perm(sw, 0, q ? 0x4342u : 0x4140u);
+            const uint32_t x2 = __byte_perm(xw, 0, q ? 0x4342u : 0x4140u);
+            w[2 * h + q] = ((s2 & 0x00800080u) << 8) | (x2 << 7) | (s2 & 0x007F007Fu);
+          }
+        }
+      } else {
+        // the limit is 2^bits - 1, so a byte above it has a bit outside the mask
+        if ((x.x | x.y) & ~(0x01010101u * P.code_limit)) err |= EQ_DEV_BAD_CODE;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t xw = k < 2 ? x.x : x.y, sh = 16 * (k & 1);
+          w[k] = pack_bf16x2(__int2float_rn(int32_t((xw >> sh) & 0xFFu) - P.zero) * P.scale,
+                             __int2float_rn(int32_t((xw >> (sh + 8)) & 0xFFu) - P.zero) * P.scale);
         }
       }
       *reinterpret_cast<uint4 *>(P.out + g) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    for (uint64_t g = gb + tid; g < o0 + m; g += T) {  // tail
-      const uint32_t s = P.sign_mant[g], x = ebuf[shift + (g - o0)];
-      P.out[g] = uint16_t(((s & 0x80u) << 8) | (x << 7) | (s & 0x7Fu));
-    }
+    for (uint64_t g = gb + tid; g < o0 + m; g += T) one(g);  // tail
     __syncthreads();  // ebuf and wsum are reused by the next block
   }
   report(P.status, err);
 }
 
-static bool g_huff_attr[64];
+static bool g_huff_attr[64][2];
+
+// validation and launch shared by the DFloat11 and the integer decoders
+template <int MODE>
+static eq_status huff_launch(HuffParams &P, uint64_t n, uint64_t total_bits,
+                             uint32_t bytes_per_thread, uint32_t T, const void *enc,
+                             const void *gaps, const void *block_out, const void *tables,
+                             uint16_t *d_out, uint32_t *d_status, void *stream) {
+  if (!d_status) return EQ_ERR_ARG;
+  if (bytes_per_thread != 8) return EQ_ERR_UNSUPPORTED;
+  if (T < 32 || T > 512 || T % 32) return EQ_ERR_UNSUPPORTED;
+  if (n == 0) return EQ_OK;
+  if (n >= (1ull << 40) || total_bits == 0 || total_bits > 32 * n || total_bits < n)
+    return EQ_ERR_ARG;
+  if (!d_out || !enc || !gaps || !block_out || !tables) return EQ_ERR_ARG;
+  if (!aligned(d_out, 16) || !aligned(enc, 8) || !aligned(tables, 16) || !aligned(block_out, 8))
+    return EQ_ERR_ARG;
+  const uint64_t threads = (total_bits + 63) / 64;
+  const uint64_t blocks = (threads + T - 1) / T;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
+  if (!g_huff_attr[dev][MODE]) {
+    if (cudaFuncSetAttribute(huff_decode_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(huff_smem_bytes(512))) != cudaSuccess)
+      return EQ_ERR_CUDA;
+    g_huff_attr[dev][MODE] = true;
+  }
+  // persistent blocks: as many as fit on the device at once, each walking many blocks
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, huff_decode_kernel<MODE>, int(T),
+                                                    huff_smem_bytes(T)) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  const uint64_t grid = std::min<uint64_t>(blocks, uint64_t(per_sm) * device_sm_count());
+  P.enc = static_cast<const uint8_t *>(enc);
+  P.gaps = static_cast<const uint8_t *>(gaps);
+  P.block_out = static_cast<const uint64_t *>(block_out);
+  P.table = static_cast<const unsigned char *>(tables);
+  P.out = d_out;
+  P.status = d_status;
+  P.n = n;
+  P.total_bits = total_bits;
+  P.threads = threads;
+  P.blocks = blocks;
+  huff_decode_kernel<MODE><<<uint32_t(grid), T, huff_smem_bytes(T), static_cast<cudaStream_t>(stream)>>>(P);
+  return cuda_status(cudaGetLastError());
+}
 
 }  // namespace eq
 
@@ -253,48 +329,26 @@ using namespace eq;
 
 extern "C" eq_status eq_huff_bf16_decode(const eq_huff_tensor *h, uint16_t *d_out,
                                          uint32_t *d_status, void *stream) {
-  if (!h || !d_status) return EQ_ERR_ARG;
-  if (h->bytes_per_thread != 8) return EQ_ERR_UNSUPPORTED;
-  const uint32_t T = h->threads_per_block;
-  if (T < 32 || T > 512 || T % 32) return EQ_ERR_UNSUPPORTED;
-  if (h->n == 0) return EQ_OK;
-  if (h->n >= (1ull << 40) || h->total_bits == 0 || h->total_bits > 32 * h->n ||
-      h->total_bits < h->n)
-    return EQ_ERR_ARG;
-  if (!d_out || !h->enc_exp || !h->sign_mant || !h->gaps || !h->block_out || !h->tables)
-    return EQ_ERR_ARG;
-  if (!aligned(d_out, 16) || !aligned(h->enc_exp, 8) || !aligned(h->sign_mant, 8) ||
-      !aligned(h->tables, 16) || !aligned(h->block_out, 8))
-    return EQ_ERR_ARG;
-  const uint64_t threads = (h->total_bits + 63) / 64;
-  const uint64_t blocks = (threads + T - 1) / T;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  if (!g_huff_attr[dev]) {
-    if (cudaFuncSetAttribute(huff_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(huff_smem_bytes(512))) != cudaSuccess)
-      return EQ_ERR_CUDA;
-    g_huff_attr[dev] = true;
-  }
-  // persistent blocks: as many as fit on the device at once, each walking many blocks
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, huff_decode_kernel, int(T),
-                                                    huff_smem_bytes(T)) != cudaSuccess ||
-      per_sm < 1)
-    per_sm = 1;
-  const uint64_t grid = std::min<uint64_t>(blocks, uint64_t(per_sm) * device_sm_count());
-  HuffParams P;
-  P.enc = h->enc_exp;
+  if (!h) return EQ_ERR_ARG;
+  if (h->n && (!h->sign_mant || !aligned(h->sign_mant, 8))) return EQ_ERR_ARG;
+  HuffParams P{};
   P.sign_mant = h->sign_mant;
-  P.gaps = h->gaps;
-  P.block_out = h->block_out;
-  P.table = static_cast<const unsigned char *>(h->tables);
-  P.out = d_out;
-  P.status = d_status;
-  P.n = h->n;
-  P.total_bits = h->total_bits;
-  P.threads = threads;
-  P.blocks = blocks;
-  huff_decode_kernel<<<uint32_t(grid), T, huff_smem_bytes(T), static_cast<cudaStream_t>(stream)>>>(P);
-  return cuda_status(cudaGetLastError());
+  return huff_launch<kHuffDf11>(P, h->n, h->total_bits, h->bytes_per_thread, h->threads_per_block,
+                                h->enc_exp, h->gaps, h->block_out, h->tables, d_out, d_status,
+                                stream);
+}
+
+extern "C" eq_status eq_huff_int_decode(const eq_huff_int_tensor *h, uint16_t *d_out,
+                                        uint32_t *d_status, void *stream) {
+  if (!h) return EQ_ERR_ARG;
+  if (h->bits != 8 && h->bits != 4) return EQ_ERR_UNSUPPORTED;
+  const int32_t L = 1 << h->bits;
+  if (h->zero < 0 || h->zero > L) return EQ_ERR_ARG;
+  HuffParams P{};
+  const uint32_t sbits = uint32_t(h->scale) << 16;
+  std::memcpy(&P.scale, &sbits, 4);
+  P.zero = h->zero;
+  P.code_limit = uint32_t(L - 1);
+  return huff_launch<kHuffInt>(P, h->n, h->total_bits, h->bytes_per_thread, h->threads_per_block,
+                               h->enc, h->gaps, h->block_out, h->tables, d_out, d_status, stream);
 }

@@ -131,6 +131,30 @@ typedef struct {
   const void *tables;          /* eq_table_bytes(EQ_TABLE_HUFF) bytes from eq_build_tables(HUFF) */
 } eq_huff_tensor;
 
+/*
+ * EntroLLM-style integer weights (EntroLLM page, "Metodologia": per-tensor unsigned or
+ * asymmetric integer quantisation, the codes Huffman-coded and decoded in parallel): n codes of
+ * `bits` bits, Huffman-coded in the layout of eq_huff_tensor with the code bytes in place of the
+ * exponents and no sign/mantissa stream.  Code q decodes to bf16_rne((q - zero) * scale); the
+ * product is exact in fp32, so that is the only rounding.
+ */
+typedef struct {
+  uint64_t n;                  /* number of weights                                            */
+  uint64_t total_bits;         /* bits in the coded stream                                     */
+  uint32_t bytes_per_thread;   /* 8                                                             */
+  uint32_t threads_per_block;  /* 32 .. 512, a multiple of 32                                  */
+  const uint8_t *enc;          /* the coded stream, MSB-first, threads * 8 + 16 bytes (zero
+                                  padded), 8-byte aligned                                       */
+  const uint8_t *gaps;         /* 5-bit Gap of each 64-bit thread segment, LSB-first packing   */
+  const uint64_t *block_out;   /* first output index of each block of threads, then n          */
+  const void *tables;          /* eq_build_tables(EQ_TABLE_HUFF) from the codes' lengths        */
+  uint32_t bits;               /* 8 or 4; a decoded code above 2^bits - 1 sets EQ_DEV_BAD_CODE  */
+  int32_t zero;                /* zero point, 0 .. 2^bits                                      */
+  uint16_t scale;              /* bf16 scale                                                   */
+  uint16_t reserved16;
+  uint32_t reserved32;
+} eq_huff_int_tensor;
+
 /* Bytes of device memory eq_build_tables writes for `kind` (0 for an unknown kind). */
 size_t eq_table_bytes(eq_table_kind kind);
 
@@ -189,6 +213,14 @@ eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x, uint32_t 
  */
 eq_status eq_huff_bf16_decode(const eq_huff_tensor *h, uint16_t *d_out, uint32_t *d_status,
                               void *stream);
+
+/*
+ * Decode n EntroLLM-style Huffman-coded integer weights to bf16 with the two-stage kernel of
+ * eq_huff_bf16_decode (same segments, Gaps, block scan and coalesced stores; the merge step
+ * turns each code q into bf16((q - zero) * scale)).  d_out: n bf16 values, 16-byte aligned.
+ */
+eq_status eq_huff_int_decode(const eq_huff_int_tensor *h, uint16_t *d_out, uint32_t *d_status,
+                             void *stream);
 
 /*
  * Beyond the four calls: a LLaMA-style MLP block straight from coded weights,

@@ -73,6 +73,28 @@ eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint32_t cols,
                               uint32_t run, uint32_t threads, uint32_t *states, uint64_t *word_off,
                               uint16_t **words, uint64_t *n_words);
 
+/*
+ * EntroLLM-style per-tensor integer quantisation of n weights to `bits`-bit codes (8 or 4):
+ *   EQ_INTQ_ASYM:     scale = bf16((max - min) / (2^bits - 1)), zero = clamp(rne(-min / scale));
+ *   EQ_INTQ_UNSIGNED: scale = bf16(max|w| / (2^(bits-1) - 1)), zero = 2^(bits-1);
+ *   code = clamp(rne(w / scale) + zero, 0, 2^bits - 1); a zero scale becomes 1.
+ */
+#define EQ_INTQ_ASYM 0u
+#define EQ_INTQ_UNSIGNED 1u
+eq_status eq_intq_quantize_host(const float *w, uint64_t n, uint32_t bits, uint32_t scheme,
+                                uint8_t *sym, uint16_t *scale, int32_t *zero);
+
+/*
+ * The eq_huff_tensor layout for any byte stream (eq_huff_int_tensor's coded codes): plan gives
+ * total_bits; encode fills enc (threads * 8 + 16 bytes), gaps (ceil(5 threads / 8) + 8 bytes)
+ * and block_out (blocks + 1 entries), all zeroed by the caller.
+ */
+eq_status eq_huff_sym_plan_host(const uint8_t *sym, uint64_t n, const uint32_t *lengths,
+                                uint64_t *total_bits);
+eq_status eq_huff_sym_encode_host(const uint8_t *sym, uint64_t n, const uint32_t *lengths,
+                                  uint32_t threads_per_block, uint64_t total_bits, uint8_t *enc,
+                                  uint8_t *gaps, uint64_t *block_out);
+
 /* Optimal Huffman code lengths (no length above max_len) for 256 symbol counts. */
 eq_status eq_huff_lengths_host(const uint64_t *counts, uint32_t max_len, uint32_t *lengths);
 

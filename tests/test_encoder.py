@@ -131,3 +131,23 @@ def test_super_weights_and_excluding_quantiser_match_oracle(eq, orc):
         assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
     with pytest.raises(eq.EqError):  # the list must increase
         eq.codec.quantize_excluding(w, 2, 4.0, ia[::-1].copy())
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_integer_quantiser_and_byte_huffman_match_oracle(eq, orc, bits):
+    rng = np.random.default_rng(bits)
+    for w in (synth.normal(128, 1024, 0.02, 9),
+              np.abs(rng.standard_normal((64, 700))).astype(np.float32) * 0.03,
+              synth.normal_with_outliers(50, 333, 0.02, 0.01, 8.0, 10)):
+        for scheme in (0, 1):
+            a = eq.codec.intq_quantize(w, bits, scheme)
+            b = orc.intq_quantize(w, bits, scheme)
+            assert np.array_equal(a[0], b[0]) and a[1:] == b[1:]
+        for tpb in (256, 32):
+            h = eq.codec.entrollm_encode(w, bits, threads_per_block=tpb)
+            sym, sc, z, _ = orc.entrollm_quantize(w, bits)
+            o = orc.huff_encode_sym(sym, bits, sc, z, threads_per_block=tpb)
+            assert (h.scale, h.zero, h.total_bits) == (o.scale, o.zero, o.total_bits)
+            assert np.array_equal(h.lengths, o.lengths)
+            for f in ("enc", "gaps", "block_out"):
+                assert np.array_equal(getattr(h, f), getattr(o, f)), f

@@ -14,12 +14,10 @@ namespace eq {
 
 // rANS: 16-byte header, then one 32-bit entry per slot of the 2^pb-slot probability space
 // (pb = prob_bits, 12 or 8), f = frequency of the slot's symbol (1 .. 2^pb - 1):
-//   12-bit: bits 31..20 f, bits 19..12 symbol, bits 11..0 slot - cum.  With f in the top bits,
-//     f * floor(x / 4096) is the high word of (e & 0xFFF00000) * (x & 0xFFFFF000).
-//   8-bit: bits 31..24 f, bits 23..16 symbol, bits 15..0 the signed correction
-//     d = (slot - cum) - floor(f * slot / 256).  The high word of (f << 24) * x is
-//     floor(f * x / 256) = f * floor(x / 256) + floor(f * slot / 256), so the decode step
-//     x' = f * floor(x / 256) + slot - cum is hi((e & 0xFF000000) * x) + d with x unmasked.
+//   12-bit: bits 31..20 f, bits 19..12 symbol, bits 11..0 slot - cum;
+//   8-bit:  bits 31..24 f, bits 23..16 symbol, bits 15..8 zero, bits 7..0 slot - cum;
+// so the decode step x' = f * floor(x / 2^pb) + slot - cum is (e >> (32 - pb)) * (x >> pb) +
+// (e & (2^pb - 1)).
 // A table whose single symbol owns every slot cannot store its frequency in pb bits; the header
 // flags it instead and the decoders take a separate path.  8-bit tables use the first 256
 // entries of the same 16 KiB allocation.

@@ -128,42 +128,30 @@ __device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
   return d;
 }
 
-// The decoding half of a step with a PB-bit table (entry layouts in eq_internal.cuh); returns
-// the entry.  Written as one PTX block: slot = x mod 2^PB, its entry from the shared-memory
-// table, then the multiply-high-add (with ptxas left to pick the address arithmetic, the step
-// took about 1.5 more instructions).  Volatile, so it is never hoisted above the barrier that
-// publishes the table.
+// The decoding half of a step with a PB-bit table (entry: f in the top PB bits, the symbol
+// above bit 8 or 12, slot - cum in the low PB bits; eq_internal.cuh); returns the entry.
+// x' = f * (x >> PB) + (slot - cum) as shifts and a low multiply-add: x >> PB is computed while
+// the table load is in flight, so the step's dependency chain is load -> shift -> multiply-add
+// (a multiply-high form, fewer instructions, measured slower: the high product's latency sits
+// on the chain).  One PTX block, so ptxas does not redo the address arithmetic; volatile, so it
+// is never hoisted above the barrier that publishes the table.
 template <bool FULL, uint32_t PB>
 __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, const uint32_t *lut) {
+  static_assert(PB == 12 || PB == 8, "12- or 8-bit tables");
   const uint32_t base = uint32_t(__cvta_generic_to_shared(lut));
   uint32_t e, nx;
-  if constexpr (PB == 8) {
-    asm volatile(
-        "{\n\t.reg .b32 a, f, d;\n\t"
-        "and.b32 a, %2, 255;\n\t"
-        "shl.b32 a, a, 2;\n\t"
-        "add.u32 a, a, %3;\n\t"
-        "ld.shared.u32 %1, [a];\n\t"
-        "and.b32 f, %1, 0xFF000000;\n\t"
-        "prmt.b32 d, %1, 0, 0x9910;\n\t"  // the signed correction, sign-extended
-        "mad.hi.u32 %0, f, %2, d;\n\t}"
-        : "=r"(nx), "=r"(e)
-        : "r"(x), "r"(base));
-  } else {
-    static_assert(PB == 12, "12- or 8-bit tables");
-    asm volatile(
-        "{\n\t.reg .b32 a, f, xm, b;\n\t"
-        "and.b32 a, %2, 4095;\n\t"
-        "shl.b32 a, a, 2;\n\t"
-        "add.u32 a, a, %3;\n\t"
-        "ld.shared.u32 %1, [a];\n\t"
-        "and.b32 f, %1, 0xFFF00000;\n\t"
-        "and.b32 xm, %2, 0xFFFFF000;\n\t"
-        "and.b32 b, %1, 4095;\n\t"
-        "mad.hi.u32 %0, f, xm, b;\n\t}"
-        : "=r"(nx), "=r"(e)
-        : "r"(x), "r"(base));
-  }
+  asm volatile(
+      "{\n\t.reg .b32 a, f, b, xs;\n\t"
+      "and.b32 a, %2, %4;\n\t"
+      "shl.b32 a, a, 2;\n\t"
+      "add.u32 a, a, %3;\n\t"
+      "shr.u32 xs, %2, %5;\n\t"
+      "ld.shared.u32 %1, [a];\n\t"
+      "shr.u32 f, %1, %6;\n\t"
+      "and.b32 b, %1, %4;\n\t"
+      "mad.lo.u32 %0, f, xs, b;\n\t}"
+      : "=r"(nx), "=r"(e)
+      : "r"(x), "r"(base), "n"((1u << PB) - 1), "n"(PB), "n"(32 - PB));
   if (FULL || act) x = nx;
   return e;
 }

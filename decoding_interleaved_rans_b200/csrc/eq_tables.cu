@@ -47,12 +47,7 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
     }
     uint32_t f = a.freq[lo];
     uint32_t fe = (f >= slots) ? 0u : f;  // a one-symbol table is handled by the flag
-    if (pb == 8) {
-      const int32_t d = int32_t(slot - cum[lo]) - int32_t((fe * slot) >> 8);
-      lut[slot] = (fe << 24) | (uint32_t(lo) << 16) | (uint32_t(d) & 0xFFFFu);
-    } else {
-      lut[slot] = (fe << (32 - pb)) | (uint32_t(lo) << pb) | (slot - cum[lo]);
-    }
+    lut[slot] = (fe << (32 - pb)) | (uint32_t(lo) << (pb == 8 ? 16 : 12)) | (slot - cum[lo]);
   }
 }
 

@@ -3,9 +3,10 @@
 // Format and parallel decomposition follow the DFloat11 page ("Kernels GPU de 2 etapas y
 // metadatos auxiliares"): thread t owns bytes [8t, 8t + 8) of EncodedExponent and decodes the
 // codes that start there, beginning at its 5-bit Gap; one output position is stored per block of
-// threads; stage 1 decodes and only counts, a block-wide prefix sum of the counts gives every
-// thread its output offset, stage 2 decodes again and writes the exponents into a shared-memory
-// buffer; the block then merges them with PackedSignMantissa and writes its span once, coalesced.
+// threads; on the page, stage 1 decodes and only counts, a block-wide prefix sum of the counts
+// gives every thread its output offset, and stage 2 decodes again and writes the exponents into a
+// shared-memory buffer; the block then merges them with PackedSignMantissa and writes its span
+// once, coalesced.
 //
 // Different from the page's kernel, for B200:
 //   * codes are read through an 11-bit window table (16 KiB in shared memory) that returns up to
@@ -15,7 +16,10 @@
 //     to be given up as a pointer;
 //   * blocks are persistent: each CTA loads the window table once and walks over many blocks of
 //     the stream, fetching the next block's bits while it merges the current one;
-//   * the block scan is a warp-shuffle scan rather than Blelloch's tree.
+//   * the block scan is a warp-shuffle scan rather than Blelloch's tree;
+//   * codes are decoded once: stage 1 packs each thread's values into its own column of the
+//     shared buffer, and stage 2 only moves them to their offsets (a second decode cost more
+//     than a third of the kernel).
 #include <algorithm>
 
 #include <cstring>
@@ -71,15 +75,38 @@ __device__ __forceinline__ uint32_t tree_decode(const uint16_t *tree, uint32_t n
   return used + rem;
 }
 
-// Decode the codes starting in bits [gap, end) of this thread's segment.  WRITE == false: count
-// them.  WRITE == true: also store their values at dst[0 .. count).  *bad is set on a pattern no
-// code matches.
-template <bool WRITE>
+// A thread's decoded values, packed as bytes (value i = byte i, little-endian) into its private
+// column of 32-bit words: word i at col[i * T], so the 32 lanes of a warp touch 32 banks.
+struct BytePacker {
+  uint32_t *col;
+  uint32_t T;
+  uint64_t acc = 0;  // pending bytes, the oldest in the low bits
+  uint32_t nb = 0, wp = 0;
+
+  // append the low k (1..4) bytes of v
+  __device__ __forceinline__ void put(uint32_t v, uint32_t k) {
+    if (k < 4) v &= (1u << (8 * k)) - 1u;
+    acc |= uint64_t(v) << (8 * nb);
+    nb += k;
+    if (nb >= 4) {
+      col[wp * T] = uint32_t(acc);
+      ++wp;
+      acc >>= 32;
+      nb -= 4;
+    }
+  }
+  __device__ __forceinline__ void flush() {
+    if (nb) col[wp * T] = uint32_t(acc);
+  }
+};
+
+// Decode the codes starting in bits [gap, end) of this thread's segment into the packer; returns
+// how many.  *bad is set on a pattern no code matches.
 __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t *tree, uint32_t ntab,
                                             uint32_t r0, uint32_t r1, uint32_t r2, uint32_t pos,
-                                            uint32_t end, uint8_t *dst, uint32_t *bad) {
+                                            uint32_t end, BytePacker &out, uint32_t *bad) {
   uint32_t cnt = 0;
-  // body: every code found inside a whole 12-bit window starts before `end`
+  // body: every code found inside a whole 11-bit window starts before `end`
   while (pos + kHuffWindowBits <= end) {
     const uint32_t w = bits32(r0, r1, r2, pos);
     const uint64_t f = win[w >> (32 - kHuffWindowBits)];
@@ -88,9 +115,9 @@ __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t 
       const uint32_t len = tree_decode(tree, ntab, w, &sym);
       if (!len) {
         *bad = EQ_DEV_BAD_CODE;
-        return cnt;
+        break;
       }
-      if (WRITE) dst[cnt] = uint8_t(sym);
+      out.put(sym, 1);
       ++cnt;
       pos += len;
       continue;
@@ -99,20 +126,14 @@ __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t 
     const uint32_t k = (hi >> 20) & 7u;
     if (k == 0) {
       *bad = EQ_DEV_BAD_CODE;
-      return cnt;
+      break;
     }
-    if (WRITE) {
-      const uint32_t lo = uint32_t(f);
-      dst[cnt] = uint8_t(lo);
-      if (k > 1) dst[cnt + 1] = uint8_t(lo >> 8);
-      if (k > 2) dst[cnt + 2] = uint8_t(lo >> 16);
-      if (k > 3) dst[cnt + 3] = uint8_t(lo >> 24);
-    }
+    out.put(uint32_t(f), k);
     cnt += k;
     pos += (hi >> 16) & 0xFu;
   }
   // tail: codes may reach past `end`; only those starting before it are this thread's
-  while (pos < end) {
+  while (pos < end && !*bad) {
     const uint32_t w = bits32(r0, r1, r2, pos);
     const uint64_t f = win[w >> (32 - kHuffWindowBits)];
     uint32_t sym, len;
@@ -124,13 +145,47 @@ __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t 
     }
     if (!len) {
       *bad = EQ_DEV_BAD_CODE;
-      return cnt;
+      break;
     }
-    if (WRITE) dst[cnt] = uint8_t(sym);
+    out.put(sym, 1);
     ++cnt;
     pos += len;
   }
+  out.flush();
   return cnt;
+}
+
+// Move this thread's cnt packed bytes (column layout, at most 64) to ebuf[D .. D + cnt).  All
+// threads first read their columns into registers; the caller's barrier separates that from the
+// writes, since the compacted ranges overlap other threads' columns.
+struct Staged {
+  uint32_t w[17];
+};
+
+__device__ __forceinline__ void stage_read(const uint32_t *col, uint32_t T, uint32_t cnt, Staged &st) {
+  const uint32_t nw = (cnt + 3) >> 2;
+#pragma unroll
+  for (uint32_t i = 0; i < 16; ++i) st.w[i] = i < nw ? col[i * T] : 0u;
+  st.w[16] = 0u;
+}
+
+__device__ __forceinline__ void stage_write(uint8_t *ebuf, uint32_t D, uint32_t cnt, const Staged &st) {
+  const uint32_t a = D & 3u, sh = 8 * a, nd = (a + cnt + 3) >> 2;
+  uint32_t *dst = reinterpret_cast<uint32_t *>(ebuf + (D - a));
+#pragma unroll
+  for (uint32_t j = 0; j < 17; ++j) {
+    if (j < nd) {
+      // destination word j holds source bytes 4j - a .. 4j - a + 3
+      const uint32_t prev = j ? st.w[j - 1] : 0u;
+      const uint32_t v = a ? __funnelshift_l(prev, st.w[j], sh) : st.w[j];
+      const uint32_t b0 = j == 0 ? a : 0u, b1 = min(4u, a + cnt - 4 * j);
+      if (b0 == 0 && b1 == 4) {
+        dst[j] = v;
+      } else {  // a word shared with a neighbouring thread's bytes: only ours
+        for (uint32_t b = b0; b < b1; ++b) ebuf[D - a + 4 * j + b] = uint8_t(v >> (8 * b));
+      }
+    }
+  }
 }
 
 // one integer code -> bf16 bits: (q - z) * s is exact in fp32, so the conversion is the rounding
@@ -138,8 +193,10 @@ __device__ __forceinline__ uint32_t int_code_bf16(uint32_t q, float s, int32_t z
   return pack_bf16x2(__int2float_rn(int32_t(q) - z) * s, 0.0f) & 0xFFFFu;
 }
 
+// At most 40 registers (3 CTAs of 512 or 6 of 256 threads per SM): the staging registers would
+// otherwise cost more in occupancy than the single decode pass saves.
 template <int MODE>
-__global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant__ HuffParams P) {
+__global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_constant__ HuffParams P) {
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t T = blockDim.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint64_t *win = reinterpret_cast<uint64_t *>(smem);
@@ -185,9 +242,10 @@ __global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant_
       end = left < 64 ? uint32_t(left) : 64u;
     }
     fetch(b + gridDim.x, n0, n1, n2, ng);  // next block's bits, in flight during this one
-    // ---- stage 1: count ----
+    // ---- stage 1: decode once, the values packed into this thread's column of ebuf ----
     uint32_t bad = 0;
-    const uint32_t cnt = segment<false>(win, tree, ntab, r0, r1, r2, pos, end, nullptr, &bad);
+    BytePacker pk{reinterpret_cast<uint32_t *>(ebuf) + tid, T};
+    const uint32_t cnt = segment(win, tree, ntab, r0, r1, r2, pos, end, pk, &bad);
     // ---- block-wide exclusive scan of the counts ----
     uint32_t incl = cnt;
 #pragma unroll
@@ -222,10 +280,13 @@ __global__ void __launch_bounds__(512) huff_decode_kernel(const __grid_constant_
       m = min(uint64_t(total), o1 - o0);
     }
     err |= bad;
-    // ---- stage 2: decode again, exponents to their block positions (shifted so that 8-aligned
-    //      outputs are 8-aligned in shared memory) ----
+    // ---- stage 2: every thread moves its values to their block positions (shifted so that
+    //      8-aligned outputs are 8-aligned in shared memory) ----
     const uint32_t shift = uint32_t(o0 & 7);
-    if (off + cnt <= m) segment<true>(win, tree, ntab, r0, r1, r2, pos, end, ebuf + shift + off, &bad);
+    Staged stg;
+    stage_read(reinterpret_cast<const uint32_t *>(ebuf) + tid, T, cnt, stg);
+    __syncthreads();
+    if (off + cnt <= m) stage_write(ebuf, shift + off, cnt, stg);
     __syncthreads();
 
     // ---- merge with PackedSignMantissa and write the block's span ----

@@ -21,7 +21,8 @@ def tbl(bits, freq_of):
 
 
 TABLES = [(8, tbl(8, {0: 128, 1: 64, 2: 64})), (8, tbl(8, {5: 1, 9: 254, 77: 1})),
-          (8, tbl(8, {0: 85, 1: 85, 2: 86})), (5, tbl(5, {0: 3, 1: 13, 2: 16})),
+          (8, tbl(8, {0: 85, 1: 85, 2: 86})), (7, tbl(7, {0: 1, 1: 126, 200: 1})),
+          (7, tbl(7, {3: 43, 4: 42, 5: 43})), (5, tbl(5, {0: 3, 1: 13, 2: 16})),
           (4, tbl(4, {0: 1, 1: 5, 2: 10}))]
 
 
@@ -131,3 +132,42 @@ def test_8bit_corruption_is_reported(orc):
     bad = st.copy()
     bad[7] ^= 0x100
     assert orc.rans_decode_chunk(words, bad, sym.size, f, 32, 8, prob_bits=8)[0] != 0
+
+
+def test_uniform_7bit_closed_form(orc):
+    """f_s = 1 for bytes 0..127 (7-bit table): coding s maps x to 128 x + s, so a pair of steps
+    adds exactly 14 bits (2^14 x + 128 s_b + s_a) and a flush removes 16.  The pair's flush
+    bound is 2^(32 - 14) = 2^18: the encoder flushes before a pair iff x has at least 19 bits.
+    So the word count follows from bit lengths alone (start 2^16: 17 bits), and the final state's
+    low 14 bits are 128 s_1 + s_0."""
+    f = np.zeros(256, np.uint32)
+    f[:128] = 1
+    rng = np.random.default_rng(16)
+    for T in range(2, 60, 2):
+        sym = rng.integers(0, 128, T, dtype=np.uint8)
+        st, words, _ = orc.rans_encode_chunk(sym, f, 1, 1, prob_bits=7)
+        bits, flushes = 17, 0
+        for _ in range(T // 2):
+            if bits >= 19:
+                bits -= 16
+                flushes += 1
+            bits += 14
+        assert words.size == flushes, T
+        assert int(st[0]).bit_length() == bits, T
+        assert int(st[0]) & 0x3FFF == 128 * int(sym[1]) + int(sym[0])
+        rc, out = orc.rans_decode_chunk(words, st, T, f, 1, 1, prob_bits=7)
+        assert rc == 0 and np.array_equal(out, sym)
+
+
+def test_int8_workload_7bit_table_near_shannon(orc):
+    wl = synth.WORKLOADS["int8_8k"]
+    w = wl.tensors[0].generate(row_lo=0, row_hi=256)
+    sym, sc = orc.quantize(w, orc.INT8, wl.int8_div)
+    t = orc.rans_encode(sym, sc, orc.INT8, 65536, 128, 8, prob_bits=7)
+    H = orc.entropy_bits(sym)
+    counts = np.bincount(sym.ravel(), minlength=256)
+    ce = orc.cross_entropy_bits(counts, t.freqs, 7)
+    assert ce - H < 0.012  # 7-bit probabilities cost about 0.4% on this alphabet
+    assert t.payload_bytes <= 1.01 * t.numel * ce / 8
+    rc, out = orc.rans_decode_bf16(t, threads=4)
+    assert rc == 0 and np.array_equal(out.reshape(sym.shape), orc.dequant(sym, sc, orc.INT8))

@@ -4,14 +4,14 @@
     torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
 
 A step decodes the whole Int8 8192x8192 Laplace weight (H = 2.0 bits, 64 KiB chunks, 128
-interleaved streams, run 8, 8-bit frequency table: one renormalisation per two steps) from its
-rANS stream in HBM into bf16 in HBM: one eq_decode launch.
+interleaved streams, run 8, 7-bit frequency table: one pair-table lookup and one renormalisation
+per two steps) from its rANS stream in HBM into bf16 in HBM: one eq_decode launch.
 Every rank decodes its own copy (weak scaling; the decode has no exchange step).  Timing: CUDA
 events on the launching stream around each step, the L2 flushed between steps by writing a
 256 MiB buffer, max over ranks.  `e2e` repeats the step through the C ABI with host buffers:
 pinned host -> device copy of the coded arrays, decode, device -> host read of the step's status
 word (the decoded weight stays in HBM for its layer; `e2e_weights_to_host` also copies it back).
-Secondary lines under "also": the same weight with a 12-bit table, the fused decode-GEMV on the
+Secondary lines under "also": the same weight with 8- and 12-bit tables, the fused decode-GEMV on the
 13B MLP (batch 1/4/16), the MLP block, the DFloat11 decode, the GPU compressor and the block
 pipeline, each with its own roofline or comparison.
 """
@@ -275,20 +275,23 @@ def run_ours(args):
 
     also = []
     if not args.no_extra:
-        # the same weight with a 12-bit table (a renormalisation point after every step)
-        _, h12 = prepare_rans(eq, WORKLOAD, prob_bits=12)
-        t12 = eq.DeviceRans.upload(h12, dev)
-        ts12 = time_steps(lambda: eq.decode([t12], [out], status, stream), max(5, args.steps // 2),
-                          3, flush, stream)
-        assert int(status.item()) == 0
-        s12 = statistics.mean(ts12)
-        a12 = (t12.compressed_bytes + 2 * numel) / s12 / 1e9
-        also.append({"what": "same Int8 weight, 12-bit table (renormalisation every step)",
-                     "params": numel, "ms": s12 * 1e3, "params_per_s": numel / s12, "gbs": a12,
-                     "frac_of_peak": a12 / peaks["hbm_gbs"],
-                     "bits_per_param": 8 * t12.compressed_bytes / numel,
-                     "kernel": "rans_decode_kernel<run 8, Int8, 12-bit table>"})
-        del t12, h12
+        # the same weight with 8-bit (one renormalisation per two steps, one lookup per step) and
+        # 12-bit tables (a renormalisation point after every step)
+        for pb, how in ((8, "renormalisation every second step"),
+                        (12, "renormalisation every step")):
+            _, hx = prepare_rans(eq, WORKLOAD, prob_bits=pb)
+            tx = eq.DeviceRans.upload(hx, dev)
+            tsx = time_steps(lambda: eq.decode([tx], [out], status, stream),
+                             max(5, args.steps // 2), 3, flush, stream)
+            assert int(status.item()) == 0
+            sx = statistics.mean(tsx)
+            ax = (tx.compressed_bytes + 2 * numel) / sx / 1e9
+            also.append({"what": f"same Int8 weight, {pb}-bit table ({how})",
+                         "params": numel, "ms": sx * 1e3, "params_per_s": numel / sx, "gbs": ax,
+                         "frac_of_peak": ax / peaks["hbm_gbs"],
+                         "bits_per_param": 8 * tx.compressed_bytes / numel,
+                         "kernel": f"rans_decode_kernel<run 8, Int8, {pb}-bit table>"})
+            del tx, hx
         also += extra_measurements(eq, dev, stream, flush, peaks, args)
     barrier(world)
     if rank != 0:
@@ -300,7 +303,7 @@ def run_ours(args):
         "ms_per_step": mean_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
         "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
-                               "chunks, 128 streams, run 8, 8-bit table -> bf16",
+                               f"chunks, 128 streams, run 8, {wl.prob_bits}-bit table -> bf16",
                    "params_per_gpu": numel, "compressed_bytes": t.compressed_bytes,
                    "bits_per_param": 8 * t.compressed_bytes / numel,
                    "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{world}"},
@@ -309,7 +312,7 @@ def run_ours(args):
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": measured_traffic("rans_decode_kernel", numel),
                      "peak_src": peaks["src"],
-                     "kernel": "rans_decode_kernel<run 8, Int8, 8-bit table>",
+                     "kernel": f"rans_decode_kernel<run 8, Int8, {wl.prob_bits}-bit table>",
                      "alg_bytes_per_launch": alg_bytes},
         "e2e": {"value": numel * world / e2e_s, "unit": "params/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": 4, "ms_per_step": e2e_s * 1e3,
@@ -392,11 +395,13 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
     sec = statistics.mean(tsw)
     alg = ts_.compressed_bytes + 2 * ts_.numel
     out.append({"what": "Int8 8192x8192 with 6 super weights (patch list written back in the "
-                        "decode epilogue), 8-bit table", "params": ts_.numel, "ms": sec * 1e3,
+                        f"decode epilogue), {wl.prob_bits}-bit table", "params": ts_.numel,
+                "ms": sec * 1e3,
                 "params_per_s": ts_.numel / sec, "gbs": alg / sec / 1e9,
                 "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"], "super_weights": int(pidx.size),
                 "zero_symbols_in_their_rows_without_exclusion": collapsed,
-                "kernel": "rans_decode_kernel<run 8, Int8, 8-bit table> + patch epilogue"})
+                "kernel": f"rans_decode_kernel<run 8, Int8, {wl.prob_bits}-bit table> + patch "
+                          "epilogue"})
     del ts_, osw, hs
     # GPU compressor: fp32 weights in HBM -> quantise, histogram, frequency table (host), rANS
     # plan + encode; wall clock around the whole call (it reads the word total back once)
@@ -557,7 +562,7 @@ def run_reference(args):
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
             "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
-                                   "chunks, 128 streams, run 8, 8-bit table -> bf16",
+                                   f"chunks, 128 streams, run 8, {wl.prob_bits}-bit table -> bf16",
                        "sample_chunks": take, "parallelism": "host cores"},
             "cpu_baseline": {"value": v, "unit": "params/s", "cores": cores, "kind": "oracle",
                              "sample": f"{take} of {o.num_chunks} chunks per step"},

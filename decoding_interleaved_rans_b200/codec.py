@@ -132,20 +132,28 @@ def rans_encode(sym: np.ndarray, scales: np.ndarray, symfmt: int, chunk_symbols:
 
 
 def choose_prob_bits(counts, max_loss: float = 0.005) -> int:
-    """8 when an 8-bit table codes these symbol counts within max_loss (relative) of the 12-bit
-    table's rate, else 12.  8-bit tables halve the decoder's renormalisation work; they suit
-    low-entropy alphabets (a few Int8 values), not the ~6.5-bit Float8 one."""
+    """The smallest table (7, then 8 bits) that codes these symbol counts within max_loss
+    (relative) of the 12-bit table's rate, else 12.  7- and 8-bit tables halve the decoder's
+    renormalisation work and 7-bit ones decode two symbols per lookup; they suit low-entropy
+    alphabets (a few Int8 values), not the ~6.5-bit Float8 one.  A 7-bit table holds at most 128
+    symbols, an 8-bit one 256."""
     c = np.asarray(counts, dtype=np.float64).ravel()
-    if c.sum() == 0 or np.count_nonzero(c) > 256:
+    used = int(np.count_nonzero(c))
+    if c.sum() == 0:
         return 12
     cu = np.ascontiguousarray(c, dtype=np.uint64)
     rate = {}
-    for pb in (8, 12):
+    for pb in (7, 8, 12):
+        if used > (1 << pb):
+            continue
         f = np.zeros(256, np.uint32)
         L.check(L.lib().eq_rans_normalize_host(_p(cu), pb, _p(f)), "eq_rans_normalize_host")
         m = c > 0
         rate[pb] = float(-(c[m] * np.log2(f[m] / float(1 << pb))).sum() / c.sum())
-    return 8 if rate[8] <= rate[12] * (1 + max_loss) else 12
+    for pb in (7, 8):
+        if pb in rate and rate[pb] <= rate[12] * (1 + max_loss):
+            return pb
+    return 12
 
 
 @dataclass

@@ -156,7 +156,7 @@ extern "C" eq_status eq_quantize_excluding_host(const float *w, uint32_t rows, u
 
 extern "C" eq_status eq_rans_normalize_host(const uint64_t *counts, uint32_t prob_bits,
                                             uint32_t *freqs) {
-  if (!counts || !freqs || prob_bits < 8 || prob_bits > 15) return EQ_ERR_ARG;
+  if (!counts || !freqs || prob_bits < 7 || prob_bits > 15) return EQ_ERR_ARG;
   const uint64_t M = 1ull << prob_bits;
   uint64_t n = 0;
   for (int s = 0; s < 256; ++s) n += counts[s];
@@ -205,9 +205,10 @@ extern "C" eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint
   uint32_t cum[257];
   cum[0] = 0;
   for (int s = 0; s < 256; ++s) cum[s + 1] = cum[s] + freqs[s];
-  if (cum[256] != 256u && cum[256] != 4096u) return EQ_ERR_FORMAT;
-  // 8-bit tables renormalise after every second step of a stream, 12-bit ones after every step
-  const uint32_t pb = cum[256] == 256u ? 8u : 12u, k = 16u / pb;
+  if (cum[256] != 128u && cum[256] != 256u && cum[256] != 4096u) return EQ_ERR_FORMAT;
+  // 7- and 8-bit tables renormalise after every second step of a stream, 12-bit ones after
+  // every step
+  const uint32_t pb = cum[256] == 128u ? 7u : cum[256] == 256u ? 8u : 12u, k = 16u / pb;
   const uint64_t nchunks = (N + chunk - 1) / chunk;
   const uint32_t groups = (streams + 31) / 32;  // 32 streams share one word substream
   std::vector<std::vector<uint16_t>> pieces(nchunks * groups);

@@ -96,7 +96,7 @@ struct EncodeParams {
   uint64_t numel;
   uint64_t units;
   uint32_t chunk, streams, groups, run;
-  uint32_t prob_bits;  // 12, or 8: renormalise after every second step (then run == 8)
+  uint32_t prob_bits;  // 12, or 8 / 7: renormalise after every second step (then run == 8)
   uint16_t freq[256];
 };
 
@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(256) rans_encode_kernel(const __grid_constant_
         // flush bound of the renormalisation group that ends at this step: one step (12-bit
         // tables), or positions p - 1 and p of the run (8-bit tables, p odd)
         if (P.prob_bits == 12) xmax = uint64_t(f) << 20;
-        else if (p & 1) xmax = (uint64_t(f) * max(fs[src[j - 1]], 1u)) << 16;
+        else if (p & 1) xmax = (uint64_t(f) * max(fs[src[j - 1]], 1u)) << (32 - 2 * P.prob_bits);
       }
       const bool emit = on && xmax && uint64_t(x) >= xmax;
       const uint32_t em = __ballot_sync(0xFFFFFFFFu, emit);
@@ -226,10 +226,10 @@ static eq_status check_encode_args(const uint8_t *d_sym, uint32_t rows, uint32_t
     sum += host_freqs[s];
     P.freq[s] = uint16_t(host_freqs[s]);
   }
-  if (sum != 256 && sum != kRansSlots) return EQ_ERR_FORMAT;
-  P.prob_bits = sum == 256 ? 8 : 12;
+  if (sum != 128 && sum != 256 && sum != kRansSlots) return EQ_ERR_FORMAT;
+  P.prob_bits = sum == 128 ? 7 : sum == 256 ? 8 : 12;
   // pairs of steps stay inside runs only when every run is whole
-  if (P.prob_bits == 8 && (run != 8 || cols % 8)) return EQ_ERR_UNSUPPORTED;
+  if (P.prob_bits != 12 && (run != 8 || cols % 8)) return EQ_ERR_UNSUPPORTED;
   P.sym = d_sym;
   P.numel = numel;
   P.chunk = chunk;

@@ -31,6 +31,8 @@ struct WordRing {
   uint32_t ready;   // segments waited for
   uint32_t ready_end;  // offsets below this have landed (ready segments)
   uint32_t refill_at;  // once q reaches this offset a slot can be refilled
+  uint32_t phase;      // bit s: the phase the next wait on slot s's barrier waits for (it
+                       // carries over from one substream to the next a warp decodes)
 
   __device__ __forceinline__ void issue(uint32_t lane) {
     if (lane == 0) {
@@ -59,12 +61,19 @@ struct WordRing {
     while (issued < min(nseg, kNumSeg)) issue(lane);
   }
 
+  // the copy into `slot` has landed (bounded wait); false on timeout
+  __device__ __forceinline__ bool wait_slot(uint32_t slot) {
+    if (!mbar_wait_bounded(&bar[slot], (phase >> slot) & 1u)) return false;
+    phase ^= 1u << slot;
+    return true;
+  }
+
   // every byte below `end` (an offset from A) must have landed; false on timeout
   __device__ __forceinline__ bool wait_below(uint32_t end) {
     if (nseg == 0) return true;
     const uint32_t last = min(nseg - 1, (end - 1) / kSegBytes);
     while (ready <= last) {
-      if (!mbar_wait_bounded(&bar[ready % kNumSeg], (ready / kNumSeg) & 1u)) return false;
+      if (!wait_slot(ready % kNumSeg)) return false;
       ++ready;
     }
     ready_end = ready * kSegBytes;
@@ -95,7 +104,7 @@ struct WordRing {
   // wait (bounded) for every copy handed to the engine; EQ_DEV_TIMEOUT or 0
   __device__ __forceinline__ uint32_t drain() {
     while (ready < issued) {
-      if (!mbar_wait_bounded(&bar[ready % kNumSeg], (ready / kNumSeg) & 1u)) return EQ_DEV_TIMEOUT;
+      if (!wait_slot(ready % kNumSeg)) return EQ_DEV_TIMEOUT;
       ++ready;
     }
     return 0;
@@ -156,6 +165,27 @@ __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, cons
   return e;
 }
 
+// Two decode steps of a 7-bit stream with one pair-table lookup (layout in eq_internal.cuh):
+// x2 = F * (x >> 14) + B.  Returns the two symbols as a 16-bit pair (the first in the low byte).
+template <bool FULL>
+__device__ __forceinline__ uint32_t rans_pair_step(uint32_t &x, bool act, const uint32_t *lut) {
+  const uint32_t base = uint32_t(__cvta_generic_to_shared(lut));
+  uint32_t w0, nx;
+  asm volatile(
+      "{\n\t.reg .b32 a, w1, f, xs;\n\t"
+      "and.b32 a, %2, 16383;\n\t"
+      "shl.b32 a, a, 3;\n\t"
+      "add.u32 a, a, %3;\n\t"
+      "shr.u32 xs, %2, 14;\n\t"
+      "ld.shared.v2.u32 {%1, w1}, [a];\n\t"
+      "and.b32 f, %1, 65535;\n\t"
+      "mad.lo.u32 %0, f, xs, w1;\n\t}"
+      : "=r"(nx), "=r"(w0)
+      : "r"(x), "r"(base));
+  if (FULL || act) x = nx;
+  return w0 >> 16;
+}
+
 // the symbol byte of a PB-bit entry
 template <uint32_t PB>
 constexpr uint32_t kSymShift = PB == 8 ? 16 : PB;
@@ -209,6 +239,7 @@ __device__ __forceinline__ void ring_init(WordRing &R, unsigned char *smem, unsi
   R.buf = rings + warp * kRingBytes;
   R.ring_off = uint32_t(R.buf - smem);
   R.bar = bars + warp * kNumSeg;
+  R.phase = 0;
   if (lane == 0) {
     for (uint32_t s = 0; s < kNumSeg; ++s) mbar_init(&R.bar[s], 1);
     fence_mbar_init();
@@ -217,10 +248,12 @@ __device__ __forceinline__ void ring_init(WordRing &R, unsigned char *smem, unsi
 
 #endif  // __CUDACC__
 
-// bytes before the first ring: the slot table (2^pb entries), padded so that every ring starts at
-// a multiple of its own size (the word address is formed with an OR)
+// bytes before the first ring: the slot table (2^pb entries; for 7-bit tables the pair table),
+// padded so that every ring starts at a multiple of its own size (the word address is formed with
+// an OR)
 __host__ __device__ constexpr uint32_t rans_lut_bytes(uint32_t pb) {
-  return ((4u << pb) + kRingBytes - 1) / kRingBytes * kRingBytes;
+  return pb == kRansPairBits ? kRansPairEntries * 8u
+                             : ((4u << pb) + kRingBytes - 1) / kRingBytes * kRingBytes;
 }
 
 // shared memory of a CTA: the slot table, then one ring per warp, then the rings' barriers

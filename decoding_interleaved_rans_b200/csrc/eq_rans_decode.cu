@@ -42,7 +42,7 @@ struct RansDesc {
   uint32_t chunk_symbols;
   uint32_t groups;        // streams / 32
   uint32_t cta_begin;     // first CTA of this tensor in the launch
-  uint32_t pad;
+  uint32_t ctas;          // CTAs of this tensor: its warps take units cta_warp, + ctas * warps, ...
 };
 
 struct RansDecodeParams {
@@ -63,16 +63,29 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
                                              const uint32_t *lut, const unsigned char *smem,
                                              const WordRing &R, uint32_t &q, uint32_t lt,
                                              uint16_t *out, float sc, bool nan_codes) {
-  static_assert(PB == 12 || G == 8, "8-bit tables need whole runs of 8");
-  uint32_t e[G];
+  static_assert(PB == 12 || G == 8, "7- and 8-bit tables need whole runs of 8");
+  if constexpr (PB == kRansPairBits) {  // one lookup per pair of steps
+    uint32_t pr[4];
 #pragma unroll
-  for (int p = 0; p < G; ++p) {
-    e[p] = rans_decode_step<FULL, PB>(x, act, lut);
-    if (PB == 12 || (p & 1)) rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
-  }
-  if (FULL || act) {
-    if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
-    else *out = dequant1<FMT>((e[0] >> kSymShift<PB>) & 0xFFu, sc);
+    for (int k = 0; k < 4; ++k) {
+      pr[k] = rans_pair_step<FULL>(x, act, lut);
+      rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
+    }
+    if (FULL || act)
+      *reinterpret_cast<uint4 *>(out) =
+          make_uint4(dequant2<FMT>(pr[0], sc, nan_codes), dequant2<FMT>(pr[1], sc, nan_codes),
+                     dequant2<FMT>(pr[2], sc, nan_codes), dequant2<FMT>(pr[3], sc, nan_codes));
+  } else {
+    uint32_t e[G];
+#pragma unroll
+    for (int p = 0; p < G; ++p) {
+      e[p] = rans_decode_step<FULL, PB>(x, act, lut);
+      if (PB == 12 || (p & 1)) rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
+    }
+    if (FULL || act) {
+      if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
+      else *out = dequant1<FMT>((e[0] >> kSymShift<PB>) & 0xFFu, sc);
+    }
   }
 }
 
@@ -144,7 +157,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   uint16_t *out = D.out + jrun;
   // ring checks once per round (12-bit: up to 256 words a round), or once per two rounds
   // (8-bit: up to 128 words a round); round_wait covers 256 words and one more
-  constexpr uint32_t kRoundsPerCheck = PB == 8 ? 2 : 1;
+  constexpr uint32_t kRoundsPerCheck = PB == 12 ? 1 : 2;
   for (uint32_t r = 0; r < rounds; r += kRoundsPerCheck) {
     if (!R.round_wait(q)) {
       status |= EQ_DEV_TIMEOUT;
@@ -180,8 +193,11 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   return status;
 }
 
+// 7-bit tables: one CTA of up to 32 warps per SM shares the 128 KiB pair table, each warp
+// decoding unit after unit; otherwise up to 16 warps per CTA, one unit each.
 template <int G, int FMT, uint32_t PB>
-__global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
+__global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
+    rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
   unsigned char *rings = smem + rans_lut_bytes(PB);
@@ -197,18 +213,25 @@ __global__ void __launch_bounds__(512) rans_decode_kernel(const __grid_constant_
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(D.table);
+  // the table is only read as far as its header says it reaches: a descriptor whose table is of
+  // another size is reported below, never read past its end
+  const bool table_ok =
+      hdr.magic == (PB == kRansPairBits ? kRansPairMagic : kRansMagic) && hdr.prob_bits == PB;
   const uint4 *src = reinterpret_cast<const uint4 *>(D.table + sizeof(RansTableHeader) / 4);
-  for (uint32_t i = threadIdx.x; i < (1u << PB) / 4; i += blockDim.x)
-    reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+  constexpr uint32_t kLutVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
+  if (table_ok)
+    for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x)
+      reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
   WordRing R;
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
-  const uint64_t unit = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
+  uint64_t unit = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
   if (unit >= D.units) return;
-  uint32_t status = 0;
-  if (hdr.magic != kRansMagic || hdr.prob_bits != PB) status = EQ_DEV_CORRUPT_STATE;
-  else status = decode_group<G, FMT, PB>(D, lut, smem, hdr.flags, hdr.single_sym, R, unit, lane);
+  const uint64_t stride = uint64_t(D.ctas) * P.warps;
+  uint32_t status = table_ok ? 0u : EQ_DEV_CORRUPT_STATE;
+  for (; unit < D.units && !status; unit += stride)
+    status = decode_group<G, FMT, PB>(D, lut, smem, hdr.flags, hdr.single_sym, R, unit, lane);
   if (lane == 0) report(P.status, status);
 }
 
@@ -223,6 +246,9 @@ static KernelFn pick_kernel(uint32_t symfmt, uint32_t run, uint32_t pb) {
     return e4 ? rans_decode_kernel<8, EQ_SYM_E4M3, 12> : rans_decode_kernel<8, EQ_SYM_INT8, 12>;
   if (run == 8 && pb == 8)
     return e4 ? rans_decode_kernel<8, EQ_SYM_E4M3, 8> : rans_decode_kernel<8, EQ_SYM_INT8, 8>;
+  if (run == 8 && pb == kRansPairBits)
+    return e4 ? rans_decode_kernel<8, EQ_SYM_E4M3, kRansPairBits>
+              : rans_decode_kernel<8, EQ_SYM_INT8, kRansPairBits>;
   if (run == 1 && pb == 12)
     return e4 ? rans_decode_kernel<1, EQ_SYM_E4M3, 12> : rans_decode_kernel<1, EQ_SYM_INT8, 12>;
   return nullptr;
@@ -232,9 +258,9 @@ static KernelFn pick_kernel(uint32_t symfmt, uint32_t run, uint32_t pb) {
 eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   if (t.version != EQ_ABI_VERSION) return EQ_ERR_ARG;
   if (t.symfmt != EQ_SYM_E4M3 && t.symfmt != EQ_SYM_INT8) return EQ_ERR_ARG;
-  if (t.prob_bits != 12 && t.prob_bits != 8) return EQ_ERR_UNSUPPORTED;
+  if (t.prob_bits != 12 && t.prob_bits != 8 && t.prob_bits != kRansPairBits) return EQ_ERR_UNSUPPORTED;
   if (t.run != 1 && t.run != 8) return EQ_ERR_UNSUPPORTED;
-  if (t.prob_bits == 8 && t.run != 8) return EQ_ERR_UNSUPPORTED;  // pairs of steps inside runs
+  if (t.prob_bits != 12 && t.run != 8) return EQ_ERR_UNSUPPORTED;  // pairs of steps inside runs
   if (t.streams == 0 || t.streams % 32 || t.streams > 1024) return EQ_ERR_UNSUPPORTED;
   const uint64_t numel = uint64_t(t.rows) * t.cols;
   if (numel >= (1ull << 40)) return EQ_ERR_UNSUPPORTED;
@@ -252,7 +278,7 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   return EQ_OK;
 }
 
-static bool g_attr_set[64][2][2][2];  // device, symfmt, run == 8, prob_bits == 8
+static bool g_attr_set[64][2][2][3];  // device, symfmt, run == 8, table (12 / 8 / 7 bits)
 
 static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
                               uint16_t *const *d_out, uint32_t *d_status, cudaStream_t st) {
@@ -261,17 +287,25 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
   if (!fn) return EQ_ERR_UNSUPPORTED;
   uint64_t total_units = 0;
   for (uint32_t i : idx) total_units += ts[i].num_chunks * (ts[i].streams / 32);
-  // warps (= groups) per CTA: 16 when the work covers every SM several times over
   const uint64_t sms = uint64_t(device_sm_count());
-  uint32_t warps = 16;
-  while (warps > 1 && (total_units + warps - 1) / warps < 4 * sms) warps >>= 1;
+  const bool pair = t0.prob_bits == kRansPairBits;
+  uint32_t warps;
+  if (pair) {
+    // one CTA per SM holds the 128 KiB pair table; enough warps that the SMs' CTAs take every
+    // unit about once (larger tensors: the warps loop)
+    warps = uint32_t(std::min<uint64_t>(32, std::max<uint64_t>(1, (total_units + sms - 1) / sms)));
+  } else {
+    // warps (= groups) per CTA: 16 when the work covers every SM several times over
+    warps = 16;
+    while (warps > 1 && (total_units + warps - 1) / warps < 4 * sms) warps >>= 1;
+  }
   const size_t smem = rans_smem_bytes(warps, t0.prob_bits);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8][t0.prob_bits == 8];
+  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8][pair ? 2 : t0.prob_bits == 8];
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(rans_smem_bytes(16, t0.prob_bits)));
+                                         int(rans_smem_bytes(pair ? 32 : 16, t0.prob_bits)));
     if (e != cudaSuccess) return EQ_ERR_CUDA;
     attr = true;
   }
@@ -302,9 +336,12 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
       D.rows = t.rows;
       D.cols = t.cols;
       D.chunk_symbols = t.chunk_symbols;
+      uint64_t n_ctas = (D.units + warps - 1) / warps;
+      if (pair)  // at most the tensor's share of the SMs, at least one CTA
+        n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, D.units * sms / total_units));
       D.cta_begin = uint32_t(ctas);
-      D.pad = 0;
-      ctas += (D.units + warps - 1) / warps;
+      D.ctas = uint32_t(n_ctas);
+      ctas += n_ctas;
     }
     if (P.n == 0) continue;
     if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
@@ -331,9 +368,11 @@ extern "C" eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uin
       return EQ_ERR_ARG;
   }
   // one launch per kernel variant (symbol format x run length x table size)
-  std::vector<std::vector<uint32_t>> groups(8);
-  for (uint32_t i = 0; i < n_tensors; ++i)
-    groups[(ts[i].symfmt - 1) * 4 + (ts[i].run == 8) * 2 + (ts[i].prob_bits == 8)].push_back(i);
+  std::vector<std::vector<uint32_t>> groups(12);
+  for (uint32_t i = 0; i < n_tensors; ++i) {
+    const uint32_t table = ts[i].prob_bits == 12 ? 0 : ts[i].prob_bits == 8 ? 1 : 2;
+    groups[(ts[i].symfmt - 1) * 6 + (ts[i].run == 8) * 3 + table].push_back(i);
+  }
   for (auto &g : groups) {
     if (g.empty()) continue;
     eq_status s = launch_group(ts, g, d_out, d_status, static_cast<cudaStream_t>(stream));

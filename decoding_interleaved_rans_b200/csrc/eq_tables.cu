@@ -51,6 +51,41 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
   }
 }
 
+// The pair table of a 7-bit frequency table (layout in eq_internal.cuh): one block of 256
+// threads, each entry from two slot -> symbol searches.
+__global__ void __launch_bounds__(256) rans_pair_build_kernel(const __grid_constant__ RansBuildArgs a) {
+  __shared__ uint32_t cum[257];
+  const uint32_t t = threadIdx.x;
+  if (t == 0) {
+    uint32_t c = 0;
+    for (int s = 0; s < 256; ++s) {
+      cum[s] = c;
+      c += a.freq[s];
+    }
+    cum[256] = c;
+    RansTableHeader h{kRansPairMagic, a.flags, a.single, kRansPairBits};
+    *reinterpret_cast<RansTableHeader *>(a.dst) = h;
+  }
+  __syncthreads();
+  auto owner = [&](uint32_t slot) {  // largest s with cum[s] <= slot
+    int lo = 0, hi = 255;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cum[mid] <= slot) lo = mid; else hi = mid - 1;
+    }
+    return uint32_t(lo);
+  };
+  uint2 *ent = reinterpret_cast<uint2 *>(a.dst + sizeof(RansTableHeader) / 4);
+  for (uint32_t i = t; i < kRansPairEntries; i += blockDim.x) {
+    const uint32_t slot1 = i & 127u, L = i >> 7;
+    const uint32_t s1 = owner(slot1), f1 = a.freq[s1];
+    const uint32_t v = f1 * L + (slot1 - cum[s1]);
+    const uint32_t slot2 = v & 127u, s2 = owner(slot2), f2 = a.freq[s2];
+    const uint32_t F = f1 * f2, B = f2 * (v >> 7) + (slot2 - cum[s2]);
+    ent[i] = make_uint2((F & 0xFFFFu) | (s1 << 16) | (s2 << 24), B);
+  }
+}
+
 struct HuffBuildArgs {
   uint32_t *dst;
   HuffTableHeader h;
@@ -177,6 +212,7 @@ using namespace eq;
 
 extern "C" size_t eq_table_bytes(eq_table_kind kind) {
   if (kind == EQ_TABLE_RANS) return kRansTableBytes;
+  if (kind == EQ_TABLE_RANS_PAIR) return kRansPairTableBytes;
   if (kind == EQ_TABLE_HUFF) return kHuffTableBytes;
   return 0;
 }
@@ -185,8 +221,9 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
                                      uint32_t prob_bits, void *d_tables, void *stream) {
   if (!host_in || !d_tables || !aligned(d_tables, 16)) return EQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (kind == EQ_TABLE_RANS) {
-    if (prob_bits != 12 && prob_bits != 8) return EQ_ERR_UNSUPPORTED;
+  if (kind == EQ_TABLE_RANS || kind == EQ_TABLE_RANS_PAIR) {
+    if (kind == EQ_TABLE_RANS ? (prob_bits != 12 && prob_bits != 8) : prob_bits != kRansPairBits)
+      return EQ_ERR_UNSUPPORTED;
     const uint32_t slots = 1u << prob_bits;
     RansBuildArgs a;
     a.dst = static_cast<uint32_t *>(d_tables);
@@ -206,7 +243,8 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
     a.flags = (host_in[0x7F] ? kRansFlagNaN7F : 0u) | (host_in[0xFF] ? kRansFlagNaNFF : 0u) |
               (used == 1 ? kRansFlagSingle : 0u);
     a.single = used == 1 ? single : 0u;
-    rans_build_kernel<<<1, 256, 0, st>>>(a);
+    if (kind == EQ_TABLE_RANS) rans_build_kernel<<<1, 256, 0, st>>>(a);
+    else rans_pair_build_kernel<<<1, 256, 0, st>>>(a);
     return cuda_status(cudaGetLastError());
   }
   if (kind == EQ_TABLE_HUFF) {

@@ -52,7 +52,7 @@ typedef enum {
 #define EQ_DEV_TIMEOUT 16u       /* a bounded wait on an asynchronous copy gave up            */
 
 typedef enum { EQ_SYM_E4M3 = 1, EQ_SYM_INT8 = 2 } eq_symfmt;
-typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
+typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2, EQ_TABLE_RANS_PAIR = 3 } eq_table_kind;
 
 /*
  * One interleaved-rANS-coded weight W[rows][cols] ("Float8@2bits: Entropy Coding Enables
@@ -61,7 +61,7 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
  * output channel, are flattened into one symbol stream and ANS-coded; a parallel ANS decoder
  * restores them on the GPU before the layer runs).  The pages fix no rANS variant; this one is:
  *
- *   probabilities M = 2^prob_bits (prob_bits = 12 or 8), state x in [2^16, 2^32), 16-bit words.
+ *   probabilities M = 2^prob_bits (prob_bits = 12, 8 or 7), state x in [2^16, 2^32), 16-bit words.
  *   The row-major symbol stream is cut into chunks of chunk_symbols symbols (the last one may be
  *   shorter); chunk c is coded on its own by `streams` interleaved rANS states.  Inside a chunk,
  *   symbol j belongs to run r = j / run, stream r % streams, round r / streams, position j % run;
@@ -71,9 +71,10 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2 } eq_table_kind;
  *   Decoding symbol s from x: slot = x mod M, s is the symbol with cum[s] <= slot < cum[s] +
  *   freq[s], x = freq[s] * (x / M) + slot - cum[s].  At a renormalisation point, if x < 2^16,
  *   x = x * 2^16 + the next word of the stream's group.  A 12-bit stream has a renormalisation
- *   point after each of its steps; an 8-bit stream after every second one of its own steps
- *   (and after its last), which is exact because two 8-bit steps shrink the state by at most
- *   2^16; it halves the renormalisation work.  A well-formed chunk ends with every state at
+ *   point after each of its steps; an 8- or 7-bit stream after every second one of its own
+ *   steps (and after its last), which is exact because two such steps shrink the state by at
+ *   most 2^16; it halves the renormalisation work.  A 7-bit table also decodes both steps of a
+ *   pair with one lookup (EQ_TABLE_RANS_PAIR).  A well-formed chunk ends with every state at
  *   2^16 and every word read.
  *   Dequantisation: out = bf16_rne( value(s) * scale[row] ), value(s) being the E4M3 value of the
  *   byte (NaN codes 0x7F/0xFF give the bf16 quiet NaN 0x7FC0 / 0xFFC0) or the byte read as int8.
@@ -87,7 +88,7 @@ typedef struct {
   uint32_t version;       /* EQ_ABI_VERSION                                                    */
   uint32_t symfmt;        /* eq_symfmt                                                         */
   uint32_t rows, cols;    /* W is rows x cols, row-major; rows*cols < 2^40                     */
-  uint32_t prob_bits;     /* 12, or 8 (then run must be 8)                                      */
+  uint32_t prob_bits;     /* 12, or 8 or 7 (then run must be 8)                                 */
   uint32_t chunk_symbols; /* symbols per chunk (>= 1); a multiple of `run`                     */
   uint32_t streams;       /* interleaved states per chunk: a multiple of 32, at most 1024      */
   uint32_t run;           /* consecutive symbols per stream visit: 1 or 8; 8 needs cols % 8 == 0 */
@@ -98,8 +99,8 @@ typedef struct {
   const uint16_t *words;  /* all substreams, chunk-major, decoder order; allocation padded with
                              zeros to a multiple of 8 words (16 bytes); base 16-byte aligned    */
   const uint16_t *scales; /* [rows] bf16 per-output-channel scales                              */
-  const void *tables;     /* eq_table_bytes(EQ_TABLE_RANS) bytes from eq_build_tables(RANS);
-                             16-byte aligned                                                    */
+  const void *tables;     /* from eq_build_tables: EQ_TABLE_RANS for 12- and 8-bit tables,
+                             EQ_TABLE_RANS_PAIR for 7-bit ones; 16-byte aligned               */
   uint64_t n_patch;       /* super weights in the list (0: none)                               */
   const uint64_t *patch_idx; /* [n_patch] flat row-major indices, strictly increasing           */
   const uint16_t *patch_val; /* [n_patch] their bf16 values                                     */
@@ -166,6 +167,10 @@ size_t eq_table_bytes(eq_table_kind kind);
  *     or 8).
  *     Builds the slot table: one 32-bit entry per slot holding the slot's symbol, its frequency
  *     and slot - cum[symbol].
+ *   EQ_TABLE_RANS_PAIR: host_in[256] = frequencies summing to 128 (prob_bits = 7).  Builds the
+ *     pair table (16384 x 8 bytes): for each value of the state's low 14 bits, the two symbols
+ *     the next two steps decode and the two steps' combined product and offset, so a pair of
+ *     steps is one lookup and one multiply-add.
  *   EQ_TABLE_HUFF: host_in[256] = code length of each exponent value (0 = absent), prob_bits
  *     ignored.  Builds the hierarchical lookup tables of the DFloat11 page ("Decodificacion
  *     basada en LUT jerarquicas": the code tree cut into height-8 subtrees, each a 256-entry

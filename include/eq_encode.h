@@ -64,8 +64,8 @@ eq_status eq_rans_normalize_host(const uint64_t *counts, uint32_t prob_bits, uin
  * Interleaved-rANS encoding of a symbol matrix sym[rows][cols] in the format of eq_rans_tensor.
  * chunk_symbols = 0 means one row per chunk.  states: [num_chunks * streams]; word_off:
  * [num_chunks * ceil(streams / 32) + 1] (one word substream per chunk and group of 32 streams).
- * freqs sums to 4096 (12-bit table) or 256 (8-bit table, whose streams renormalise after every
- * second step).  The words are returned in a buffer the library allocates (*words, *n_words
+ * freqs sums to 4096 (12-bit table), or 256 / 128 (8- / 7-bit table, whose streams renormalise
+ * after every second step).  The words are returned in a buffer the library allocates (*words, *n_words
  * words, zero-padded to a multiple of 8); release it with eq_free_host.
  */
 eq_status eq_rans_encode_host(const uint8_t *sym, uint32_t rows, uint32_t cols,
@@ -127,8 +127,8 @@ void eq_free_host(void *p);
  *   offsets d_word_off ([num_chunks * streams / 32 + 1]; d_word_off[last] = total words).
  * eq_rans_encode_device: encodes again and writes the words at those offsets into d_words (room
  *   for d_word_off[last] words, rounded up to a multiple of 8 and zero-filled by the caller).
- * host_freqs: the frequency table (host memory, 256 entries summing to 4096, or to 256 for an
- * 8-bit table, which needs run == 8 and cols % 8 == 0, else EQ_ERR_UNSUPPORTED).  A symbol without
+ * host_freqs: the frequency table (host memory, 256 entries summing to 4096, or to 256 / 128 for
+ * an 8- / 7-bit table, which needs run == 8 and cols % 8 == 0, else EQ_ERR_UNSUPPORTED).  A symbol without
  * frequency sets EQ_DEV_BAD_CODE in *d_status; a word count that does not match the plan sets
  * EQ_DEV_COUNT_MISMATCH.
  */

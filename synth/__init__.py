@@ -189,7 +189,7 @@ class Workload:
     int8_div: float = 0.0          # Int8: scale = absmax(row) / int8_div
     batches: tuple = field(default=())
     chunk_rows: int = 0            # > 0: chunks of this many whole rows (overrides chunk_symbols)
-    prob_bits: int = 12            # rANS table precision: 12, or 8 for low-entropy alphabets
+    prob_bits: int = 12            # rANS table precision: 12, or 8 / 7 for low-entropy alphabets
 
     def chunk_for(self, spec: "TensorSpec") -> int:
         """Chunk length in symbols for one tensor of the workload."""
@@ -223,7 +223,7 @@ WORKLOADS = {
                         symfmt="e4m3", chunk_symbols=16384, streams=32, run=8),
     "int8_8k": Workload("int8_8k", (TensorSpec("w", 8192, 8192, "laplace_clipped", 2, 0),),
                         symfmt="int8", chunk_symbols=65536, streams=128, run=8,
-                        int8_div=INT8_DIV_LAPLACE_8K, prob_bits=8),
+                        int8_div=INT8_DIV_LAPLACE_8K, prob_bits=7),
     "llama2_7b": Workload("llama2_7b", _llama2_7b(), symfmt="e4m3", chunk_symbols=65536,
                           streams=128, run=8),
     "mlp_13b": Workload("mlp_13b", (TensorSpec("gate", 13824, 5120, "normal", 4, 0),

@@ -50,24 +50,27 @@ def test_rans_encode_matches_oracle(eq, orc, chunk, S, G):
     assert np.array_equal(a.words, b.words)
 
 
+@pytest.mark.parametrize("pb", [8, 7])
 @pytest.mark.parametrize("chunk,S,G", [(65536, 128, 8), (999, 32, 1), (0, 64, 8), (4096, 32, 3)])
-def test_rans_encode_8bit_matches_oracle(eq, orc, chunk, S, G):
+def test_rans_encode_8bit_matches_oracle(eq, orc, chunk, S, G, pb):
     w = synth.laplace_clipped(96, 1024, 0.01, 0.06, 7)
     sym, sc = orc.quantize(w, orc.INT8, synth.INT8_DIV_LAPLACE_8K)
-    f = orc.rans_freqs(sym, 8)
-    assert np.array_equal(eq.codec.rans_freqs(sym, 8), f)
-    a = eq.codec.rans_encode(sym, sc, 2, chunk, S, G, prob_bits=8)
-    b = orc.rans_encode(sym, sc, 2, chunk, S, G, prob_bits=8)
+    f = orc.rans_freqs(sym, pb)
+    assert np.array_equal(eq.codec.rans_freqs(sym, pb), f)
+    a = eq.codec.rans_encode(sym, sc, 2, chunk, S, G, prob_bits=pb)
+    b = orc.rans_encode(sym, sc, 2, chunk, S, G, prob_bits=pb)
     assert np.array_equal(a.states, b.states)
     assert np.array_equal(a.word_off, b.word_off)
     assert np.array_equal(a.words, b.words)
 
 
 def test_choose_prob_bits(eq, orc):
-    """8-bit tables for the 2-bit Int8 workload, 12-bit ones for ~6.5-bit Float8 weights."""
+    """7-bit tables for the 2-bit Int8 workload, 12-bit ones for ~6.5-bit Float8 weights, 8-bit
+    ones where 7 bits would lose too much."""
     wl = synth.WORKLOADS["int8_8k"]
     sym, _ = orc.quantize(wl.tensors[0].generate(row_lo=0, row_hi=256), orc.INT8, wl.int8_div)
-    assert eq.codec.choose_prob_bits(np.bincount(sym.ravel(), minlength=256)) == wl.prob_bits == 8
+    assert eq.codec.choose_prob_bits(np.bincount(sym.ravel(), minlength=256)) == wl.prob_bits == 7
+    assert eq.codec.choose_prob_bits(np.bincount(sym.ravel(), minlength=256), 0.002) == 8
     sym, _ = orc.quantize(synth.WORKLOADS["e4m3_1k"].tensors[0].generate(), orc.E4M3)
     assert eq.codec.choose_prob_bits(np.bincount(sym.ravel(), minlength=256)) == 12
 

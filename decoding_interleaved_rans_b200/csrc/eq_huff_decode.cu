@@ -246,6 +246,11 @@ __global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_consta
     uint32_t bad = 0;
     BytePacker pk{reinterpret_cast<uint32_t *>(ebuf) + tid, T};
     const uint32_t cnt = segment(win, tree, ntab, r0, r1, r2, pos, end, pk, &bad);
+    // the values leave this thread's column for registers now: the scan's barriers then also
+    // order every column read before the compacting writes below
+    Staged stg;
+    stage_read(reinterpret_cast<const uint32_t *>(ebuf) + tid, T, cnt, stg);
+    const uint64_t o0 = __ldg(P.block_out + b), o1 = __ldg(P.block_out + b + 1);  // in flight
     // ---- block-wide exclusive scan of the counts ----
     uint32_t incl = cnt;
 #pragma unroll
@@ -270,7 +275,6 @@ __global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_consta
     const uint32_t total = wsum[32];
     const uint32_t off = wsum[warp] + incl - cnt;
 
-    const uint64_t o0 = P.block_out[b], o1 = P.block_out[b + 1];
     uint64_t m = total;
     if (o1 < o0 || o1 > P.n) {
       err |= EQ_DEV_OVERRUN;
@@ -283,9 +287,6 @@ __global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_consta
     // ---- stage 2: every thread moves its values to their block positions (shifted so that
     //      8-aligned outputs are 8-aligned in shared memory) ----
     const uint32_t shift = uint32_t(o0 & 7);
-    Staged stg;
-    stage_read(reinterpret_cast<const uint32_t *>(ebuf) + tid, T, cnt, stg);
-    __syncthreads();
     if (off + cnt <= m) stage_write(ebuf, shift + off, cnt, stg);
     __syncthreads();
 

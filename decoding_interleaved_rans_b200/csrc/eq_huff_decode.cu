@@ -83,9 +83,9 @@ struct BytePacker {
   uint64_t acc = 0;  // pending bytes, the oldest in the low bits
   uint32_t nb = 0, wp = 0;
 
-  // append the low k (1..4) bytes of v
+  // append the low k (1..4) bytes of v, whose higher bytes are zero (window-table entries hold
+  // zeros past their k values; single values are below 256)
   __device__ __forceinline__ void put(uint32_t v, uint32_t k) {
-    if (k < 4) v &= (1u << (8 * k)) - 1u;
     acc |= uint64_t(v) << (8 * nb);
     nb += k;
     if (nb >= 4) {

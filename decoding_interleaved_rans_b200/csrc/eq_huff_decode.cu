@@ -55,11 +55,6 @@ __host__ __device__ constexpr size_t huff_smem_bytes(uint32_t tpb) {
 
 __device__ __forceinline__ uint32_t bswap32(uint32_t v) { return __byte_perm(v, 0, 0x0123); }
 
-// the 32 code bits starting at bit `pos` (0..63) of the thread's 96-bit window r0:r1:r2
-__device__ __forceinline__ uint32_t bits32(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t pos) {
-  return pos < 32 ? __funnelshift_l(r1, r0, pos) : __funnelshift_l(r2, r1, pos);
-}
-
 __device__ __forceinline__ uint32_t tree_decode(const uint16_t *tree, uint32_t ntab, uint32_t w,
                                                 uint32_t *sym) {
   uint32_t e = __ldg(tree + (w >> 24)), used = 0;
@@ -105,10 +100,21 @@ struct BytePacker {
 __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t *tree, uint32_t ntab,
                                             uint32_t r0, uint32_t r1, uint32_t r2, uint32_t pos,
                                             uint32_t end, BytePacker &out, uint32_t *bad) {
+  // the next 64 bits of the stream are r0:r1 (r2 behind them); pos, end count from r0's top bit,
+  // and the words slide up once pos passes 32, so every lookup is one funnel shift
   uint32_t cnt = 0;
-  // body: every code found inside a whole 11-bit window starts before `end`
+  // body: every code found inside a whole 11-bit window starts before `end`.  A window whose
+  // first code does not fit (or matches no code) is flagged long and goes to the tree, which
+  // reports bad patterns.
   while (pos + kHuffWindowBits <= end) {
-    const uint32_t w = bits32(r0, r1, r2, pos);
+    if (pos >= 32) {
+      r0 = r1;
+      r1 = r2;
+      r2 = 0;
+      pos -= 32;
+      end -= 32;
+    }
+    const uint32_t w = __funnelshift_l(r1, r0, pos);
     const uint64_t f = win[w >> (32 - kHuffWindowBits)];
     if (f & kHuffLong) {
       uint32_t sym;
@@ -124,24 +130,27 @@ __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t 
     }
     const uint32_t hi = uint32_t(f >> 32);
     const uint32_t k = (hi >> 20) & 7u;
-    if (k == 0) {
-      *bad = EQ_DEV_BAD_CODE;
-      break;
-    }
     out.put(uint32_t(f), k);
     cnt += k;
     pos += (hi >> 16) & 0xFu;
   }
   // tail: codes may reach past `end`; only those starting before it are this thread's
   while (pos < end && !*bad) {
-    const uint32_t w = bits32(r0, r1, r2, pos);
+    if (pos >= 32) {
+      r0 = r1;
+      r1 = r2;
+      r2 = 0;
+      pos -= 32;
+      end -= 32;
+    }
+    const uint32_t w = __funnelshift_l(r1, r0, pos);
     const uint64_t f = win[w >> (32 - kHuffWindowBits)];
     uint32_t sym, len;
     if (f & kHuffLong) {
       len = tree_decode(tree, ntab, w, &sym);
-    } else {
+    } else {  // the first code of the window (a window that is not long holds at least one)
       sym = uint32_t(f) & 0xFFu;
-      len = ((f >> 52) & 7u) ? uint32_t(f >> 32) & 0xFu : 0u;
+      len = uint32_t(f >> 32) & 0xFu;
     }
     if (!len) {
       *bad = EQ_DEV_BAD_CODE;

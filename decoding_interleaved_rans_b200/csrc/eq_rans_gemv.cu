@@ -43,25 +43,25 @@ struct GemvParams {
 __device__ __forceinline__ float lo_bf16(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// acc[b] += sum_i w[i] * x[b][col + i] over one run of 8 weights (packed bf16 pairs)
+__device__ __forceinline__ float2 bf16x2_f2(uint32_t v) { return make_float2(lo_bf16(v), hi_bf16(v)); }
+
+// acc[b] += w[i] * x[b][col + i] over one run of 8 weights (packed bf16 pairs), the even columns
+// in acc[b].x and the odd ones in acc[b].y: two-wide fp32 FMAs, half the instructions and half
+// the dependency chain of one running sum
 template <int BMAX>
-__device__ __forceinline__ void fma_run(float (&acc)[BMAX], uint2 wa, uint2 wb, const uint16_t *x,
+__device__ __forceinline__ void fma_run(float2 (&acc)[BMAX], uint2 wa, uint2 wb, const uint16_t *x,
                                         uint32_t cols, uint32_t col, uint32_t batch) {
-  const float wv[8] = {lo_bf16(wa.x), hi_bf16(wa.x), lo_bf16(wa.y), hi_bf16(wa.y),
-                       lo_bf16(wb.x), hi_bf16(wb.x), lo_bf16(wb.y), hi_bf16(wb.y)};
+  const float2 w01 = bf16x2_f2(wa.x), w23 = bf16x2_f2(wa.y), w45 = bf16x2_f2(wb.x),
+               w67 = bf16x2_f2(wb.y);
 #pragma unroll
   for (int b = 0; b < BMAX; ++b) {
     if (b < int(batch)) {
       const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + size_t(b) * cols + col));
-      float a = acc[b];
-      a = fmaf(wv[0], lo_bf16(xv.x), a);
-      a = fmaf(wv[1], hi_bf16(xv.x), a);
-      a = fmaf(wv[2], lo_bf16(xv.y), a);
-      a = fmaf(wv[3], hi_bf16(xv.y), a);
-      a = fmaf(wv[4], lo_bf16(xv.z), a);
-      a = fmaf(wv[5], hi_bf16(xv.z), a);
-      a = fmaf(wv[6], lo_bf16(xv.w), a);
-      a = fmaf(wv[7], hi_bf16(xv.w), a);
+      float2 a = acc[b];
+      a = __ffma2_rn(w01, bf16x2_f2(xv.x), a);
+      a = __ffma2_rn(w23, bf16x2_f2(xv.y), a);
+      a = __ffma2_rn(w45, bf16x2_f2(xv.z), a);
+      a = __ffma2_rn(w67, bf16x2_f2(xv.w), a);
       acc[b] = a;
     }
   }
@@ -107,9 +107,9 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
   const uint32_t rounds = (runs + S - 1) / S;
   const uint32_t row0 = uint32_t(chunk * P.rows_per_chunk);
   const uint32_t batch = P.batch;
-  float acc[BMAX];
+  float2 acc[BMAX];
 #pragma unroll
-  for (int b = 0; b < BMAX; ++b) acc[b] = 0.0f;
+  for (int b = 0; b < BMAX; ++b) acc[b] = make_float2(0.0f, 0.0f);
   uint32_t row_local = 0;
   float sc = bf16_bits_to_float(P.scales[row0]);
   uint32_t q = R.off0;
@@ -153,16 +153,16 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
           const float v = bf16_bits_to_float(__ldg(P.patch_val + i));
 #pragma unroll
           for (int b = 0; b < BMAX; ++b)
-            if (b < int(batch)) acc[b] = fmaf(v, bf16_bits_to_float(P.x[size_t(b) * P.cols + col]), acc[b]);
+            if (b < int(batch)) acc[b].x = fmaf(v, bf16_bits_to_float(P.x[size_t(b) * P.cols + col]), acc[b].x);
         }
       }
 #pragma unroll
       for (int b = 0; b < BMAX; ++b) {
-        float v = acc[b];
+        float v = acc[b].x + acc[b].y;
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, d);
         if (lane == 0 && b < int(batch)) P.y[size_t(b) * P.rows + row0 + row_local] = v;
-        acc[b] = 0.0f;
+        acc[b] = make_float2(0.0f, 0.0f);
       }
       ++row_local;
       if (row_local < P.rows_per_chunk && r + 1 < rounds)

@@ -252,3 +252,66 @@ def huff_encode(w_bf16: np.ndarray, threads_per_block: int = 256, lengths=None,
             "eq_huff_encode_host")
     return HostHuff(n, total_bits, threads_per_block, lengths.astype(np.uint8), enc, sm[:n],
                     gaps, block_out)
+
+
+# ------------------------------------------------------------------------------------------------
+# On-disk containers (the compressed weight is the checkpoint): a versioned file holding one
+# coded tensor, loadable without re-encoding.
+#   bytes 0..3   magic: b"EQRT" (rANS), b"EQHF" (DFloat11), b"EQHI" (Huffman-coded integers)
+#   bytes 4..7   format version (little-endian u32, currently 1)
+#   bytes 8..15  header length H (u64); then H bytes of UTF-8 JSON:
+#                {"fields": {scalar fields}, "arrays": [[name, dtype, shape, offset, nbytes], ...]}
+#   arrays at the listed byte offsets (16-byte aligned, little-endian)
+# ------------------------------------------------------------------------------------------------
+import json as _json
+
+_MAGIC = {HostRans: b"EQRT", HostHuff: b"EQHF", HostHuffInt: b"EQHI"}
+_KIND = {v: k for k, v in _MAGIC.items()}
+_ARRAYS = {HostRans: ("freqs", "states", "word_off", "words", "scales", "patch_idx", "patch_val"),
+           HostHuff: ("lengths", "enc_exp", "sign_mant", "gaps", "block_out"),
+           HostHuffInt: ("lengths", "enc", "gaps", "block_out")}
+CONTAINER_VERSION = 1
+
+
+def save(path: str, h) -> None:
+    """Write one coded tensor (HostRans, HostHuff or HostHuffInt) to `path`."""
+    cls = type(h)
+    if cls not in _MAGIC:
+        raise TypeError(f"cannot save {cls.__name__}")
+    names = _ARRAYS[cls]
+    fields = {k: int(v) for k, v in vars(h).items() if k not in names}
+    arrays, blobs, off = [], [], 0
+    for nm in names:
+        a = np.ascontiguousarray(getattr(h, nm))
+        arrays.append([nm, a.dtype.str, list(a.shape), off, a.nbytes])
+        blobs.append((off, a))
+        off = (off + a.nbytes + 15) // 16 * 16
+    head = _json.dumps({"fields": fields, "arrays": arrays}).encode()
+    base = (16 + len(head) + 15) // 16 * 16
+    with open(path, "wb") as f:
+        f.write(_MAGIC[cls] + np.uint32(CONTAINER_VERSION).tobytes()
+                + np.uint64(len(head)).tobytes() + head)
+        f.write(b"\0" * (base - 16 - len(head)))
+        for o, a in blobs:
+            f.seek(base + o)
+            f.write(a.tobytes())
+
+
+def load(path: str):
+    """Read a container written by save()."""
+    with open(path, "rb") as f:
+        raw = f.read()
+    cls = _KIND.get(raw[:4])
+    if cls is None:
+        raise ValueError("not a coded-tensor file")
+    ver = int(np.frombuffer(raw[4:8], np.uint32)[0])
+    if ver != CONTAINER_VERSION:
+        raise ValueError(f"container version {ver}, expected {CONTAINER_VERSION}")
+    hl = int(np.frombuffer(raw[8:16], np.uint64)[0])
+    head = _json.loads(raw[16:16 + hl].decode())
+    base = (16 + hl + 15) // 16 * 16
+    kw = dict(head["fields"])
+    for nm, dt, shape, off, nb in head["arrays"]:
+        kw[nm] = np.frombuffer(raw, dtype=np.dtype(dt), count=nb // np.dtype(dt).itemsize,
+                               offset=base + off).reshape(shape).copy()
+    return cls(**kw)

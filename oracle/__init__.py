@@ -643,3 +643,41 @@ def int8_div_for_entropy(w: np.ndarray, target_bits: float, lo: float = 0.5, hi:
 
 def log2_state_bits(x: int) -> float:
     return math.log2(x)
+
+
+# ----------------------------------------------------------------------------------------------
+# Coded-tensor files (read independently of the library's writer, to check the format):
+# magic (4 bytes) | version u32 | header length u64 | JSON header | arrays at 16-aligned offsets
+# after the header.  Returns the oracle's container for the magic.
+# ----------------------------------------------------------------------------------------------
+
+def load_container(path: str):
+    import json
+    import struct
+    with open(path, "rb") as f:
+        raw = f.read()
+    magic = raw[:4]
+    version, hlen = struct.unpack("<IQ", raw[4:16])
+    if version != 1:
+        raise ValueError("unknown container version")
+    head = json.loads(raw[16:16 + hlen].decode("utf-8"))
+    start = 16 + hlen
+    start += (-start) % 16
+    arr = {}
+    for name, dtype, shape, off, nbytes in head["arrays"]:
+        dt = np.dtype(dtype)
+        arr[name] = np.frombuffer(raw[start + off:start + off + nbytes], dt).reshape(shape).copy()
+    fl = head["fields"]
+    if magic == b"EQRT":
+        return RansTensor(fl["rows"], fl["cols"], fl["symfmt"], fl["prob_bits"],
+                          fl["chunk_symbols"], fl["streams"], fl["run"], arr["freqs"],
+                          arr["states"], arr["word_off"], arr["words"], arr["scales"],
+                          arr["patch_idx"], arr["patch_val"])
+    if magic == b"EQHF":
+        return HuffTensor(fl["n"], 8, fl["threads_per_block"], fl["total_bits"], arr["lengths"],
+                          arr["enc_exp"], arr["sign_mant"], arr["gaps"], arr["block_out"])
+    if magic == b"EQHI":
+        return HuffSymTensor(fl["n"], fl["bits"], fl["threads_per_block"], fl["total_bits"],
+                             arr["lengths"], arr["enc"], arr["gaps"], arr["block_out"],
+                             fl["scale"], fl["zero"])
+    raise ValueError("unknown container magic")

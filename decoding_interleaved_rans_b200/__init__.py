@@ -13,7 +13,7 @@ from ._lib import (EQ_DEV_BAD_CODE, EQ_DEV_CORRUPT_STATE, EQ_DEV_COUNT_MISMATCH,
                    EQ_TABLE_RANS, EQ_TABLE_RANS_PAIR, EXPORTS, EqError, lib)
 from .api import (DeviceHuff, DeviceHuffInt, DeviceRans, bf16_bits, build_tables,  # noqa: F401
                   decode, decode_gemv, histogram_device, huff_bf16_decode, huff_int_decode,
-                  mlp_decode,
+                  mlp_decode, selftest_bounded_wait,
                   mlp_scratch_bytes, new_status, normalize_freqs,
                   quantize_device, rans_encode_device, table_bytes)
 from . import codec  # noqa: F401

@@ -20,7 +20,7 @@ EQ_ABI_VERSION = 2
 
 # every exported function of include/eq.h and include/eq_encode.h
 EXPORTS = ("eq_table_bytes", "eq_build_tables", "eq_decode", "eq_decode_gemv",
-           "eq_huff_bf16_decode", "eq_huff_int_decode", "eq_mlp_scratch_bytes", "eq_mlp_decode", "eq_mlp_decode_noalloc",
+           "eq_huff_bf16_decode", "eq_huff_int_decode", "eq_mlp_scratch_bytes", "eq_mlp_decode", "eq_mlp_decode_noalloc", "eq_selftest_bounded_wait",
            "eq_status_string",
            "eq_abi_version", "eq_quantize_host", "eq_super_weights_host", "eq_quantize_excluding_host",
            "eq_rans_freqs_host", "eq_rans_encode_host", "eq_huff_lengths_host",
@@ -94,6 +94,7 @@ def lib() -> C.CDLL:
                 "eq_mlp_scratch_bytes": (C.c_size_t, [u32, u32]),
                 "eq_mlp_decode": (i32, [p, p, p, p, u32, p, p, C.c_size_t, p, p]),
                 "eq_mlp_decode_noalloc": (i32, [p, p, p, p, u32, p, p, p]),
+                "eq_selftest_bounded_wait": (i32, [p, p]),
                 "eq_status_string": (C.c_char_p, [i32]),
                 "eq_abi_version": (u32, []),
                 "eq_quantize_host": (i32, [p, u32, u32, u32, C.c_float, p, p, u32]),

@@ -277,6 +277,16 @@ def mlp_decode(gate: DeviceRans, up: DeviceRans, down: DeviceRans, x: torch.Tens
     return y, status
 
 
+def selftest_bounded_wait(status=None, stream=None, device="cuda"):
+    """eq_selftest_bounded_wait: a wait for a copy that never lands ends, after about a second,
+    with EQ_DEV_TIMEOUT in the status word."""
+    if status is None:
+        status = new_status(device)
+    L.check(L.lib().eq_selftest_bounded_wait(_ptr(status), _stream(stream)),
+            "eq_selftest_bounded_wait")
+    return status
+
+
 def huff_bf16_decode(h: DeviceHuff, out=None, status=None, stream=None):
     """eq_huff_bf16_decode: DFloat11 -> bf16 [n]."""
     dev = h.enc_exp.device

@@ -261,6 +261,15 @@ eq_status eq_mlp_decode_noalloc(const eq_rans_tensor *gate, const eq_rans_tensor
                                 const eq_rans_tensor *down, const uint16_t *d_x, uint32_t batch,
                                 float *d_y, uint32_t *d_status, void *stream);
 
+/*
+ * Not on the pages: a check of the library's own failure reporting.  The decode kernels wait only
+ * for their own bulk copies, and every such wait gives up after about a second with
+ * EQ_DEV_TIMEOUT in *d_status instead of hanging.  This launches one warp that waits, through
+ * the same bounded wait, for a copy that is never issued: after about a second *d_status has
+ * EQ_DEV_TIMEOUT and the context stays usable.  Nothing is left in flight.
+ */
+eq_status eq_selftest_bounded_wait(uint32_t *d_status, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *eq_status_string(eq_status s);
 

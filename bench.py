@@ -534,6 +534,30 @@ def extra_measurements(eq, dev, stream, flush, peaks, args):
                             f"batch {batch}",
                     "params": params, "ms": sec * 1e3, "params_per_s": params / sec,
                     "kernel": "rans_gemv_kernel x3 + silu_mul_kernel", "launches_per_step": 4})
+    del mats
+    # fused decode + GEMV over the ~2-bit Int8 8192x8192 weight, one row per chunk and 32 streams
+    # (the fused kernel's layout), with the 7-bit pair table and with the 12-bit table
+    wl8 = synth.WORKLOADS["int8_8k"]
+    spec = wl8.tensors[0]
+    sym, sc = eq.codec.quantize(spec.generate(), eq.EQ_SYM_INT8, wl8.int8_div)
+    for pb in (7, 12):
+        m = eq.DeviceRans.upload(
+            eq.codec.rans_encode(sym, sc, eq.EQ_SYM_INT8, spec.cols, 32, 8, prob_bits=pb), dev)
+        for batch in (1, 4, 16):
+            x = torch.randn(batch, m.cols, device=dev).to(torch.bfloat16)
+            y = torch.empty(batch, m.rows, dtype=torch.float32, device=dev)
+            st = eq.new_status(dev)
+            ts = time_steps(lambda: eq.decode_gemv(m, x, y, st, stream), steps, 3, flush, stream)
+            assert int(st.item()) == 0
+            sec = statistics.mean(ts)
+            alg = m.compressed_bytes + x.numel() * 2 + y.numel() * 4
+            out.append({"what": f"fused decode+GEMV, Int8 8192x8192 (~2 bits/param), one row per "
+                                f"chunk, {pb}-bit table, batch {batch}",
+                        "params": m.numel, "ms": sec * 1e3, "params_per_s": m.numel / sec,
+                        "gbs": alg / sec / 1e9, "frac_of_peak": alg / sec / 1e9 / peaks["hbm_gbs"],
+                        "bits_per_param": 8 * m.compressed_bytes / m.numel,
+                        "kernel": "rans_gemv_tc_kernel" if batch >= 8 else "rans_gemv_kernel"})
+        del m
     return out
 
 

@@ -13,7 +13,8 @@
 //     y[b][row] once.  The reduction order is fixed, so results are reproducible.
 // The chunk has one group of 32 streams (streams == 32), so its partial sums never leave the warp.
 // With chunks of several rows, a round (32 * 8 symbols) must not straddle a row, so cols must be a
-// multiple of 256.
+// multiple of 256.  12-, 8- and 7-bit tables take the decode kernel's steps (7-bit: the 128 KiB
+// pair table, one CTA per SM whose warps take chunk after chunk).
 #include <algorithm>
 
 #include "eq_dequant.cuh"
@@ -67,38 +68,60 @@ __device__ __forceinline__ void fma_run(float2 (&acc)[BMAX], uint2 wa, uint2 wb,
   }
 }
 
+// One round (8 steps) of the lane's stream -> its 8 symbols as 4 pairs, the first of each in the
+// low byte.  12-bit tables renormalise after every step, 8-bit ones after every second, 7-bit ones
+// look up two steps at once in the pair table (the steps of the decode kernel).
+template <uint32_t PB>
+__device__ __forceinline__ void round_pairs(uint32_t (&pr)[4], uint32_t &x, bool act,
+                                            const uint32_t *lut, const unsigned char *smem,
+                                            const WordRing &R, uint32_t &q, uint32_t lt) {
+  if constexpr (PB == kRansPairBits) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      pr[k] = rans_pair_step<false>(x, act, lut);
+      rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
+    }
+  } else {
+    uint32_t e[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      e[p] = rans_decode_step<false, PB>(x, act, lut);
+      if (PB == 12 || (p & 1)) rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pr[k] = sym_pair<PB>(e[2 * k], e[2 * k + 1]);
+  }
+}
+
+// Copy the PB-bit slot table (7 bits: the pair table) behind the header into shared memory, only
+// when the header names a table of that size; false otherwise (a table of another size is never
+// read past its end).
+template <uint32_t PB>
+__device__ __forceinline__ bool load_table(uint32_t *lut, const uint32_t *table,
+                                           const RansTableHeader &hdr) {
+  const bool ok = hdr.magic == (PB == kRansPairBits ? kRansPairMagic : kRansMagic) && hdr.prob_bits == PB;
+  constexpr uint32_t kVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
+  const uint4 *src = reinterpret_cast<const uint4 *>(table + sizeof(RansTableHeader) / 4);
+  if (ok)
+    for (uint32_t i = threadIdx.x; i < kVec; i += blockDim.x) reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+  return ok;
+}
+
 // One warp = one chunk of whole rows, 32 streams (one per lane), run length 8.
-template <int FMT, int BMAX>
-__global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ GemvParams P) {
+template <int FMT, int BMAX, uint32_t PB>
+__device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chunk,
+                                               const RansTableHeader &hdr, const uint32_t *lut,
+                                               const unsigned char *smem, WordRing &R,
+                                               uint32_t lane) {
   constexpr uint32_t S = 32;
-  extern __shared__ __align__(128) unsigned char smem[];
-  uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-  unsigned char *rings = smem + rans_lut_bytes(12);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * kRingBytes);
-  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
-  const uint4 *src = reinterpret_cast<const uint4 *>(P.table + sizeof(RansTableHeader) / 4);
-  for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
-    reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
-  WordRing R;
-  ring_init(R, smem, rings, bars, warp, lane);
-  __syncthreads();
-
-  const uint64_t chunk = uint64_t(blockIdx.x) * P.warps + warp;
-  if (chunk >= P.num_chunks) return;
-  uint32_t status = hdr.magic == kRansMagic && hdr.prob_bits == 12 ? 0u : EQ_DEV_CORRUPT_STATE;
+  uint32_t status = 0;
   const bool single = hdr.flags & kRansFlagSingle;
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (hdr.flags & (kRansFlagNaN7F | kRansFlagNaNFF));
   const uint64_t j0 = chunk * uint64_t(P.chunk_symbols);
   const uint32_t n = uint32_t(P.numel - j0 < P.chunk_symbols ? P.numel - j0 : P.chunk_symbols);
   const uint64_t w0 = P.word_off[chunk], w1 = P.word_off[chunk + 1];
-  if (w1 < w0 || w1 - w0 >= (1ull << 30)) status |= EQ_DEV_OVERRUN;
+  if (w1 < w0 || w1 - w0 >= (1ull << 30)) return EQ_DEV_OVERRUN;
   uint32_t x = P.states[chunk * S + lane];
-  if (status) {
-    if (lane == 0) report(P.status, status);
-    return;
-  }
   const uint32_t nwords = uint32_t(w1 - w0);
   if (!single) R.start(P.words, w0, nwords, lane);
 
@@ -124,11 +147,7 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
         status |= EQ_DEV_TIMEOUT;
         break;
       }
-      uint32_t e[8];
-#pragma unroll
-      for (int p = 0; p < 8; ++p) e[p] = rans_step<false>(x, act, lut, smem, R.ring_off, q, lt);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) pr[k] = sym_pair(e[2 * k], e[2 * k + 1]);
+      round_pairs<PB>(pr, x, act, lut, smem, R, q, lt);
       if (q - R.off0 > 2 * nwords) {
         status |= EQ_DEV_OVERRUN;
         break;
@@ -173,7 +192,38 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
     const bool ok = single ? (nwords == 0 && x == kRansL) : (q - R.off0 == 2 * nwords && x == kRansL);
     if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
   }
+  // every copy handed to the engine lands before the ring takes the warp's next chunk
   if (!single) status |= R.drain();
+  return status;
+}
+
+// CTA size bound: 7-bit tables run one CTA of up to 32 warps per SM (the pair table fills most of
+// its shared memory) while the accumulators are few; otherwise up to 16 warps
+__host__ __device__ constexpr uint32_t gemv_max_warps(uint32_t pb, int bmax) {
+  return pb == kRansPairBits && bmax <= 4 ? 32u : 16u;
+}
+
+template <int FMT, int BMAX, uint32_t PB>
+__global__ void __launch_bounds__(32 * gemv_max_warps(PB, BMAX))
+    rans_gemv_kernel(const __grid_constant__ GemvParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
+  unsigned char *rings = smem + rans_lut_bytes(PB);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * kRingBytes);
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
+  const bool table_ok = load_table<PB>(lut, P.table, hdr);
+  WordRing R;
+  ring_init(R, smem, rings, bars, warp, lane);
+  __syncthreads();
+
+  uint64_t chunk = uint64_t(blockIdx.x) * P.warps + warp;
+  if (chunk >= P.num_chunks) return;
+  const uint64_t stride = uint64_t(gridDim.x) * P.warps;
+  uint32_t status = table_ok ? 0u : EQ_DEV_CORRUPT_STATE;
+  for (; chunk < P.num_chunks && !status; chunk += stride)
+    status = gemv_chunk<FMT, BMAX, PB>(P, chunk, hdr, lut, smem, R, lane);
   if (lane == 0) report(P.status, status);
 }
 
@@ -189,10 +239,18 @@ __global__ void __launch_bounds__(512) rans_gemv_kernel(const __grid_constant__ 
 constexpr uint32_t kTcWarps = 16;
 constexpr uint32_t kTcRowBytes = 256 * 2 + 16;  // one tile row, padded against bank conflicts
 constexpr uint32_t kTcTileBytes = kTcWarps * kTcRowBytes;
+constexpr uint32_t kTcRedBytes = kTcWarps * 16 * 16 * 4;  // [16 warps][16 rows][16 b] fp32
+static_assert(2 * kTcTileBytes >= kTcRedBytes, "the reduction buffer fits over the two tiles");
 
-__host__ __device__ constexpr size_t gemv_tc_smem_bytes() {
-  return rans_smem_bytes(kTcWarps) + 2 * kTcTileBytes + kTcWarps * 16 * 16 * 4;
+// A CTA is HALVES independent groups of 16 warps.  With two (7-bit tables, one CTA per SM beside
+// the pair table), each half's reduction buffer lies over its own two tiles, so both fit.
+__host__ __device__ constexpr uint32_t gemv_tc_half_bytes(int halves) {
+  return halves > 1 ? 2 * kTcTileBytes : 2 * kTcTileBytes + kTcRedBytes;
 }
+__host__ __device__ constexpr size_t gemv_tc_smem_bytes(uint32_t pb, int halves) {
+  return rans_smem_bytes(halves * kTcWarps, pb) + halves * gemv_tc_half_bytes(halves);
+}
+static_assert(gemv_tc_smem_bytes(kRansPairBits, 2) <= 227 * 1024, "two halves beside the pair table");
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
@@ -209,166 +267,188 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], uint32_t addr) {
                : "r"(addr));
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(kTcWarps * 32) rans_gemv_tc_kernel(const __grid_constant__ GemvParams P) {
+// Each half of the CTA takes group after group of 16 chunks; every warp of a half runs the same
+// rounds, so its barriers line up.
+template <int FMT, uint32_t PB, int HALVES>
+__global__ void __launch_bounds__(HALVES * kTcWarps * 32)
+    rans_gemv_tc_kernel(const __grid_constant__ GemvParams P) {
   constexpr uint32_t S = 32;
+  constexpr bool kAlias = HALVES > 1;  // the reduction buffer lies over the half's tiles
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-  unsigned char *rings = smem + rans_lut_bytes(12);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + kTcWarps * kRingBytes);
-  unsigned char *tiles = smem + rans_smem_bytes(kTcWarps);          // 2 x [16][264] bf16
-  float *red = reinterpret_cast<float *>(tiles + 2 * kTcTileBytes);  // [16 warps][16 rows][16 b]
+  unsigned char *rings = smem + rans_lut_bytes(PB);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + HALVES * kTcWarps * kRingBytes);
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t half = warp / kTcWarps, hw = warp % kTcWarps;  // hw: this warp's tile row
   const uint32_t grp = lane >> 2, tig = lane & 3;
+  unsigned char *tiles = smem + rans_smem_bytes(HALVES * kTcWarps, PB) +
+                         half * gemv_tc_half_bytes(HALVES);  // 2 x [16][264] bf16
+  float *red = reinterpret_cast<float *>(kAlias ? tiles : tiles + 2 * kTcTileBytes);
+  // the half's own barrier (named barrier 1 + half; barrier 0 is the CTA's)
+  auto half_sync = [&]() {
+    if constexpr (HALVES == 1) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(1u + half), "n"(kTcWarps * 32) : "memory");
+  };
 
   const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
-  const uint4 *src = reinterpret_cast<const uint4 *>(P.table + sizeof(RansTableHeader) / 4);
-  for (uint32_t i = threadIdx.x; i < kRansSlots / 4; i += blockDim.x)
-    reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+  const bool table_ok = load_table<PB>(lut, P.table, hdr);
   WordRing R;
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
-  // every warp runs the same number of rounds (a full chunk's), so the barriers line up;
-  // a warp without a chunk, or whose chunk failed, feeds zeros
-  const uint64_t chunk = uint64_t(blockIdx.x) * kTcWarps + warp;
-  const bool have = chunk < P.num_chunks;
-  uint32_t status = have && (hdr.magic != kRansMagic || hdr.prob_bits != 12) ? EQ_DEV_CORRUPT_STATE : 0u;
   const bool single = hdr.flags & kRansFlagSingle;
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (hdr.flags & (kRansFlagNaN7F | kRansFlagNaNFF));
-  uint32_t x = kRansL, nwords = 0, q = 0, n = 0;
-  bool started = false;
-  if (have && !status) {
-    const uint64_t j0 = chunk * uint64_t(P.chunk_symbols);
-    n = uint32_t(P.numel - j0 < P.chunk_symbols ? P.numel - j0 : P.chunk_symbols);
-    const uint64_t w0 = P.word_off[chunk], w1 = P.word_off[chunk + 1];
-    if (w1 < w0 || w1 - w0 >= (1ull << 30)) status |= EQ_DEV_OVERRUN;
-    nwords = status ? 0u : uint32_t(w1 - w0);
-    x = P.states[chunk * S + lane];
-    if (!status && !single) {
-      R.start(P.words, w0, nwords, lane);
-      q = R.off0;
-      started = true;
-    }
-  }
-  bool live = have && !status && !single;  // decoding from the stream
   const uint32_t lt = lanemask_lt();
-  const uint32_t runs = n / 8;
   const uint32_t rounds = P.chunk_symbols / 256;  // the same for every warp of the launch
   const uint32_t rpr = P.rows_per_chunk > 1 ? P.rounds_per_row : rounds;
-  const uint32_t row0 = uint32_t(chunk * P.rows_per_chunk);
   const uint32_t ntiles = (P.batch + 7) / 8;
-  float c[2][4] = {};
-  uint32_t row_local = 0;
-  float sc = have && !status ? bf16_bits_to_float(P.scales[row0]) : 0.0f;
   const uint32_t tiles_addr = smem_addr(tiles);
+  const uint64_t ngroups = (P.num_chunks + kTcWarps - 1) / kTcWarps;
+  // sticky: a warp whose chunk failed feeds zeros from then on (the launch reports the failure)
+  uint32_t status = 0;
 
-  for (uint32_t r = 0; r < rounds; ++r) {
-    const bool act = have && !status && r * S + lane < runs;
-    uint32_t pr[4] = {0u, 0u, 0u, 0u};
-    if (live) {
-      if (!R.round_wait(q)) {
-        status |= EQ_DEV_TIMEOUT;
-        live = false;
-      } else {
-        uint32_t e[8];
-#pragma unroll
-        for (int p = 0; p < 8; ++p) e[p] = rans_step<false>(x, act, lut, smem, R.ring_off, q, lt);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) pr[k] = sym_pair(e[2 * k], e[2 * k + 1]);
-        if (q - R.off0 > 2 * nwords) {
-          status |= EQ_DEV_OVERRUN;
+  for (uint64_t cg = uint64_t(blockIdx.x) * HALVES + half; cg < ngroups; cg += uint64_t(gridDim.x) * HALVES) {
+    // a warp without a chunk, or whose chunk failed, feeds zeros
+    const uint64_t chunk = cg * kTcWarps + hw;
+    const bool have = chunk < P.num_chunks;
+    if (have && !table_ok) status |= EQ_DEV_CORRUPT_STATE;
+    uint32_t x = kRansL, nwords = 0, q = 0, n = 0;
+    bool started = false;
+    if (have && !status) {
+      const uint64_t j0 = chunk * uint64_t(P.chunk_symbols);
+      n = uint32_t(P.numel - j0 < P.chunk_symbols ? P.numel - j0 : P.chunk_symbols);
+      const uint64_t w0 = P.word_off[chunk], w1 = P.word_off[chunk + 1];
+      if (w1 < w0 || w1 - w0 >= (1ull << 30)) status |= EQ_DEV_OVERRUN;
+      nwords = status ? 0u : uint32_t(w1 - w0);
+      x = P.states[chunk * S + lane];
+      if (!status && !single) {
+        R.start(P.words, w0, nwords, lane);
+        q = R.off0;
+        started = true;
+      }
+    }
+    const bool valid = have && !status;  // this chunk decodes (status may still turn nonzero)
+    bool live = valid && !single;        // decoding from the stream
+    const uint32_t runs = n / 8;
+    const uint32_t row0 = uint32_t(chunk * P.rows_per_chunk);
+    float c[2][4] = {};
+    uint32_t row_local = 0;
+    float sc = valid ? bf16_bits_to_float(P.scales[row0]) : 0.0f;
+
+    for (uint32_t r = 0; r < rounds; ++r) {
+      const bool act = valid && !status && r * S + lane < runs;
+      uint32_t pr[4] = {0u, 0u, 0u, 0u};
+      if (live) {
+        if (!R.round_wait(q)) {
+          status |= EQ_DEV_TIMEOUT;
           live = false;
         } else {
-          R.round_refill(q, lane);
-        }
-      }
-    } else if (single) {
-      pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
-    }
-    // this warp's 256 weights of the round -> tile row `warp`
-    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
-    if (act && !status) {
-      wv.x = dequant2<FMT>(pr[0], sc, nan_codes);
-      wv.y = dequant2<FMT>(pr[1], sc, nan_codes);
-      wv.z = dequant2<FMT>(pr[2], sc, nan_codes);
-      wv.w = dequant2<FMT>(pr[3], sc, nan_codes);
-    }
-    unsigned char *tile = tiles + (r & 1) * kTcTileBytes;
-    *reinterpret_cast<uint4 *>(tile + warp * kTcRowBytes + lane * 16) = wv;
-    __syncthreads();
-    // warp w multiplies tile columns [16 w, 16 w + 16) by x[:, col0 + 16 w ...]
-    {
-      uint32_t a[4];
-      const uint32_t arow = lane & 15, acol = (lane >> 4) * 8 + warp * 16;
-      ldmatrix_x4(a, tiles_addr + (r & 1) * kTcTileBytes + arow * kTcRowBytes + acol * 2);
-      const uint32_t col0 = (r % rpr) * 256 + warp * 16 + 2 * tig;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        if (uint32_t(nt) < ntiles) {
-          const uint32_t b = nt * 8 + grp;
-          uint32_t b0 = 0, b1 = 0;
-          if (b < P.batch) {
-            const uint16_t *xr = P.x + size_t(b) * P.cols + col0;
-            b0 = __ldg(reinterpret_cast<const uint32_t *>(xr));
-            b1 = __ldg(reinterpret_cast<const uint32_t *>(xr + 8));
+          round_pairs<PB>(pr, x, act, lut, smem, R, q, lt);
+          if (q - R.off0 > 2 * nwords) {
+            status |= EQ_DEV_OVERRUN;
+            live = false;
+          } else {
+            R.round_refill(q, lane);
           }
-          mma_bf16_16816(c[nt], a, b0, b1);
         }
+      } else if (single) {
+        pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
       }
-    }
-    // end of a weight row: sum the 16 warps' partial products in a fixed order
-    if ((r + 1) % rpr == 0) {
-      float *mine = red + warp * 256;
+      // this warp's 256 weights of the round -> tile row hw
+      uint4 wv = make_uint4(0u, 0u, 0u, 0u);
+      if (act && !status) {
+        wv.x = dequant2<FMT>(pr[0], sc, nan_codes);
+        wv.y = dequant2<FMT>(pr[1], sc, nan_codes);
+        wv.z = dequant2<FMT>(pr[2], sc, nan_codes);
+        wv.w = dequant2<FMT>(pr[3], sc, nan_codes);
+      }
+      unsigned char *tile = tiles + (r & 1) * kTcTileBytes;
+      *reinterpret_cast<uint4 *>(tile + hw * kTcRowBytes + lane * 16) = wv;
+      half_sync();
+      // warp w multiplies tile columns [16 w, 16 w + 16) by x[:, col0 + 16 w ...]
+      {
+        uint32_t a[4];
+        const uint32_t arow = lane & 15, acol = (lane >> 4) * 8 + hw * 16;
+        ldmatrix_x4(a, tiles_addr + (r & 1) * kTcTileBytes + arow * kTcRowBytes + acol * 2);
+        const uint32_t col0 = (r % rpr) * 256 + hw * 16 + 2 * tig;
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        mine[grp * 16 + nt * 8 + 2 * tig] = c[nt][0];
-        mine[grp * 16 + nt * 8 + 2 * tig + 1] = c[nt][1];
-        mine[(grp + 8) * 16 + nt * 8 + 2 * tig] = c[nt][2];
-        mine[(grp + 8) * 16 + nt * 8 + 2 * tig + 1] = c[nt][3];
-        c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.0f;
-      }
-      __syncthreads();
-      if (threadIdx.x < 256) {
-        const uint32_t wr = threadIdx.x >> 4, b = threadIdx.x & 15;  // tile row = warp wr
-        float v = 0.0f;
-        for (uint32_t w = 0; w < kTcWarps; ++w) v += red[w * 256 + wr * 16 + b];
-        const uint64_t ch = uint64_t(blockIdx.x) * kTcWarps + wr;
-        const uint64_t row = ch * P.rows_per_chunk + (r / rpr);
-        if (P.n_patch && ch < P.num_chunks && b < P.batch && row < P.rows) {  // super weights
-          const uint64_t rs = row * P.cols;
-          const uint64_t hi = patch_lower_bound(P.patch_idx, P.n_patch, rs + P.cols);
-          for (uint64_t i = patch_lower_bound(P.patch_idx, P.n_patch, rs); i < hi; ++i)
-            v = fmaf(bf16_bits_to_float(__ldg(P.patch_val + i)),
-                     bf16_bits_to_float(P.x[size_t(b) * P.cols + (__ldg(P.patch_idx + i) - rs)]), v);
+        for (int nt = 0; nt < 2; ++nt) {
+          if (uint32_t(nt) < ntiles) {
+            const uint32_t b = nt * 8 + grp;
+            uint32_t b0 = 0, b1 = 0;
+            if (b < P.batch) {
+              const uint16_t *xr = P.x + size_t(b) * P.cols + col0;
+              b0 = __ldg(reinterpret_cast<const uint32_t *>(xr));
+              b1 = __ldg(reinterpret_cast<const uint32_t *>(xr + 8));
+            }
+            mma_bf16_16816(c[nt], a, b0, b1);
+          }
         }
-        if (ch < P.num_chunks && b < P.batch && row < P.rows) P.y[size_t(b) * P.rows + row] = v;
       }
-      ++row_local;
-      if (have && !status && row_local < P.rows_per_chunk)
-        sc = bf16_bits_to_float(P.scales[row0 + row_local]);
+      // end of a weight row: sum the 16 warps' partial products in a fixed order
+      if ((r + 1) % rpr == 0) {
+        if constexpr (kAlias) half_sync();  // every warp is done with the tiles
+        float *mine = red + hw * 256;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          mine[grp * 16 + nt * 8 + 2 * tig] = c[nt][0];
+          mine[grp * 16 + nt * 8 + 2 * tig + 1] = c[nt][1];
+          mine[(grp + 8) * 16 + nt * 8 + 2 * tig] = c[nt][2];
+          mine[(grp + 8) * 16 + nt * 8 + 2 * tig + 1] = c[nt][3];
+          c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.0f;
+        }
+        half_sync();
+        const uint32_t th = threadIdx.x - half * kTcWarps * 32;
+        if (th < 256) {
+          const uint32_t wr = th >> 4, b = th & 15;  // tile row wr
+          float v = 0.0f;
+          for (uint32_t w = 0; w < kTcWarps; ++w) v += red[w * 256 + wr * 16 + b];
+          const uint64_t ch = cg * kTcWarps + wr;
+          const uint64_t row = ch * P.rows_per_chunk + (r / rpr);
+          if (P.n_patch && ch < P.num_chunks && b < P.batch && row < P.rows) {  // super weights
+            const uint64_t rs = row * P.cols;
+            const uint64_t hi = patch_lower_bound(P.patch_idx, P.n_patch, rs + P.cols);
+            for (uint64_t i = patch_lower_bound(P.patch_idx, P.n_patch, rs); i < hi; ++i)
+              v = fmaf(bf16_bits_to_float(__ldg(P.patch_val + i)),
+                       bf16_bits_to_float(P.x[size_t(b) * P.cols + (__ldg(P.patch_idx + i) - rs)]), v);
+          }
+          if (ch < P.num_chunks && b < P.batch && row < P.rows) P.y[size_t(b) * P.rows + row] = v;
+        }
+        if constexpr (kAlias) half_sync();  // the sums are read before the tiles are rewritten
+        ++row_local;
+        if (valid && !status && row_local < P.rows_per_chunk)
+          sc = bf16_bits_to_float(P.scales[row0 + row_local]);
+      }
     }
+    if (valid && !status) {
+      const bool ok = single ? (nwords == 0 && x == kRansL) : (q - R.off0 == 2 * nwords && x == kRansL);
+      if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
+    }
+    // every copy handed to the engine lands before the ring takes the next chunk
+    if (started) status |= R.drain();
   }
-  if (have && !status) {
-    const bool ok = single ? (nwords == 0 && x == kRansL) : (q - R.off0 == 2 * nwords && x == kRansL);
-    if (!__all_sync(0xFFFFFFFFu, ok)) status |= EQ_DEV_CORRUPT_STATE;
-  }
-  if (started) status |= R.drain();
   if (lane == 0) report(P.status, status);
 }
 
 using GemvFn = void (*)(GemvParams);
 
-template <int FMT>
-static GemvFn pick_b(uint32_t batch) {
-  if (batch <= 1) return rans_gemv_kernel<FMT, 1>;
-  if (batch <= 2) return rans_gemv_kernel<FMT, 2>;
-  if (batch <= 4) return rans_gemv_kernel<FMT, 4>;
-  if (batch <= 8) return rans_gemv_kernel<FMT, 8>;
-  return rans_gemv_kernel<FMT, 16>;
+template <int FMT, uint32_t PB>
+static GemvFn pick_b(uint32_t batch, bool tc) {
+  if (tc) return rans_gemv_tc_kernel<FMT, PB, PB == kRansPairBits ? 2 : 1>;
+  if (batch <= 1) return rans_gemv_kernel<FMT, 1, PB>;
+  if (batch <= 2) return rans_gemv_kernel<FMT, 2, PB>;
+  if (batch <= 4) return rans_gemv_kernel<FMT, 4, PB>;
+  if (batch <= 8) return rans_gemv_kernel<FMT, 8, PB>;
+  return rans_gemv_kernel<FMT, 16, PB>;
 }
 
-static bool g_gemv_attr[64][2][6];
+template <int FMT>
+static GemvFn pick_pb(uint32_t pb, uint32_t batch, bool tc) {
+  return pb == 12 ? pick_b<FMT, 12>(batch, tc) : pb == 8 ? pick_b<FMT, 8>(batch, tc)
+                                                         : pick_b<FMT, kRansPairBits>(batch, tc);
+}
+
+static bool g_gemv_attr[64][2][3][6];  // device, symfmt, table (12 / 8 / 7 bits), kernel instance
 
 }  // namespace eq
 
@@ -382,28 +462,43 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   if (batch < 1 || batch > 16) return EQ_ERR_ARG;
   if (t->rows == 0 || t->cols == 0) return EQ_OK;
   if (!d_x || !d_y || !aligned(d_x, 16) || !aligned(d_y, 4)) return EQ_ERR_ARG;
-  if (t->prob_bits != 12 || t->run != 8 || t->streams != 32 || t->chunk_symbols % t->cols)
-    return EQ_ERR_UNSUPPORTED;
+  if (t->run != 8 || t->streams != 32 || t->chunk_symbols % t->cols) return EQ_ERR_UNSUPPORTED;
   const uint32_t rpc = t->chunk_symbols / t->cols;
   if (rpc > 1 && t->cols % (t->streams * 8)) return EQ_ERR_UNSUPPORTED;
   // batch >= 8 on the tensor cores when a round never straddles a chunk's 256-column tiles
   const bool tc = batch >= 8 && t->chunk_symbols % 256 == 0;
-  GemvFn fn = tc ? (t->symfmt == EQ_SYM_E4M3 ? rans_gemv_tc_kernel<EQ_SYM_E4M3> : rans_gemv_tc_kernel<EQ_SYM_INT8>)
-                 : (t->symfmt == EQ_SYM_E4M3 ? pick_b<EQ_SYM_E4M3>(batch) : pick_b<EQ_SYM_INT8>(batch));
+  const uint32_t pb = t->prob_bits;
+  const bool pair = pb == kRansPairBits;
+  GemvFn fn = t->symfmt == EQ_SYM_E4M3 ? pick_pb<EQ_SYM_E4M3>(pb, batch, tc) : pick_pb<EQ_SYM_INT8>(pb, batch, tc);
   const uint64_t sms = uint64_t(device_sm_count());
-  uint32_t warps = 16;
-  if (!tc)
+  const int bmax = batch <= 1 ? 1 : batch <= 2 ? 2 : batch <= 4 ? 4 : batch <= 8 ? 8 : 16;
+  uint32_t warps, max_warps;
+  uint64_t ctas;
+  if (tc) {
+    // 7-bit tables: one CTA per SM, two halves of 16 warps, each taking group after group
+    warps = max_warps = pair ? 2 * kTcWarps : kTcWarps;
+    ctas = (t->num_chunks + warps - 1) / warps;
+    if (pair) ctas = std::min<uint64_t>(ctas, sms);
+  } else if (pair) {
+    // one CTA per SM holds the pair table; enough warps that the SMs' CTAs take every chunk
+    // about once (more chunks: the warps loop)
+    max_warps = gemv_max_warps(pb, bmax);
+    warps = uint32_t(std::min<uint64_t>(max_warps, std::max<uint64_t>(1, (t->num_chunks + sms - 1) / sms)));
+    ctas = std::min<uint64_t>(sms, (t->num_chunks + warps - 1) / warps);
+  } else {
+    warps = max_warps = 16;
     while (warps > 1 && (t->num_chunks + warps - 1) / warps < 4 * sms) warps >>= 1;
-  const uint64_t ctas = (t->num_chunks + warps - 1) / warps;
+    ctas = (t->num_chunks + warps - 1) / warps;
+  }
   if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  // one flag per kernel instance that pick_b / the tensor-core choice can return
-  const int bi = tc ? 5 : batch <= 1 ? 0 : batch <= 2 ? 1 : batch <= 4 ? 2 : batch <= 8 ? 3 : 4;
-  bool &attr = g_gemv_attr[dev][t->symfmt - 1][bi];
+  // one flag per kernel instance that pick_pb can return
+  const int bi = tc ? 5 : bmax == 1 ? 0 : bmax == 2 ? 1 : bmax == 4 ? 2 : bmax == 8 ? 3 : 4;
+  bool &attr = g_gemv_attr[dev][t->symfmt - 1][pb == 12 ? 0 : pb == 8 ? 1 : 2][bi];
   if (!attr) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(tc ? gemv_tc_smem_bytes() : rans_smem_bytes(16))) != cudaSuccess)
+                             int(tc ? gemv_tc_smem_bytes(pb, pair ? 2 : 1) : rans_smem_bytes(max_warps, pb))) != cudaSuccess)
       return EQ_ERR_CUDA;
     attr = true;
   }
@@ -428,7 +523,7 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   P.rounds_per_row = rpc > 1 ? t->cols / (t->streams * 8) : 0;
   P.batch = batch;
   P.warps = warps;
-  fn<<<uint32_t(ctas), 32 * warps, tc ? gemv_tc_smem_bytes() : rans_smem_bytes(warps),
+  fn<<<uint32_t(ctas), 32 * warps, tc ? gemv_tc_smem_bytes(pb, pair ? 2 : 1) : rans_smem_bytes(warps, pb),
        static_cast<cudaStream_t>(stream)>>>(P);
   return cuda_status(cudaGetLastError());
 }

@@ -201,8 +201,9 @@ eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uint16_t *cons
  * x: bf16 [batch][cols], 16-byte aligned.  y: fp32 [batch][rows].  batch 1..16; for batch >= 8
  * (and chunk_symbols % 256 == 0) the product of each 16-row x 256-column decoded tile with x runs
  * on the tensor cores (mma, bf16 in, fp32 accumulate).
- * Requires prob_bits == 12, run == 8, streams == 32 (one warp owns a chunk, so its sums never
- * leave the warp)
+ * Takes 12-, 8- and 7-bit tables (the decode steps of eq_decode; a 7-bit table's pair table fills
+ * most of an SM's shared memory, so one CTA per SM takes chunk after chunk).
+ * Requires run == 8, streams == 32 (one warp owns a chunk, so its sums never leave the warp)
  * and whole rows per chunk (chunk_symbols a multiple of cols); a chunk of several rows also needs
  * cols % 256 == 0, so that one decode round never straddles two rows.  Otherwise
  * EQ_ERR_UNSUPPORTED.

@@ -197,14 +197,20 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
   return status;
 }
 
-// CTA size bound: 7-bit tables run one CTA of up to 32 warps per SM (the pair table fills most of
-// its shared memory) while the accumulators are few; otherwise up to 16 warps
+// CTA shapes.  7-bit tables: one CTA of up to 32 warps per SM (the pair table fills most of its
+// shared memory) while the accumulators are few, else 16.  Other tables with few accumulators:
+// CTAs of 4 warps, 9 per SM (at most 56 registers a thread), so that 36 warps share an SM and a
+// tensor of long rows (5120 chunks of 13824 weights) runs in one wave instead of a full wave and a
+// tail; else up to 16 warps.
 __host__ __device__ constexpr uint32_t gemv_max_warps(uint32_t pb, int bmax) {
-  return pb == kRansPairBits && bmax <= 4 ? 32u : 16u;
+  return pb == kRansPairBits ? (bmax <= 4 ? 32u : 16u) : (bmax <= 4 ? 4u : 16u);
+}
+__host__ __device__ constexpr uint32_t gemv_min_ctas(uint32_t pb, int bmax) {
+  return pb != kRansPairBits && bmax <= 4 ? 9u : 1u;
 }
 
 template <int FMT, int BMAX, uint32_t PB>
-__global__ void __launch_bounds__(32 * gemv_max_warps(PB, BMAX))
+__global__ void __launch_bounds__(32 * gemv_max_warps(PB, BMAX), gemv_min_ctas(PB, BMAX))
     rans_gemv_kernel(const __grid_constant__ GemvParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
@@ -486,7 +492,7 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
     warps = uint32_t(std::min<uint64_t>(max_warps, std::max<uint64_t>(1, (t->num_chunks + sms - 1) / sms)));
     ctas = std::min<uint64_t>(sms, (t->num_chunks + warps - 1) / warps);
   } else {
-    warps = max_warps = 16;
+    warps = max_warps = gemv_max_warps(pb, bmax);
     while (warps > 1 && (t->num_chunks + warps - 1) / warps < 4 * sms) warps >>= 1;
     ctas = (t->num_chunks + warps - 1) / warps;
   }

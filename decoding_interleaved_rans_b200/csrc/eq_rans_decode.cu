@@ -158,7 +158,34 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   // ring checks once per round (12-bit: up to 256 words a round), or once per two rounds
   // (8-bit: up to 128 words a round); round_wait covers 256 words and one more
   constexpr uint32_t kRoundsPerCheck = PB == 12 ? 1 : 2;
-  for (uint32_t r = 0; r < rounds; r += kRoundsPerCheck) {
+  // the rounds in which every lane of the group holds a run, with no per-round tests
+  uint32_t r0 = 0;
+  for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
+    if (!R.round_wait(q)) {
+      status |= EQ_DEV_TIMEOUT;
+      break;
+    }
+#pragma unroll
+    for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
+      decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
+      out += step;
+      col += step;
+      if (col >= cols) {
+        do {
+          col -= cols;
+          ++row;
+        } while (col >= cols);
+        if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
+      }
+    }
+    if (q - R.off0 > 2 * nwords) {
+      status |= EQ_DEV_OVERRUN;
+      break;
+    }
+    R.round_refill(q, lane);
+  }
+  // the rest (lanes without a run from some round on)
+  for (uint32_t r = r0; r < rounds && !status; r += kRoundsPerCheck) {
     if (!R.round_wait(q)) {
       status |= EQ_DEV_TIMEOUT;
       break;

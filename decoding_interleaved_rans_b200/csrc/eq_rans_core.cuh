@@ -91,6 +91,16 @@ struct WordRing {
     if (q >= refill_at) refill(q, lane);
   }
 
+  // The offset below which the per-round checks have nothing to do: no wait (the landed bytes
+  // cover q plus a round's worth and one word), no refill (no slot used up) and no overrun
+  // (q_end: one past the substream's last byte).
+  __device__ __forceinline__ uint32_t quiet_until(uint32_t q_end) const {
+    constexpr uint32_t kAhead = 2 * kRoundWords + 2;
+    uint32_t t = ready >= nseg ? 0xFFFFFFFFu : (ready_end >= kAhead ? ready_end - kAhead + 1 : 0u);
+    t = min(t, refill_at);
+    return min(t, q_end + 1);
+  }
+
   // hand out the slots of segments lying wholly below offset q
   __device__ __forceinline__ void refill(uint32_t q, uint32_t lane) {
     const uint32_t cur = q / kSegBytes;

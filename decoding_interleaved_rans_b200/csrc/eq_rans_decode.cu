@@ -158,12 +158,24 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   // ring checks once per round (12-bit: up to 256 words a round), or once per two rounds
   // (8-bit: up to 128 words a round); round_wait covers 256 words and one more
   constexpr uint32_t kRoundsPerCheck = PB == 12 ? 1 : 2;
-  // the rounds in which every lane of the group holds a run, with no per-round tests
+  // The rounds in which every lane of the group holds a run, with no per-round tests.  The ring
+  // work (overrun check, refill, wait) runs only once q reaches q_next; refill comes before the
+  // wait, so every segment a wait needs has been handed to the copy engine.
+  const uint32_t q_end = R.off0 + 2 * nwords;
+  uint32_t q_next = 0;
   uint32_t r0 = 0;
   for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
-    if (!R.round_wait(q)) {
-      status |= EQ_DEV_TIMEOUT;
-      break;
+    if (q >= q_next) {
+      if (q > q_end) {
+        status |= EQ_DEV_OVERRUN;
+        break;
+      }
+      R.round_refill(q, lane);
+      if (!R.round_wait(q)) {
+        status |= EQ_DEV_TIMEOUT;
+        break;
+      }
+      q_next = R.quiet_until(q_end);
     }
 #pragma unroll
     for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
@@ -178,11 +190,10 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
         if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
       }
     }
-    if (q - R.off0 > 2 * nwords) {
-      status |= EQ_DEV_OVERRUN;
-      break;
-    }
-    R.round_refill(q, lane);
+  }
+  if (!status) {  // the general loop below waits first: hand out the used-up slots
+    if (q > q_end) status |= EQ_DEV_OVERRUN;
+    else R.round_refill(q, lane);
   }
   // the rest (lanes without a run from some round on)
   for (uint32_t r = r0; r < rounds && !status; r += kRoundsPerCheck) {

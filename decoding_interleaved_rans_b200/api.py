@@ -45,9 +45,12 @@ def new_status(device) -> torch.Tensor:
     return torch.zeros(1, dtype=torch.int32, device=device)
 
 
-def rans_table_kind(prob_bits: int) -> int:
-    """7-bit tables decode through a pair table, the others through a slot table."""
-    return L.EQ_TABLE_RANS_PAIR if prob_bits == 7 else L.EQ_TABLE_RANS
+def rans_table_kind(prob_bits: int, symfmt: int) -> int:
+    """7-bit tables decode through a pair table carrying the symbols' values (one kind per symbol
+    format), the others through a slot table."""
+    if prob_bits != 7:
+        return L.EQ_TABLE_RANS
+    return L.EQ_TABLE_RANS_PAIR_E4M3 if symfmt == L.EQ_SYM_E4M3 else L.EQ_TABLE_RANS_PAIR_INT8
 
 
 @dataclass
@@ -114,9 +117,9 @@ class DeviceRans:
                 _dev(np.asarray(h.word_off, np.uint64), device, np.int64),
                 _dev(words, device, np.int16),
                 _dev(np.asarray(h.scales, np.uint16), device, np.int16),
-                torch.empty(table_bytes(rans_table_kind(int(h.prob_bits))), dtype=torch.uint8,
-                            device=device))
-        build_tables(rans_table_kind(t.prob_bits), h.freqs, t.prob_bits, t.tables, stream)
+                torch.empty(table_bytes(rans_table_kind(int(h.prob_bits), int(h.symfmt))),
+                            dtype=torch.uint8, device=device))
+        build_tables(rans_table_kind(t.prob_bits, t.symfmt), h.freqs, t.prob_bits, t.tables, stream)
         pidx = getattr(h, "patch_idx", None)
         if pidx is not None and len(pidx):
             t.patch_idx = _dev(np.asarray(pidx, np.uint64), device, np.int64)
@@ -364,7 +367,7 @@ def rans_encode_device(sym: torch.Tensor, scales: torch.Tensor, symfmt: int, chu
                                           _stream(stream)), "eq_rans_encode_device")
     t = DeviceRans(rows, cols, symfmt, prob_bits, chunk_symbols, streams, run, nchunks,
                    states[:nchunks * streams] if nchunks else states, word_off, words,
-                   scales, torch.empty(table_bytes(rans_table_kind(prob_bits)),
+                   scales, torch.empty(table_bytes(rans_table_kind(prob_bits, symfmt)),
                                        dtype=torch.uint8, device=dev))
-    build_tables(rans_table_kind(prob_bits), freqs, prob_bits, t.tables, stream)
+    build_tables(rans_table_kind(prob_bits, symfmt), freqs, prob_bits, t.tables, stream)
     return t

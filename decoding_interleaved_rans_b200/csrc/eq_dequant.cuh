@@ -70,6 +70,35 @@ __device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, b
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// a symbol's value as bf16 bits, exactly (E4M3: at most 4 significant bits, exponent within
+// bf16's range; Int8: at most 8 bits); the E4M3 NaN codes give the quiet NaN with their sign
+__device__ __forceinline__ uint32_t symbol_bf16(uint32_t s, uint32_t symfmt) {
+  if (symfmt == EQ_SYM_E4M3) {
+    if ((s & 0x7Fu) == 0x7Fu) return 0x7FC0u | ((s & 0x80u) << 8);
+    return __float_as_uint(sym2_value<EQ_SYM_E4M3>(s).x) >> 16;
+  }
+  return __float_as_uint(float(int32_t(s << 24) >> 24)) >> 16;
+}
+
+// A pair of symbol values from a 7-bit pair table (bf16x2, exact) times the row scale: one
+// bf16x2 multiply, whose single round-to-nearest-even of the exact product is bf16_rne(value *
+// scale).  sc2: the scale's bf16 bits in both halves.  Halves holding an E4M3 NaN code's value
+// (the quiet NaN with the code's sign) pass through unscaled when nan_codes.
+__device__ __forceinline__ uint32_t pair_dequant(uint32_t vals, uint32_t sc2, bool nan_codes) {
+  uint32_t o;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(o) : "r"(vals), "r"(sc2));
+  if (nan_codes) {
+    if ((vals & 0x7FFFu) > 0x7F80u) o = (o & 0xFFFF0000u) | (vals & 0xFFFFu);
+    if ((vals & 0x7FFF0000u) > 0x7F800000u) o = (o & 0x0000FFFFu) | (vals & 0xFFFF0000u);
+  }
+  return o;
+}
+
+// the bf16 bits of a scale held as fp32 (converted exactly from bf16), in both halves
+__device__ __forceinline__ uint32_t scale_bf16x2(float sc) {
+  return __byte_perm(__float_as_uint(sc), 0u, 0x3232u);
+}
+
 // one symbol -> bf16 bits
 template <int FMT>
 __device__ __forceinline__ uint16_t dequant1(uint32_t sym, float scale) {

@@ -31,17 +31,25 @@ struct RansTableHeader {
   uint32_t prob_bits;    // 12 or 8
 };
 constexpr uint32_t kRansMagic = 0x52414E53u;  // "RANS"
-// rANS pair table of a 7-bit frequency table (EQ_TABLE_RANS_PAIR): two decode steps at once.
-// Entry i (i = x mod 2^14, the state's low 14 bits) for slot1 = i mod 128, L = i >> 7:
+// rANS pair table of a 7-bit frequency table (EQ_TABLE_RANS_PAIR_E4M3 / _INT8): two decode
+// steps at once.  Entry i (i = x mod 2^14, the state's low 14 bits) for slot1 = i mod 128,
+// L = i >> 7:
 //   s1 = symbol of slot1, v = f1 * L + (slot1 - cum1), slot2 = v mod 128, s2 = its symbol,
 //   F = f1 * f2, B = f2 * (v >> 7) + (slot2 - cum2);
-//   word 0 = F | s1 << 16 | s2 << 24, word 1 = B.
+//   word 0 = value(s1) | value(s2) << 16, each the symbol's value as bf16 bits (exact: an Int8
+//            value has at most 8 significant bits, an E4M3 one 4 within bf16's exponent range;
+//            the E4M3 NaN codes give 0x7FC0 / 0xFFC0),
+//   word 1 = F << 14 | B.
 // Then the two steps x -> x1 -> x2 are x2 = F * (x >> 14) + B: with x >> 7 = 128 H + L
 // (H = x >> 14), x1 = f1 (x >> 7) + slot1 - cum1 = 128 f1 H + v, so x1 mod 128 = slot2 and
-// x1 >> 7 = f1 H + (v >> 7).  F and B stay below 2^14.
+// x1 >> 7 = f1 H + (v >> 7).  B < F < 2^14 unless one symbol owns all 128 slots (F = 2^14), a
+// table the header flags and the decoders never look up.  Dequantisation of the pair is one
+// bf16x2 multiply of word 0 by the row scale: the product of two bf16 values is exact in fp32,
+// so the multiply's one round-to-nearest-even gives bf16_rne(value * scale).
 constexpr uint32_t kRansPairBits = 7;
 constexpr uint32_t kRansPairEntries = 1u << (2 * kRansPairBits);
-constexpr uint32_t kRansPairMagic = 0x52505237u;  // "RPR7"
+constexpr uint32_t kRansPairMagicE4M3 = 0x52504537u;  // "RPE7"
+constexpr uint32_t kRansPairMagicInt8 = 0x52504937u;  // "RPI7"
 constexpr size_t kRansPairTableBytes = 16 + size_t(kRansPairEntries) * 8;
 constexpr uint32_t kRansFlagNaN7F = 1u;       // frequency of byte 0x7F is nonzero
 constexpr uint32_t kRansFlagNaNFF = 2u;       // frequency of byte 0xFF is nonzero

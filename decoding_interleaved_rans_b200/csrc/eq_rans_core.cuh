@@ -176,7 +176,7 @@ __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, cons
 }
 
 // Two decode steps of a 7-bit stream with one pair-table lookup (layout in eq_internal.cuh):
-// x2 = F * (x >> 14) + B.  Returns the two symbols as a 16-bit pair (the first in the low byte).
+// x2 = F * (x >> 14) + B.  Returns the two symbols' values as bf16x2 (the first in the low half).
 template <bool FULL>
 __device__ __forceinline__ uint32_t rans_pair_step(uint32_t &x, bool act, const uint32_t *lut) {
   const uint32_t base = uint32_t(__cvta_generic_to_shared(lut));
@@ -188,12 +188,21 @@ __device__ __forceinline__ uint32_t rans_pair_step(uint32_t &x, bool act, const 
       "add.u32 a, a, %3;\n\t"
       "shr.u32 xs, %2, 14;\n\t"
       "ld.shared.v2.u32 {%1, w1}, [a];\n\t"
-      "and.b32 f, %1, 65535;\n\t"
+      "shr.u32 f, w1, 14;\n\t"
+      "and.b32 w1, w1, 16383;\n\t"
       "mad.lo.u32 %0, f, xs, w1;\n\t}"
       : "=r"(nx), "=r"(w0)
       : "r"(x), "r"(base));
   if (FULL || act) x = nx;
-  return w0 >> 16;
+  return w0;
+}
+
+// the header magic of a PB-bit table for symbols of format FMT (7-bit pair tables carry the
+// symbols' values, so they are specific to the format)
+template <int FMT, uint32_t PB>
+__device__ __forceinline__ constexpr uint32_t rans_table_magic() {
+  return PB != kRansPairBits ? kRansMagic
+                             : FMT == EQ_SYM_E4M3 ? kRansPairMagicE4M3 : kRansPairMagicInt8;
 }
 
 // the symbol byte of a PB-bit entry

@@ -65,16 +65,18 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
                                              uint16_t *out, float sc, bool nan_codes) {
   static_assert(PB == 12 || G == 8, "7- and 8-bit tables need whole runs of 8");
   if constexpr (PB == kRansPairBits) {  // one lookup per pair of steps
-    uint32_t pr[4];
+    uint32_t pv[4];  // the pairs' values (bf16x2)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      pr[k] = rans_pair_step<FULL>(x, act, lut);
+      pv[k] = rans_pair_step<FULL>(x, act, lut);
       rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
     }
-    if (FULL || act)
+    if (FULL || act) {
+      const uint32_t sc2 = scale_bf16x2(sc);
       *reinterpret_cast<uint4 *>(out) =
-          make_uint4(dequant2<FMT>(pr[0], sc, nan_codes), dequant2<FMT>(pr[1], sc, nan_codes),
-                     dequant2<FMT>(pr[2], sc, nan_codes), dequant2<FMT>(pr[3], sc, nan_codes));
+          make_uint4(pair_dequant(pv[0], sc2, nan_codes), pair_dequant(pv[1], sc2, nan_codes),
+                     pair_dequant(pv[2], sc2, nan_codes), pair_dequant(pv[3], sc2, nan_codes));
+    }
   } else {
     uint32_t e[G];
 #pragma unroll
@@ -253,8 +255,7 @@ __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
   const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(D.table);
   // the table is only read as far as its header says it reaches: a descriptor whose table is of
   // another size is reported below, never read past its end
-  const bool table_ok =
-      hdr.magic == (PB == kRansPairBits ? kRansPairMagic : kRansMagic) && hdr.prob_bits == PB;
+  const bool table_ok = hdr.magic == rans_table_magic<FMT, PB>() && hdr.prob_bits == PB;
   const uint4 *src = reinterpret_cast<const uint4 *>(D.table + sizeof(RansTableHeader) / 4);
   constexpr uint32_t kLutVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
   if (table_ok)

@@ -69,8 +69,9 @@ __device__ __forceinline__ void fma_run(float2 (&acc)[BMAX], uint2 wa, uint2 wb,
 }
 
 // One round (8 steps) of the lane's stream -> its 8 symbols as 4 pairs, the first of each in the
-// low byte.  12-bit tables renormalise after every step, 8-bit ones after every second, 7-bit ones
-// look up two steps at once in the pair table (the steps of the decode kernel).
+// low byte (7-bit tables: the symbols' values, bf16x2).  12-bit tables renormalise after every
+// step, 8-bit ones after every second, 7-bit ones look up two steps at once in the pair table (the
+// steps of the decode kernel).
 template <uint32_t PB>
 __device__ __forceinline__ void round_pairs(uint32_t (&pr)[4], uint32_t &x, bool act,
                                             const uint32_t *lut, const unsigned char *smem,
@@ -93,13 +94,28 @@ __device__ __forceinline__ void round_pairs(uint32_t (&pr)[4], uint32_t &x, bool
   }
 }
 
+// Two weights, exactly as eq_decode writes them, from a pair: of symbols (12/8-bit tables) or of
+// the symbols' values (7-bit pair tables).
+template <int FMT, uint32_t PB>
+__device__ __forceinline__ uint32_t weights2(uint32_t pair, float sc, bool nan_codes) {
+  if constexpr (PB == kRansPairBits) return pair_dequant(pair, scale_bf16x2(sc), nan_codes);
+  else return dequant2<FMT>(pair, sc, nan_codes);
+}
+
+// the pair a one-symbol table decodes to, in the form weights2 takes
+template <int FMT, uint32_t PB>
+__device__ __forceinline__ uint32_t single_pair(uint32_t sym) {
+  if constexpr (PB == kRansPairBits) return symbol_bf16(sym, FMT) * 0x10001u;
+  else return sym * 0x0101u;
+}
+
 // Copy the PB-bit slot table (7 bits: the pair table) behind the header into shared memory, only
 // when the header names a table of that size; false otherwise (a table of another size is never
 // read past its end).
-template <uint32_t PB>
+template <int FMT, uint32_t PB>
 __device__ __forceinline__ bool load_table(uint32_t *lut, const uint32_t *table,
                                            const RansTableHeader &hdr) {
-  const bool ok = hdr.magic == (PB == kRansPairBits ? kRansPairMagic : kRansMagic) && hdr.prob_bits == PB;
+  const bool ok = hdr.magic == rans_table_magic<FMT, PB>() && hdr.prob_bits == PB;
   constexpr uint32_t kVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
   const uint4 *src = reinterpret_cast<const uint4 *>(table + sizeof(RansTableHeader) / 4);
   if (ok)
@@ -139,9 +155,9 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
 
   for (uint32_t r = 0; r < rounds; ++r) {
     const bool act = r * S + lane < runs;
-    uint32_t pr[4];  // the round's 8 symbols as 4 pairs
+    uint32_t pr[4];  // the round's 8 symbols as 4 pairs (7-bit tables: their values, bf16x2)
     if (single) {
-      pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
+      pr[0] = pr[1] = pr[2] = pr[3] = single_pair<FMT, PB>(hdr.single_sym);
     } else {
       if (!R.round_wait(q)) {
         status |= EQ_DEV_TIMEOUT;
@@ -156,8 +172,8 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
     }
     if (act) {  // the weights exactly as eq_decode writes them, times the activations
       const uint32_t col = (r * S + lane) * 8 - row_local * P.cols;
-      const uint2 wa = make_uint2(dequant2<FMT>(pr[0], sc, nan_codes), dequant2<FMT>(pr[1], sc, nan_codes));
-      const uint2 wb = make_uint2(dequant2<FMT>(pr[2], sc, nan_codes), dequant2<FMT>(pr[3], sc, nan_codes));
+      const uint2 wa = make_uint2(weights2<FMT, PB>(pr[0], sc, nan_codes), weights2<FMT, PB>(pr[1], sc, nan_codes));
+      const uint2 wb = make_uint2(weights2<FMT, PB>(pr[2], sc, nan_codes), weights2<FMT, PB>(pr[3], sc, nan_codes));
       fma_run<BMAX>(acc, wa, wb, P.x, P.cols, col, batch);
     }
     // end of a weight row: add its super weights' products, reduce across the warp, write y
@@ -219,7 +235,7 @@ __global__ void __launch_bounds__(32 * gemv_max_warps(PB, BMAX), gemv_min_ctas(P
   const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
-  const bool table_ok = load_table<PB>(lut, P.table, hdr);
+  const bool table_ok = load_table<FMT, PB>(lut, P.table, hdr);
   WordRing R;
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
@@ -297,7 +313,7 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
   };
 
   const RansTableHeader hdr = *reinterpret_cast<const RansTableHeader *>(P.table);
-  const bool table_ok = load_table<PB>(lut, P.table, hdr);
+  const bool table_ok = load_table<FMT, PB>(lut, P.table, hdr);
   WordRing R;
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
@@ -358,15 +374,15 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
           }
         }
       } else if (single) {
-        pr[0] = pr[1] = pr[2] = pr[3] = hdr.single_sym * 0x0101u;
+        pr[0] = pr[1] = pr[2] = pr[3] = single_pair<FMT, PB>(hdr.single_sym);
       }
       // this warp's 256 weights of the round -> tile row hw
       uint4 wv = make_uint4(0u, 0u, 0u, 0u);
       if (act && !status) {
-        wv.x = dequant2<FMT>(pr[0], sc, nan_codes);
-        wv.y = dequant2<FMT>(pr[1], sc, nan_codes);
-        wv.z = dequant2<FMT>(pr[2], sc, nan_codes);
-        wv.w = dequant2<FMT>(pr[3], sc, nan_codes);
+        wv.x = weights2<FMT, PB>(pr[0], sc, nan_codes);
+        wv.y = weights2<FMT, PB>(pr[1], sc, nan_codes);
+        wv.z = weights2<FMT, PB>(pr[2], sc, nan_codes);
+        wv.w = weights2<FMT, PB>(pr[3], sc, nan_codes);
       }
       unsigned char *tile = tiles + (r & 1) * kTcTileBytes;
       *reinterpret_cast<uint4 *>(tile + hw * kTcRowBytes + lane * 16) = wv;

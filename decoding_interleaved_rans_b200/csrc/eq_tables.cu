@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <vector>
 
+#include "eq_dequant.cuh"
 #include "eq_internal.cuh"
 
 namespace eq {
@@ -18,6 +19,7 @@ struct RansBuildArgs {
   uint32_t *dst;           // device table (header + 2^prob_bits entries)
   uint32_t flags, single;  // header fields
   uint32_t prob_bits;
+  uint32_t symfmt;         // pair tables: the format of the values they carry
   uint16_t freq[256];
 };
 
@@ -63,7 +65,8 @@ __global__ void __launch_bounds__(256) rans_pair_build_kernel(const __grid_const
       c += a.freq[s];
     }
     cum[256] = c;
-    RansTableHeader h{kRansPairMagic, a.flags, a.single, kRansPairBits};
+    RansTableHeader h{a.symfmt == EQ_SYM_E4M3 ? kRansPairMagicE4M3 : kRansPairMagicInt8, a.flags,
+                      a.single, kRansPairBits};
     *reinterpret_cast<RansTableHeader *>(a.dst) = h;
   }
   __syncthreads();
@@ -82,7 +85,9 @@ __global__ void __launch_bounds__(256) rans_pair_build_kernel(const __grid_const
     const uint32_t v = f1 * L + (slot1 - cum[s1]);
     const uint32_t slot2 = v & 127u, s2 = owner(slot2), f2 = a.freq[s2];
     const uint32_t F = f1 * f2, B = f2 * (v >> 7) + (slot2 - cum[s2]);
-    ent[i] = make_uint2((F & 0xFFFFu) | (s1 << 16) | (s2 << 24), B);
+    // F = 2^14 only in a one-symbol table, which the decoders never look up
+    ent[i] = make_uint2(symbol_bf16(s1, a.symfmt) | (symbol_bf16(s2, a.symfmt) << 16),
+                        ((F & 0x3FFFu) << 14) | B);
   }
 }
 
@@ -212,7 +217,7 @@ using namespace eq;
 
 extern "C" size_t eq_table_bytes(eq_table_kind kind) {
   if (kind == EQ_TABLE_RANS) return kRansTableBytes;
-  if (kind == EQ_TABLE_RANS_PAIR) return kRansPairTableBytes;
+  if (kind == EQ_TABLE_RANS_PAIR_E4M3 || kind == EQ_TABLE_RANS_PAIR_INT8) return kRansPairTableBytes;
   if (kind == EQ_TABLE_HUFF) return kHuffTableBytes;
   return 0;
 }
@@ -221,13 +226,14 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
                                      uint32_t prob_bits, void *d_tables, void *stream) {
   if (!host_in || !d_tables || !aligned(d_tables, 16)) return EQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (kind == EQ_TABLE_RANS || kind == EQ_TABLE_RANS_PAIR) {
+  if (kind == EQ_TABLE_RANS || kind == EQ_TABLE_RANS_PAIR_E4M3 || kind == EQ_TABLE_RANS_PAIR_INT8) {
     if (kind == EQ_TABLE_RANS ? (prob_bits != 12 && prob_bits != 8) : prob_bits != kRansPairBits)
       return EQ_ERR_UNSUPPORTED;
     const uint32_t slots = 1u << prob_bits;
     RansBuildArgs a;
     a.dst = static_cast<uint32_t *>(d_tables);
     a.prob_bits = prob_bits;
+    a.symfmt = kind == EQ_TABLE_RANS_PAIR_E4M3 ? EQ_SYM_E4M3 : EQ_SYM_INT8;
     uint64_t sum = 0;
     uint32_t used = 0, single = 0;
     for (int s = 0; s < 256; ++s) {

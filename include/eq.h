@@ -34,7 +34,7 @@
 extern "C" {
 #endif
 
-#define EQ_ABI_VERSION 2u
+#define EQ_ABI_VERSION 3u
 
 typedef enum {
   EQ_OK = 0,
@@ -52,7 +52,12 @@ typedef enum {
 #define EQ_DEV_TIMEOUT 16u       /* a bounded wait on an asynchronous copy gave up            */
 
 typedef enum { EQ_SYM_E4M3 = 1, EQ_SYM_INT8 = 2 } eq_symfmt;
-typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2, EQ_TABLE_RANS_PAIR = 3 } eq_table_kind;
+typedef enum {
+  EQ_TABLE_RANS = 1,
+  EQ_TABLE_HUFF = 2,
+  EQ_TABLE_RANS_PAIR_E4M3 = 3, /* 7-bit pair table carrying the symbols' Float8-E4M3 values */
+  EQ_TABLE_RANS_PAIR_INT8 = 4  /* 7-bit pair table carrying the symbols' Int8 values         */
+} eq_table_kind;
 
 /*
  * One interleaved-rANS-coded weight W[rows][cols] ("Float8@2bits: Entropy Coding Enables
@@ -74,10 +79,12 @@ typedef enum { EQ_TABLE_RANS = 1, EQ_TABLE_HUFF = 2, EQ_TABLE_RANS_PAIR = 3 } eq
  *   point after each of its steps; an 8- or 7-bit stream after every second one of its own
  *   steps (and after its last), which is exact because two such steps shrink the state by at
  *   most 2^16; it halves the renormalisation work.  A 7-bit table also decodes both steps of a
- *   pair with one lookup (EQ_TABLE_RANS_PAIR).  A well-formed chunk ends with every state at
- *   2^16 and every word read.
+ *   pair with one lookup (EQ_TABLE_RANS_PAIR_E4M3 / _INT8).  A well-formed chunk ends with every
+ *   state at 2^16 and every word read.
  *   Dequantisation: out = bf16_rne( value(s) * scale[row] ), value(s) being the E4M3 value of the
  *   byte (NaN codes 0x7F/0xFF give the bf16 quiet NaN 0x7FC0 / 0xFFC0) or the byte read as int8.
+ *   Scales are finite (the quantisers make them so); with an infinite or NaN scale a product that
+ *   is NaN comes out as some bf16 NaN.
  *   Super weights ("Float8@2bits" summary, "Manejo de Pesos Superiores": extreme outliers of Int8
  *   weights kept out of the entropy coding): an optional sorted list of (flat index, bf16 value)
  *   written over the decoded weight.  The coded symbol at a listed position must dequantise to
@@ -100,7 +107,8 @@ typedef struct {
                              zeros to a multiple of 8 words (16 bytes); base 16-byte aligned    */
   const uint16_t *scales; /* [rows] bf16 per-output-channel scales                              */
   const void *tables;     /* from eq_build_tables: EQ_TABLE_RANS for 12- and 8-bit tables,
-                             EQ_TABLE_RANS_PAIR for 7-bit ones; 16-byte aligned               */
+                             EQ_TABLE_RANS_PAIR_E4M3 / _INT8 (matching symfmt) for 7-bit ones;
+                             16-byte aligned                                                  */
   uint64_t n_patch;       /* super weights in the list (0: none)                               */
   const uint64_t *patch_idx; /* [n_patch] flat row-major indices, strictly increasing           */
   const uint16_t *patch_val; /* [n_patch] their bf16 values                                     */
@@ -167,10 +175,13 @@ size_t eq_table_bytes(eq_table_kind kind);
  *     or 8).
  *     Builds the slot table: one 32-bit entry per slot holding the slot's symbol, its frequency
  *     and slot - cum[symbol].
- *   EQ_TABLE_RANS_PAIR: host_in[256] = frequencies summing to 128 (prob_bits = 7).  Builds the
- *     pair table (16384 x 8 bytes): for each value of the state's low 14 bits, the two symbols
- *     the next two steps decode and the two steps' combined product and offset, so a pair of
- *     steps is one lookup and one multiply-add.
+ *   EQ_TABLE_RANS_PAIR_E4M3 / EQ_TABLE_RANS_PAIR_INT8: host_in[256] = frequencies summing to
+ *     128 (prob_bits = 7).  Builds the pair table (16384 x 8 bytes): for each value of the
+ *     state's low 14 bits, the values (as bf16, exact) of the two symbols the next two steps
+ *     decode, in the symbol format the kind names, and the two steps' combined product and
+ *     offset, so a pair of steps is one lookup and one multiply-add and its dequantisation one
+ *     bf16x2 multiply by the row scale.  A tensor's table must be of its own symbol format
+ *     (eq_decode reports EQ_DEV_CORRUPT_STATE otherwise).
  *   EQ_TABLE_HUFF: host_in[256] = code length of each exponent value (0 = absent), prob_bits
  *     ignored.  Builds the hierarchical lookup tables of the DFloat11 page ("Decodificacion
  *     basada en LUT jerarquicas": the code tree cut into height-8 subtrees, each a 256-entry

@@ -38,10 +38,13 @@ def test_every_declared_symbol_is_exported(eq):
 
 def test_version_and_strings(eq):
     L = eq.lib()
-    assert L.eq_abi_version() == 2
+    assert L.eq_abi_version() == 3
     for code in range(5):
         assert L.eq_status_string(code)
     assert eq.table_bytes(1) >= 4096 * 4 and eq.table_bytes(2) > 0 and eq.table_bytes(7) == 0
+    # 7-bit pair tables, one kind per symbol format: 16384 entries of 8 bytes behind the header
+    assert eq.table_bytes(eq.EQ_TABLE_RANS_PAIR_E4M3) == eq.table_bytes(eq.EQ_TABLE_RANS_PAIR_INT8) \
+        == 16 + 16384 * 8
 
 
 def test_build_tables_rejects_bad_input_on_host(eq):
@@ -56,6 +59,13 @@ def test_build_tables_rejects_bad_input_on_host(eq):
     assert L.eq_build_tables(2, too_long, 0, fake, None) == 2
     over_kraft = (C.c_uint32 * 256)(*([1, 1, 1] + [0] * 253))
     assert L.eq_build_tables(2, over_kraft, 0, fake, None) == 2
+    # pair tables (both symbol formats) take 7-bit frequencies only
+    seven = (C.c_uint32 * 256)(*([1] * 128 + [0] * 128))
+    for kind in (eq.EQ_TABLE_RANS_PAIR_E4M3, eq.EQ_TABLE_RANS_PAIR_INT8):
+        assert L.eq_build_tables(kind, ok, 12, fake, None) == 3
+        assert L.eq_build_tables(kind, bad_sum, 7, fake, None) == 2
+        assert L.eq_build_tables(kind, seven, 7, C.c_void_p((1 << 20) + 8), None) == 1
+    assert L.eq_build_tables(5, seven, 7, fake, None) == 1  # no such kind
 
 
 def test_decode_rejects_bad_descriptors_on_host(eq):

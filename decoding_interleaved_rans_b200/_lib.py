@@ -16,6 +16,7 @@ EQ_DEV_CORRUPT_STATE, EQ_DEV_OVERRUN, EQ_DEV_BAD_CODE = 1, 2, 4
 EQ_DEV_COUNT_MISMATCH, EQ_DEV_TIMEOUT = 8, 16
 EQ_SYM_E4M3, EQ_SYM_INT8 = 1, 2
 EQ_TABLE_RANS, EQ_TABLE_HUFF, EQ_TABLE_RANS_PAIR_E4M3, EQ_TABLE_RANS_PAIR_INT8 = 1, 2, 3, 4
+EQ_TABLE_RANS8_E4M3, EQ_TABLE_RANS8_INT8 = 5, 6
 EQ_ABI_VERSION = 3
 
 # every exported function of include/eq.h and include/eq_encode.h

@@ -46,11 +46,14 @@ def new_status(device) -> torch.Tensor:
 
 
 def rans_table_kind(prob_bits: int, symfmt: int) -> int:
-    """7-bit tables decode through a pair table carrying the symbols' values (one kind per symbol
-    format), the others through a slot table."""
-    if prob_bits != 7:
-        return L.EQ_TABLE_RANS
-    return L.EQ_TABLE_RANS_PAIR_E4M3 if symfmt == L.EQ_SYM_E4M3 else L.EQ_TABLE_RANS_PAIR_INT8
+    """12-bit tables decode through a slot table of symbols; 8-bit ones through a slot table and
+    7-bit ones through a pair table, both carrying the symbols' values (one kind per format)."""
+    e4 = symfmt == L.EQ_SYM_E4M3
+    if prob_bits == 7:
+        return L.EQ_TABLE_RANS_PAIR_E4M3 if e4 else L.EQ_TABLE_RANS_PAIR_INT8
+    if prob_bits == 8:
+        return L.EQ_TABLE_RANS8_E4M3 if e4 else L.EQ_TABLE_RANS8_INT8
+    return L.EQ_TABLE_RANS
 
 
 @dataclass

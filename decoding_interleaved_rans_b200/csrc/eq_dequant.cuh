@@ -5,6 +5,8 @@
 // channel (section "Optimizacion con Restriccion de Entropia": per-channel scales S).  Both
 // factors are exact in fp32 and their product has at most 15 significant bits, so the fp32
 // multiply is exact and the conversion to bf16 is the only rounding (round to nearest even).
+// 8- and 7-bit tables carry the symbols' values as bf16 (exact): there one bf16x2 multiply
+// computes two weights, its single rounding being the same round to nearest even.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,27 +51,6 @@ __device__ __forceinline__ uint32_t dequant2(uint32_t pair, float scale, bool na
   return o;
 }
 
-// the eight symbols of a round, taken from their PB-bit slot-table entries (symbol in bits
-// 19..12 of 12-bit entries, 23..16 of 8-bit ones), scaled -> eight bf16 (one 16-byte store)
-template <int FMT, uint32_t PB = 12>
-__device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, bool nan_codes) {
-  uint32_t o[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    if constexpr (FMT == EQ_SYM_INT8) {
-      // the symbol byte sign-extended straight out of the entry
-      constexpr int kUp = PB == 8 ? 8 : 24 - int(PB);
-      const float v0 = float(int32_t(e[2 * k] << kUp) >> 24);
-      const float v1 = float(int32_t(e[2 * k + 1] << kUp) >> 24);
-      o[k] = pack_bf16x2(v0 * scale, v1 * scale);
-    } else {
-      if constexpr (PB == 8) o[k] = dequant2<FMT>(__byte_perm(e[2 * k], e[2 * k + 1], 0x0062u), scale, nan_codes);
-      else o[k] = dequant2<FMT>(((e[2 * k] >> PB) & 0xFFu) | ((e[2 * k + 1] >> (PB - 8)) & 0xFF00u), scale, nan_codes);
-    }
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
 // a symbol's value as bf16 bits, exactly (E4M3: at most 4 significant bits, exponent within
 // bf16's range; Int8: at most 8 bits); the E4M3 NaN codes give the quiet NaN with their sign
 __device__ __forceinline__ uint32_t symbol_bf16(uint32_t s, uint32_t symfmt) {
@@ -80,7 +61,8 @@ __device__ __forceinline__ uint32_t symbol_bf16(uint32_t s, uint32_t symfmt) {
   return __float_as_uint(float(int32_t(s << 24) >> 24)) >> 16;
 }
 
-// A pair of symbol values from a 7-bit pair table (bf16x2, exact) times the row scale: one
+// A pair of symbol values from an 8-bit slot table or a 7-bit pair table (bf16x2, exact) times
+// the row scale: one
 // bf16x2 multiply, whose single round-to-nearest-even of the exact product is bf16_rne(value *
 // scale).  sc2: the scale's bf16 bits in both halves.  Halves holding an E4M3 NaN code's value
 // (the quiet NaN with the code's sign) pass through unscaled when nan_codes.
@@ -97,6 +79,37 @@ __device__ __forceinline__ uint32_t pair_dequant(uint32_t vals, uint32_t sc2, bo
 // the bf16 bits of a scale held as fp32 (converted exactly from bf16), in both halves
 __device__ __forceinline__ uint32_t scale_bf16x2(float sc) {
   return __byte_perm(__float_as_uint(sc), 0u, 0x3232u);
+}
+
+// the values (bf16x2, first in the low half) of two 8-bit slot-table entries (value in bits 23..8)
+__device__ __forceinline__ uint32_t value_pair8(uint32_t e0, uint32_t e1) {
+  return __byte_perm(e0, e1, 0x6521u);
+}
+
+// the eight symbols of a round, taken from their PB-bit slot-table entries (12-bit: the symbol in
+// bits 19..12; 8-bit: the symbol's value as bf16 in bits 23..8), scaled -> eight bf16 (one 16-byte
+// store)
+template <int FMT, uint32_t PB = 12>
+__device__ __forceinline__ uint4 dequant8(const uint32_t (&e)[8], float scale, bool nan_codes) {
+  uint32_t o[4];
+  if constexpr (PB == 8) {
+    const uint32_t sc2 = scale_bf16x2(scale);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] = pair_dequant(value_pair8(e[2 * k], e[2 * k + 1]), sc2, nan_codes);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (FMT == EQ_SYM_INT8) {
+        // the symbol byte sign-extended straight out of the entry
+        const float v0 = float(int32_t(e[2 * k] << 12) >> 24);
+        const float v1 = float(int32_t(e[2 * k + 1] << 12) >> 24);
+        o[k] = pack_bf16x2(v0 * scale, v1 * scale);
+      } else {
+        o[k] = dequant2<FMT>(((e[2 * k] >> 12) & 0xFFu) | ((e[2 * k + 1] >> 4) & 0xFF00u), scale, nan_codes);
+      }
+    }
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // one symbol -> bf16 bits

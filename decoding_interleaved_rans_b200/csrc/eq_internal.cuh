@@ -15,22 +15,26 @@ namespace eq {
 // rANS: 16-byte header, then one 32-bit entry per slot of the 2^pb-slot probability space
 // (pb = prob_bits, 12 or 8), f = frequency of the slot's symbol (1 .. 2^pb - 1):
 //   12-bit: bits 31..20 f, bits 19..12 symbol, bits 11..0 slot - cum;
-//   8-bit:  bits 31..24 f, bits 23..16 symbol, bits 15..8 zero, bits 7..0 slot - cum;
+//   8-bit:  bits 31..24 f, bits 23..8 the symbol's value as bf16, bits 7..0 slot - cum;
 // so the decode step x' = f * floor(x / 2^pb) + slot - cum is (e >> (32 - pb)) * (x >> pb) +
 // (e & (2^pb - 1)).
 // A table whose single symbol owns every slot cannot store its frequency in pb bits; the header
-// flags it instead and the decoders take a separate path.  8-bit tables use the first 256
-// entries of the same 16 KiB allocation.
+// flags it instead and the decoders take a separate path.
 constexpr uint32_t kRansProbBits = 12;                 // the larger table
 constexpr uint32_t kRansSlots = 1u << kRansProbBits;  // entries the table allocation holds
 constexpr uint32_t kRansL = 1u << 16;
 struct RansTableHeader {
-  uint32_t magic;        // kRansMagic
+  uint32_t magic;        // kRansMagic, kRans8Magic*, kRansPairMagic*
   uint32_t flags;        // kRansFlag*
   uint32_t single_sym;   // symbol of a one-symbol table
   uint32_t prob_bits;    // 12 or 8
 };
-constexpr uint32_t kRansMagic = 0x52414E53u;  // "RANS"
+constexpr uint32_t kRansMagic = 0x52414E53u;  // "RANS" (12-bit slot table)
+// 8-bit slot tables (EQ_TABLE_RANS8_E4M3 / _INT8) carry the symbol's value as bf16 bits (exact, as
+// in the pair tables below) instead of the symbol, so they are specific to the symbol format.
+constexpr uint32_t kRans8MagicE4M3 = 0x52563845u;  // "RV8E"
+constexpr uint32_t kRans8MagicInt8 = 0x52563849u;  // "RV8I"
+constexpr size_t kRans8TableBytes = 16 + 256 * 4;
 // rANS pair table of a 7-bit frequency table (EQ_TABLE_RANS_PAIR_E4M3 / _INT8): two decode
 // steps at once.  Entry i (i = x mod 2^14, the state's low 14 bits) for slot1 = i mod 128,
 // L = i >> 7:

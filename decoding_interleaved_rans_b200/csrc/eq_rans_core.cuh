@@ -197,17 +197,18 @@ __device__ __forceinline__ uint32_t rans_pair_step(uint32_t &x, bool act, const 
   return w0;
 }
 
-// the header magic of a PB-bit table for symbols of format FMT (7-bit pair tables carry the
-// symbols' values, so they are specific to the format)
+// the header magic of a PB-bit table for symbols of format FMT (8-bit slot tables and 7-bit pair
+// tables carry the symbols' values, so they are specific to the format)
 template <int FMT, uint32_t PB>
 __device__ __forceinline__ constexpr uint32_t rans_table_magic() {
-  return PB != kRansPairBits ? kRansMagic
-                             : FMT == EQ_SYM_E4M3 ? kRansPairMagicE4M3 : kRansPairMagicInt8;
+  return PB == 12 ? kRansMagic
+         : PB == 8 ? (FMT == EQ_SYM_E4M3 ? kRans8MagicE4M3 : kRans8MagicInt8)
+                   : (FMT == EQ_SYM_E4M3 ? kRansPairMagicE4M3 : kRansPairMagicInt8);
 }
 
 // the symbol byte of a PB-bit entry
 template <uint32_t PB>
-constexpr uint32_t kSymShift = PB == 8 ? 16 : PB;
+constexpr uint32_t kSymShift = PB;
 
 // A renormalisation point: every lane below 2^16 takes the group's next word, in lane order.
 // All lanes load (the others drop the word), which keeps the step free of branches; the load
@@ -245,11 +246,9 @@ __device__ __forceinline__ uint64_t patch_lower_bound(const uint64_t *idx, uint6
   return lo;
 }
 
-// symbols of two PB-bit slot-table entries as one 16-bit pair (first in the low byte)
-template <uint32_t PB = 12>
+// symbols of two 12-bit slot-table entries as one 16-bit pair (first in the low byte)
 __device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {
-  if constexpr (PB == 8) return __byte_perm(e0, e1, 0x0062u);
-  else return ((e0 >> PB) & 0xFFu) | ((e1 >> (PB - 8)) & 0xFF00u);
+  return ((e0 >> 12) & 0xFFu) | ((e1 >> 4) & 0xFF00u);
 }
 
 // Init the rings' mbarriers (lane 0 of each warp) -- call before the block-wide sync.

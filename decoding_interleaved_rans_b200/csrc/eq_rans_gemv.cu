@@ -69,7 +69,7 @@ __device__ __forceinline__ void fma_run(float2 (&acc)[BMAX], uint2 wa, uint2 wb,
 }
 
 // One round (8 steps) of the lane's stream -> its 8 symbols as 4 pairs, the first of each in the
-// low byte (7-bit tables: the symbols' values, bf16x2).  12-bit tables renormalise after every
+// low byte (8- and 7-bit tables: the symbols' values, bf16x2).  12-bit tables renormalise after every
 // step, 8-bit ones after every second, 7-bit ones look up two steps at once in the pair table (the
 // steps of the decode kernel).
 template <uint32_t PB>
@@ -90,22 +90,23 @@ __device__ __forceinline__ void round_pairs(uint32_t (&pr)[4], uint32_t &x, bool
       if (PB == 12 || (p & 1)) rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) pr[k] = sym_pair<PB>(e[2 * k], e[2 * k + 1]);
+    for (int k = 0; k < 4; ++k)
+      pr[k] = PB == 8 ? value_pair8(e[2 * k], e[2 * k + 1]) : sym_pair(e[2 * k], e[2 * k + 1]);
   }
 }
 
-// Two weights, exactly as eq_decode writes them, from a pair: of symbols (12/8-bit tables) or of
-// the symbols' values (7-bit pair tables).
+// Two weights, exactly as eq_decode writes them, from a pair: of symbols (12-bit tables) or of
+// the symbols' values (8-bit slot and 7-bit pair tables).
 template <int FMT, uint32_t PB>
 __device__ __forceinline__ uint32_t weights2(uint32_t pair, float sc, bool nan_codes) {
-  if constexpr (PB == kRansPairBits) return pair_dequant(pair, scale_bf16x2(sc), nan_codes);
+  if constexpr (PB != 12) return pair_dequant(pair, scale_bf16x2(sc), nan_codes);
   else return dequant2<FMT>(pair, sc, nan_codes);
 }
 
 // the pair a one-symbol table decodes to, in the form weights2 takes
 template <int FMT, uint32_t PB>
 __device__ __forceinline__ uint32_t single_pair(uint32_t sym) {
-  if constexpr (PB == kRansPairBits) return symbol_bf16(sym, FMT) * 0x10001u;
+  if constexpr (PB != 12) return symbol_bf16(sym, FMT) * 0x10001u;
   else return sym * 0x0101u;
 }
 

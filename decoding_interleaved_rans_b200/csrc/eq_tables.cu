@@ -34,7 +34,9 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
       c += a.freq[s];
     }
     cum[256] = c;
-    RansTableHeader h{kRansMagic, a.flags, a.single, a.prob_bits};
+    const uint32_t magic = a.prob_bits == 12 ? kRansMagic
+                           : a.symfmt == EQ_SYM_E4M3 ? kRans8MagicE4M3 : kRans8MagicInt8;
+    RansTableHeader h{magic, a.flags, a.single, a.prob_bits};
     *reinterpret_cast<RansTableHeader *>(a.dst) = h;
   }
   __syncthreads();
@@ -49,7 +51,8 @@ __global__ void __launch_bounds__(256) rans_build_kernel(const __grid_constant__
     }
     uint32_t f = a.freq[lo];
     uint32_t fe = (f >= slots) ? 0u : f;  // a one-symbol table is handled by the flag
-    lut[slot] = (fe << (32 - pb)) | (uint32_t(lo) << (pb == 8 ? 16 : 12)) | (slot - cum[lo]);
+    if (pb == 8) lut[slot] = (fe << 24) | (symbol_bf16(uint32_t(lo), a.symfmt) << 8) | (slot - cum[lo]);
+    else lut[slot] = (fe << 20) | (uint32_t(lo) << 12) | (slot - cum[lo]);
   }
 }
 
@@ -217,6 +220,7 @@ using namespace eq;
 
 extern "C" size_t eq_table_bytes(eq_table_kind kind) {
   if (kind == EQ_TABLE_RANS) return kRansTableBytes;
+  if (kind == EQ_TABLE_RANS8_E4M3 || kind == EQ_TABLE_RANS8_INT8) return kRans8TableBytes;
   if (kind == EQ_TABLE_RANS_PAIR_E4M3 || kind == EQ_TABLE_RANS_PAIR_INT8) return kRansPairTableBytes;
   if (kind == EQ_TABLE_HUFF) return kHuffTableBytes;
   return 0;
@@ -226,14 +230,15 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
                                      uint32_t prob_bits, void *d_tables, void *stream) {
   if (!host_in || !d_tables || !aligned(d_tables, 16)) return EQ_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (kind == EQ_TABLE_RANS || kind == EQ_TABLE_RANS_PAIR_E4M3 || kind == EQ_TABLE_RANS_PAIR_INT8) {
-    if (kind == EQ_TABLE_RANS ? (prob_bits != 12 && prob_bits != 8) : prob_bits != kRansPairBits)
-      return EQ_ERR_UNSUPPORTED;
+  const bool pair = kind == EQ_TABLE_RANS_PAIR_E4M3 || kind == EQ_TABLE_RANS_PAIR_INT8;
+  const bool rans8 = kind == EQ_TABLE_RANS8_E4M3 || kind == EQ_TABLE_RANS8_INT8;
+  if (kind == EQ_TABLE_RANS || pair || rans8) {
+    if (prob_bits != (pair ? kRansPairBits : rans8 ? 8u : 12u)) return EQ_ERR_UNSUPPORTED;
     const uint32_t slots = 1u << prob_bits;
     RansBuildArgs a;
     a.dst = static_cast<uint32_t *>(d_tables);
     a.prob_bits = prob_bits;
-    a.symfmt = kind == EQ_TABLE_RANS_PAIR_E4M3 ? EQ_SYM_E4M3 : EQ_SYM_INT8;
+    a.symfmt = kind == EQ_TABLE_RANS_PAIR_E4M3 || kind == EQ_TABLE_RANS8_E4M3 ? EQ_SYM_E4M3 : EQ_SYM_INT8;
     uint64_t sum = 0;
     uint32_t used = 0, single = 0;
     for (int s = 0; s < 256; ++s) {
@@ -249,8 +254,8 @@ extern "C" eq_status eq_build_tables(eq_table_kind kind, const uint32_t *host_in
     a.flags = (host_in[0x7F] ? kRansFlagNaN7F : 0u) | (host_in[0xFF] ? kRansFlagNaNFF : 0u) |
               (used == 1 ? kRansFlagSingle : 0u);
     a.single = used == 1 ? single : 0u;
-    if (kind == EQ_TABLE_RANS) rans_build_kernel<<<1, 256, 0, st>>>(a);
-    else rans_pair_build_kernel<<<1, 256, 0, st>>>(a);
+    if (pair) rans_pair_build_kernel<<<1, 256, 0, st>>>(a);
+    else rans_build_kernel<<<1, 256, 0, st>>>(a);
     return cuda_status(cudaGetLastError());
   }
   if (kind == EQ_TABLE_HUFF) {

@@ -56,7 +56,9 @@ typedef enum {
   EQ_TABLE_RANS = 1,
   EQ_TABLE_HUFF = 2,
   EQ_TABLE_RANS_PAIR_E4M3 = 3, /* 7-bit pair table carrying the symbols' Float8-E4M3 values */
-  EQ_TABLE_RANS_PAIR_INT8 = 4  /* 7-bit pair table carrying the symbols' Int8 values         */
+  EQ_TABLE_RANS_PAIR_INT8 = 4, /* 7-bit pair table carrying the symbols' Int8 values         */
+  EQ_TABLE_RANS8_E4M3 = 5,     /* 8-bit slot table carrying the symbols' Float8-E4M3 values */
+  EQ_TABLE_RANS8_INT8 = 6      /* 8-bit slot table carrying the symbols' Int8 values         */
 } eq_table_kind;
 
 /*
@@ -106,9 +108,10 @@ typedef struct {
   const uint16_t *words;  /* all substreams, chunk-major, decoder order; allocation padded with
                              zeros to a multiple of 8 words (16 bytes); base 16-byte aligned    */
   const uint16_t *scales; /* [rows] bf16 per-output-channel scales                              */
-  const void *tables;     /* from eq_build_tables: EQ_TABLE_RANS for 12- and 8-bit tables,
-                             EQ_TABLE_RANS_PAIR_E4M3 / _INT8 (matching symfmt) for 7-bit ones;
-                             16-byte aligned                                                  */
+  const void *tables;     /* from eq_build_tables: EQ_TABLE_RANS for 12-bit tables,
+                             EQ_TABLE_RANS8_E4M3 / _INT8 for 8-bit ones and
+                             EQ_TABLE_RANS_PAIR_E4M3 / _INT8 for 7-bit ones (the kind matching
+                             symfmt); 16-byte aligned                                         */
   uint64_t n_patch;       /* super weights in the list (0: none)                               */
   const uint64_t *patch_idx; /* [n_patch] flat row-major indices, strictly increasing           */
   const uint16_t *patch_val; /* [n_patch] their bf16 values                                     */
@@ -171,10 +174,14 @@ size_t eq_table_bytes(eq_table_kind kind);
  * Build the device decode tables of one tensor into d_tables (eq_table_bytes(kind) bytes,
  * 16-byte aligned, caller-owned).  The table contents travel as kernel arguments: no host
  * buffer outlives the call and no copy engine is used.
- *   EQ_TABLE_RANS: host_in[256] = symbol frequencies, summing to 2^prob_bits (prob_bits = 12
- *     or 8).
+ *   EQ_TABLE_RANS: host_in[256] = symbol frequencies, summing to 4096 (prob_bits = 12).
  *     Builds the slot table: one 32-bit entry per slot holding the slot's symbol, its frequency
  *     and slot - cum[symbol].
+ *   EQ_TABLE_RANS8_E4M3 / EQ_TABLE_RANS8_INT8: host_in[256] = frequencies summing to 256
+ *     (prob_bits = 8).  Builds the 8-bit slot table: one 32-bit entry per slot holding the
+ *     frequency, slot - cum[symbol] and, instead of the symbol, its value as bf16 (exact) in the
+ *     symbol format the kind names, so that two decoded symbols dequantise with one bf16x2
+ *     multiply by the row scale.
  *   EQ_TABLE_RANS_PAIR_E4M3 / EQ_TABLE_RANS_PAIR_INT8: host_in[256] = frequencies summing to
  *     128 (prob_bits = 7).  Builds the pair table (16384 x 8 bytes): for each value of the
  *     state's low 14 bits, the values (as bf16, exact) of the two symbols the next two steps

@@ -42,9 +42,11 @@ def test_version_and_strings(eq):
     for code in range(5):
         assert L.eq_status_string(code)
     assert eq.table_bytes(1) >= 4096 * 4 and eq.table_bytes(2) > 0 and eq.table_bytes(7) == 0
-    # 7-bit pair tables, one kind per symbol format: 16384 entries of 8 bytes behind the header
+    # 7-bit pair tables, one kind per symbol format: 16384 entries of 8 bytes behind the header;
+    # 8-bit slot tables likewise: 256 entries of 4 bytes
     assert eq.table_bytes(eq.EQ_TABLE_RANS_PAIR_E4M3) == eq.table_bytes(eq.EQ_TABLE_RANS_PAIR_INT8) \
         == 16 + 16384 * 8
+    assert eq.table_bytes(eq.EQ_TABLE_RANS8_E4M3) == eq.table_bytes(eq.EQ_TABLE_RANS8_INT8) == 16 + 256 * 4
 
 
 def test_build_tables_rejects_bad_input_on_host(eq):
@@ -65,7 +67,13 @@ def test_build_tables_rejects_bad_input_on_host(eq):
         assert L.eq_build_tables(kind, ok, 12, fake, None) == 3
         assert L.eq_build_tables(kind, bad_sum, 7, fake, None) == 2
         assert L.eq_build_tables(kind, seven, 7, C.c_void_p((1 << 20) + 8), None) == 1
-    assert L.eq_build_tables(5, seven, 7, fake, None) == 1  # no such kind
+    # 8-bit slot tables (both formats) take 8-bit frequencies only; the 12-bit kind 12-bit ones
+    eight = (C.c_uint32 * 256)(*([1] * 256))
+    for kind in (eq.EQ_TABLE_RANS8_E4M3, eq.EQ_TABLE_RANS8_INT8):
+        assert L.eq_build_tables(kind, ok, 12, fake, None) == 3
+        assert L.eq_build_tables(kind, seven, 7, fake, None) == 3
+    assert L.eq_build_tables(eq.EQ_TABLE_RANS, eight, 8, fake, None) == 3
+    assert L.eq_build_tables(7, seven, 7, fake, None) == 1  # no such kind
 
 
 def test_decode_rejects_bad_descriptors_on_host(eq):

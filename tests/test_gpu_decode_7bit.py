@@ -100,8 +100,8 @@ def test_corruption_and_mismatched_tables(eq, orc):
     # read, nothing past the table is touched, and the tensor is reported
     h = orc.rans_encode(sym, sc, orc.INT8, 16384, 32, 8, prob_bits=7)
     t = eq.DeviceRans.upload(h)
-    small = torch.zeros(eq.table_bytes(eq.EQ_TABLE_RANS), dtype=torch.uint8, device="cuda")
-    eq.build_tables(eq.EQ_TABLE_RANS, orc.rans_freqs(sym, 8), 8, small)
+    small = torch.zeros(eq.table_bytes(eq.EQ_TABLE_RANS8_INT8), dtype=torch.uint8, device="cuda")
+    eq.build_tables(eq.EQ_TABLE_RANS8_INT8, orc.rans_freqs(sym, 8), 8, small)
     t.tables = small
     _, status = eq.decode([t])
     torch.cuda.synchronize()

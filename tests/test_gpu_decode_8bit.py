@@ -106,14 +106,16 @@ def test_corruption_and_mismatched_table(eq, orc):
     h.word_off[1:] -= 1
     h.words = np.concatenate([h.words[:int(h.word_off[1])], h.words[int(h.word_off[1]) + 1:]])
     assert run_decode(eq, [h])[1] & 3
-    # a 12-bit table under an 8-bit descriptor: caught on the device, nothing decoded from it
+    # a 12-bit table, or an 8-bit one of the other symbol format, under an 8-bit Int8
+    # descriptor: caught on the device, nothing decoded from it
     h = orc.rans_encode(sym, sc, orc.INT8, 16384, 32, 8, prob_bits=8)
-    t = eq.DeviceRans.upload(h)
-    f12 = orc.rans_freqs(sym, 12)
-    eq.build_tables(eq.EQ_TABLE_RANS, f12, 12, t.tables)
-    outs, status = eq.decode([t])
-    torch.cuda.synchronize()
-    assert int(status.item()) & eq.EQ_DEV_CORRUPT_STATE
+    for kind, pb in ((eq.EQ_TABLE_RANS, 12), (eq.EQ_TABLE_RANS8_E4M3, 8)):
+        t = eq.DeviceRans.upload(h)
+        t.tables = torch.zeros(eq.table_bytes(kind), dtype=torch.uint8, device="cuda")
+        eq.build_tables(kind, orc.rans_freqs(sym, pb), pb, t.tables)
+        outs, status = eq.decode([t])
+        torch.cuda.synchronize()
+        assert int(status.item()) & eq.EQ_DEV_CORRUPT_STATE
 
 
 def test_8bit_needs_runs_of_8(eq, orc):

@@ -117,8 +117,8 @@ def test_table_of_another_size_is_reported(eq, orc, batch):
     is read, nothing past it is touched, and the launch reports the tensor."""
     sym, sc = int8_syms(orc, 64, 1024, 550)
     t = eq.DeviceRans.upload(orc.rans_encode(sym, sc, orc.INT8, 1024, 32, 8, prob_bits=7))
-    small = torch.zeros(eq.table_bytes(eq.EQ_TABLE_RANS), dtype=torch.uint8, device="cuda")
-    eq.build_tables(eq.EQ_TABLE_RANS, orc.rans_freqs(sym, 8), 8, small)
+    small = torch.zeros(eq.table_bytes(eq.EQ_TABLE_RANS8_INT8), dtype=torch.uint8, device="cuda")
+    eq.build_tables(eq.EQ_TABLE_RANS8_INT8, orc.rans_freqs(sym, 8), 8, small)
     t.tables = small
     x = torch.zeros(batch, 1024, dtype=torch.bfloat16, device="cuda")
     _, status = eq.decode_gemv(t, x)

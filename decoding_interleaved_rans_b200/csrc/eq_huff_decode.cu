@@ -145,20 +145,35 @@ __device__ __forceinline__ uint32_t segment(const uint64_t *win, const uint16_t 
     }
     const uint32_t w = __funnelshift_l(r1, r0, pos);
     const uint64_t f = win[w >> (32 - kHuffWindowBits)];
-    uint32_t sym, len;
     if (f & kHuffLong) {
-      len = tree_decode(tree, ntab, w, &sym);
-    } else {  // the first code of the window (a window that is not long holds at least one)
-      sym = uint32_t(f) & 0xFFu;
-      len = uint32_t(f >> 32) & 0xFu;
+      uint32_t sym;
+      const uint32_t len = tree_decode(tree, ntab, w, &sym);
+      if (!len) {
+        *bad = EQ_DEV_BAD_CODE;
+        break;
+      }
+      out.put(sym, 1);
+      ++cnt;
+      pos += len;
+      continue;
     }
-    if (!len) {
+    // the window's codes that start before `end` (the first always does)
+    const uint32_t hi = uint32_t(f >> 32), k = (hi >> 20) & 7u;
+    if (k == 0) {  // no code fits and the first is not long: no code matches
       *bad = EQ_DEV_BAD_CODE;
       break;
     }
-    out.put(sym, 1);
-    ++cnt;
-    pos += len;
+    uint32_t kk = 1, p = pos + (hi & 0xFu);
+#pragma unroll
+    for (uint32_t i = 1; i < 4; ++i) {
+      if (i < k && p < end) {
+        ++kk;
+        p += (hi >> (4 * i)) & 0xFu;
+      }
+    }
+    out.put(uint32_t(f) & (0xFFFFFFFFu >> (32 - 8 * kk)), kk);
+    cnt += kk;
+    pos = p;
   }
   out.flush();
   return cnt;

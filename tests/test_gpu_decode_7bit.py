@@ -31,15 +31,17 @@ def int8_syms(orc, rows, cols, seed):
     return orc.quantize(w, orc.INT8, synth.INT8_DIV_LAPLACE_8K)
 
 
-def test_int8_full_size(eq, orc):
+@pytest.mark.parametrize("streams", [None, 128, 96])
+def test_int8_full_size(eq, orc, streams):
+    """The bench weight in the bench's layout, and with 128 / 96 streams per chunk."""
     wl = synth.WORKLOADS["int8_8k"]
     sym, sc = orc.quantize(wl.tensors[0].generate(), orc.INT8, wl.int8_div)
-    h = orc.rans_encode(sym, sc, orc.INT8, wl.chunk_symbols, wl.streams, wl.run, prob_bits=7)
+    h = orc.rans_encode(sym, sc, orc.INT8, wl.chunk_symbols, streams or wl.streams, wl.run, prob_bits=7)
     (out,), st = run_decode(eq, [h])
     assert st == 0 and np.array_equal(out, orc.dequant(sym, sc, orc.INT8).ravel())
 
 
-@pytest.mark.parametrize("streams", [32, 64, 128, 256, 1024])
+@pytest.mark.parametrize("streams", [32, 64, 96, 128, 192, 256, 1024])
 def test_layouts(eq, orc, streams):
     sym, sc = int8_syms(orc, 512, 2048, 400 + streams)
     h = orc.rans_encode(sym, sc, orc.INT8, 65536 * (1 + streams // 256), streams, 8, prob_bits=7)
@@ -57,21 +59,23 @@ def test_ragged_shapes_and_unit_loops(eq, orc, rows, cols, chunk, streams):
     assert st == 0 and np.array_equal(out, orc.dequant(sym, sc, orc.INT8).ravel())
 
 
-def test_e4m3_symbols_and_nan_codes(eq, orc):
+@pytest.mark.parametrize("streams", [32, 64])
+def test_e4m3_symbols_and_nan_codes(eq, orc, streams):
     rng = np.random.default_rng(420)
     alphabet = rng.choice(256, 120, replace=False).astype(np.uint8)
     alphabet[:2] = [0x7F, 0xFF]  # NaN codes decode to the signed quiet NaN
     sym = rng.choice(alphabet, (64, 1024)).astype(np.uint8)
     sc = synth.bf16_bits(rng.uniform(1e-3, 2.0, 64).astype(np.float32))
-    h = orc.rans_encode(sym, sc, orc.E4M3, 16384, 32, 8, prob_bits=7)
+    h = orc.rans_encode(sym, sc, orc.E4M3, 16384, streams, 8, prob_bits=7)
     (out,), st = run_decode(eq, [h])
     assert st == 0 and np.array_equal(out, orc.dequant(sym, sc, orc.E4M3).ravel())
 
 
-def test_single_symbol_table(eq, orc):
+@pytest.mark.parametrize("streams", [32, 64])
+def test_single_symbol_table(eq, orc, streams):
     sym = np.full((16, 256), 0x03, np.uint8)
     sc = np.full(16, 0x3F80, np.uint16)
-    h = orc.rans_encode(sym, sc, orc.INT8, 1024, 32, 8, prob_bits=7)
+    h = orc.rans_encode(sym, sc, orc.INT8, 1024, streams, 8, prob_bits=7)
     (out,), st = run_decode(eq, [h])
     assert st == 0 and np.array_equal(out, orc.dequant(sym, sc, orc.INT8).ravel())
 

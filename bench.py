@@ -40,7 +40,7 @@ METRIC = "decoded params/s (rANS decode to bf16)"
 KERNEL_SOURCES = {
     "rans_decode_kernel": ["eq_rans_decode.cu", "eq_rans_core.cuh", "eq_dequant.cuh",
                            "eq_internal.cuh"],
-    "huff_decode_kernel": ["eq_huff_decode.cu", "eq_internal.cuh"],
+    "huff_decode_kernel": ["eq_huff_decode.cu", "eq_dequant.cuh", "eq_internal.cuh"],
     "rans_gemv_kernel": ["eq_rans_gemv.cu", "eq_rans_core.cuh", "eq_dequant.cuh",
                          "eq_internal.cuh"],
 }
@@ -54,16 +54,39 @@ def kernel_sources_sha(kernel: str) -> str:
     return h.hexdigest()
 
 
-def measured_traffic(kernel: str, units: int):
-    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json), scaled to
-    `units` weights; None when the kernel's sources changed since the capture."""
+def measured_record(kernel: str):
+    """The kernel's committed ncu figures (profiles/traffic.json), or None when its sources
+    changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     rec = json.load(open(p)).get(kernel)
     if not rec or rec.get("sources_sha256") != kernel_sources_sha(kernel):
         return None
-    return rec["dram_bytes_per_launch"] * units / rec["weights_per_launch"]
+    return rec
+
+
+def measured_traffic(kernel: str, units: int):
+    """DRAM bytes per launch from the committed ncu capture, scaled to `units` weights."""
+    rec = measured_record(kernel)
+    return None if rec is None else rec["dram_bytes_per_launch"] * units / rec["weights_per_launch"]
+
+
+def issue_roofline(kernel: str, units: int, seconds: float, sm_mhz):
+    """The instruction-issue roofline beside the HBM one: lane-instructions per weight from the
+    committed ncu capture (warp instructions x 32), issued per second, against SMs x 4 schedulers
+    x 32 lanes x the SM clock sampled during the timed region."""
+    import torch
+    rec = measured_record(kernel)
+    if rec is None or "warp_instructions_per_launch" not in rec or not sm_mhz:
+        return None
+    per_weight = 32.0 * rec["warp_instructions_per_launch"] / rec["weights_per_launch"]
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    peak = sms * 4 * 32 * sm_mhz * 1e6
+    achieved = per_weight * units / seconds
+    return {"bound": "issue", "lane_instr_per_weight": per_weight, "achieved": achieved,
+            "peak": peak, "unit": "lane-instr/s", "frac": achieved / peak, "sms": sms,
+            "sm_mhz": sm_mhz, "source": "warp instructions of the committed ncu capture"}
 
 
 def measured_peaks() -> dict:
@@ -303,7 +326,7 @@ def run_ours(args):
         "ms_per_step": mean_s * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8->bf16", "data": "synthetic",
         "config": {"workload": "Int8 8192x8192 Laplace(0,0.01) clip 6b, H=2.0 bits, 64 KiB "
-                               f"chunks, 128 streams, run 8, {wl.prob_bits}-bit table -> bf16",
+                               f"chunks, {wl.streams} streams, run 8, {wl.prob_bits}-bit table -> bf16",
                    "params_per_gpu": numel, "compressed_bytes": t.compressed_bytes,
                    "bits_per_param": 8 * t.compressed_bytes / numel,
                    "l2": "flushed between steps (256 MiB write)", "parallelism": f"replicas x{world}"},
@@ -324,6 +347,8 @@ def run_ours(args):
         "clocks": clk.summary(),
         "also": also,
     }
+    line["issue_roofline"] = issue_roofline("rans_decode_kernel", numel, mean_s,
+                                            line["clocks"].get("sm_mhz"))
     if not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(h, numel)
     print(json.dumps(line), flush=True)

@@ -12,8 +12,8 @@ from ._lib import (EQ_DEV_BAD_CODE, EQ_DEV_CORRUPT_STATE, EQ_DEV_COUNT_MISMATCH,
                    EQ_DEV_OVERRUN, EQ_DEV_TIMEOUT, EQ_SYM_E4M3, EQ_SYM_INT8, EQ_TABLE_HUFF,
                    EQ_TABLE_RANS, EQ_TABLE_RANS8_E4M3, EQ_TABLE_RANS8_INT8, EQ_TABLE_RANS_PAIR_E4M3,
                    EQ_TABLE_RANS_PAIR_INT8, EXPORTS, EqError, lib)
-from .api import (DeviceHuff, DeviceHuffInt, DeviceRans, bf16_bits, build_tables,  # noqa: F401
-                  decode, decode_gemv, histogram_device, huff_bf16_decode, huff_int_decode,
+from .api import (DeviceHuff, DeviceHuffInt, DeviceRans, PinnedRans, bf16_bits, build_tables,  # noqa: F401
+                  decode, decode_from_host, decode_gemv, histogram_device, huff_bf16_decode, huff_int_decode,
                   mlp_decode, selftest_bounded_wait,
                   mlp_scratch_bytes, new_status, normalize_freqs,
                   quantize_device, rans_encode_device, table_bytes)

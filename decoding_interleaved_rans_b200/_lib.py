@@ -20,7 +20,7 @@ EQ_TABLE_RANS8_E4M3, EQ_TABLE_RANS8_INT8 = 5, 6
 EQ_ABI_VERSION = 3
 
 # every exported function of include/eq.h and include/eq_encode.h
-EXPORTS = ("eq_table_bytes", "eq_build_tables", "eq_decode", "eq_decode_gemv",
+EXPORTS = ("eq_table_bytes", "eq_build_tables", "eq_decode", "eq_decode_from_host", "eq_decode_gemv",
            "eq_huff_bf16_decode", "eq_huff_int_decode", "eq_mlp_scratch_bytes", "eq_mlp_decode", "eq_mlp_decode_noalloc", "eq_selftest_bounded_wait",
            "eq_status_string",
            "eq_abi_version", "eq_quantize_host", "eq_super_weights_host", "eq_quantize_excluding_host",
@@ -86,6 +86,7 @@ def lib() -> C.CDLL:
                 "eq_table_bytes": (C.c_size_t, [i32]),
                 "eq_build_tables": (i32, [i32, p, u32, p, p]),
                 "eq_decode": (i32, [p, u32, p, p, p]),
+                "eq_decode_from_host": (i32, [p, p, p, p, u64, p, u32, p, p, p, p]),
                 "eq_decode_gemv": (i32, [p, p, u32, p, p, p]),
                 "eq_huff_bf16_decode": (i32, [p, p, p, p]),
                 "eq_huff_int_decode": (i32, [p, p, p, p]),

@@ -246,6 +246,53 @@ def decode(tensors, outs=None, status=None, stream=None):
     return outs, status
 
 
+@dataclass
+class PinnedRans:
+    """A coded weight's arrays in pinned host memory, the source of decode_from_host."""
+    states: torch.Tensor    # int32 [num_chunks * streams]
+    word_off: torch.Tensor  # int64 [units + 1]
+    words: torch.Tensor     # int16, padded to a multiple of 8 words
+    scales: torch.Tensor    # int16 (bf16 bits) [rows]
+    offsets: np.ndarray     # word_off as numpy, to find each piece's word range on the host
+
+    @classmethod
+    def from_host(cls, h) -> "PinnedRans":
+        words = np.ascontiguousarray(h.words, dtype=np.uint16)
+        if words.size % 8 or words.size == 0:
+            words = np.concatenate([words, np.zeros(8 - words.size % 8, np.uint16)])
+        pin = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).pin_memory()  # noqa: E731
+        return cls(pin(np.asarray(h.states, np.uint32), np.int32),
+                   pin(np.asarray(h.word_off, np.uint64), np.int64), pin(words, np.int16),
+                   pin(np.asarray(h.scales, np.uint16), np.int16),
+                   np.asarray(h.word_off, np.uint64).copy())
+
+    def h2d_bytes(self) -> int:
+        return sum(x.numel() * x.element_size() for x in (self.states, self.word_off, self.words, self.scales))
+
+
+def decode_from_host(t: DeviceRans, src: PinnedRans, out: torch.Tensor, status=None, stream=None,
+                     pieces: int = 1, copy_stream=None):
+    """eq_decode_from_host: decode a coded weight straight from pinned host memory.  Its arrays
+    are copied into the device container t (same layout, table already built) piece by piece on
+    copy_stream, each piece a run of whole chunks ending on a row boundary, and each piece
+    decodes on `stream` as soon as its copy has landed.  Returns (out, status)."""
+    dev = t.words.device
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    if copy_stream is None:
+        copy_stream = torch.cuda.Stream(dev)
+    if status is None:
+        status = new_status(dev)
+    assert out.dtype == torch.bfloat16 and out.is_contiguous() and out.numel() == t.numel
+    assert t.words.numel() >= src.words.numel()
+    d = t.desc()
+    L.check(L.lib().eq_decode_from_host(C.byref(d), _ptr(src.states), _ptr(src.word_off),
+                                        _ptr(src.words), src.words.numel(), _ptr(src.scales),
+                                        int(pieces), _ptr(out), _ptr(status), _stream(stream),
+                                        _stream(copy_stream)), "eq_decode_from_host")
+    return out, status
+
+
 def decode_gemv(t: DeviceRans, x: torch.Tensor, y=None, status=None, stream=None):
     """eq_decode_gemv: y[b] = W x[b] with W decoded on chip.  x bf16 [batch, cols]."""
     assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape[-1] == t.cols

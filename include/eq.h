@@ -212,6 +212,26 @@ eq_status eq_decode(const eq_rans_tensor *ts, uint32_t n_tensors, uint16_t *cons
                     uint32_t *d_status, void *stream);
 
 /*
+ * eq_decode of one tensor whose coded arrays are in host memory (pinned, for the copies to
+ * overlap).  No counterpart in the pages, which keep the coded weights in GPU memory
+ * ("Float8@2bits" summary, "Decodificacion en Tiempo de Inferencia"); this is the offloaded case
+ * the DFloat11 page compares against.  The host arrays h_states [num_chunks * streams],
+ * h_word_off [num_chunks * streams / 32 + 1], h_words [n_words] and h_scales [rows] are copied
+ * into the device arrays *t points at (same layout; t->words must hold n_words words, the rest
+ * as in eq_rans_tensor) piece by piece on copy_stream, each piece a run of whole chunks ending on
+ * a row boundary; each piece decodes on `stream` as soon as its copy has landed, while the next
+ * one is copied.  pieces: how many (1 = copy everything, then decode); a tensor with super
+ * weights, or whose chunks end on a row boundary only at the end, goes in one piece.  copy_stream
+ * may equal stream (nothing then overlaps).  The call returns once everything is enqueued; the
+ * host arrays must stay valid until the stream's work is done.  Errors as eq_decode;
+ * EQ_ERR_ARG for null host pointers or n_words below the last word offset.
+ */
+eq_status eq_decode_from_host(const eq_rans_tensor *t, const uint32_t *h_states,
+                              const uint64_t *h_word_off, const uint16_t *h_words, uint64_t n_words,
+                              const uint16_t *h_scales, uint32_t pieces, uint16_t *d_out,
+                              uint32_t *d_status, void *stream, void *copy_stream);
+
+/*
  * y[b][r] = sum_c W[r][c] * x[b][c] for b < batch, with W decoded from its rANS stream on chip
  * and never written to memory ("Float8@2bits" summary, closing section: fused decompression
  * kernels are the next step; the decoded values are consumed where they are produced).  W is

@@ -186,18 +186,21 @@ struct Staged {
   uint32_t w[17];
 };
 
+// NW: words read (16 for any segment; 8 when every lane of the warp holds at most 32 values)
+template <uint32_t NW>
 __device__ __forceinline__ void stage_read(const uint32_t *col, uint32_t T, uint32_t cnt, Staged &st) {
   const uint32_t nw = (cnt + 3) >> 2;
 #pragma unroll
-  for (uint32_t i = 0; i < 16; ++i) st.w[i] = i < nw ? col[i * T] : 0u;
-  st.w[16] = 0u;
+  for (uint32_t i = 0; i < NW; ++i) st.w[i] = i < nw ? col[i * T] : 0u;
+  st.w[NW] = 0u;
 }
 
+template <uint32_t NW>
 __device__ __forceinline__ void stage_write(uint8_t *ebuf, uint32_t D, uint32_t cnt, const Staged &st) {
   const uint32_t a = D & 3u, sh = 8 * a, nd = (a + cnt + 3) >> 2;
   uint32_t *dst = reinterpret_cast<uint32_t *>(ebuf + (D - a));
 #pragma unroll
-  for (uint32_t j = 0; j < 17; ++j) {
+  for (uint32_t j = 0; j < NW + 1; ++j) {
     if (j < nd) {
       // destination word j holds source bytes 4j - a .. 4j - a + 3
       const uint32_t prev = j ? st.w[j - 1] : 0u;
@@ -273,7 +276,10 @@ __global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_consta
     // the values leave this thread's column for registers now: the scan's barriers then also
     // order every column read before the compacting writes below
     Staged stg;
-    stage_read(reinterpret_cast<const uint32_t *>(ebuf) + tid, T, cnt, stg);
+    // the common case (every lane of the warp at most 32 values) stages half the words
+    const bool small = __all_sync(0xFFFFFFFFu, cnt <= 32);
+    if (small) stage_read<8>(reinterpret_cast<const uint32_t *>(ebuf) + tid, T, cnt, stg);
+    else stage_read<16>(reinterpret_cast<const uint32_t *>(ebuf) + tid, T, cnt, stg);
     const uint64_t o0 = __ldg(P.block_out + b), o1 = __ldg(P.block_out + b + 1);  // in flight
     // ---- block-wide exclusive scan of the counts ----
     uint32_t incl = cnt;
@@ -311,7 +317,10 @@ __global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_consta
     // ---- stage 2: every thread moves its values to their block positions (shifted so that
     //      8-aligned outputs are 8-aligned in shared memory) ----
     const uint32_t shift = uint32_t(o0 & 7);
-    if (off + cnt <= m) stage_write(ebuf, shift + off, cnt, stg);
+    if (off + cnt <= m) {
+      if (small) stage_write<8>(ebuf, shift + off, cnt, stg);
+      else stage_write<16>(ebuf, shift + off, cnt, stg);
+    }
     __syncthreads();
 
     // ---- merge with PackedSignMantissa and write the block's span ----

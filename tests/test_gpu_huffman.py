@@ -69,6 +69,25 @@ def test_all_exponents_and_long_codes(eq, orc):
     assert st == 0 and np.array_equal(out, w)
 
 
+def test_warps_with_short_and_long_segments(eq, orc):
+    """Regions of ~2.6-bit exponent codes (about 24 values a 64-bit segment) alternate with runs
+    of one exponent (1-bit codes, 64 values a segment), so some warps stage at most 32 values per
+    lane and others more, and the boundaries fall inside warps and blocks."""
+    rng = np.random.default_rng(44)
+    parts = []
+    for i in range(9):
+        n = int(rng.integers(3000, 40000))
+        if i % 2 == 0:
+            parts.append(synth.bf16_normal(1, n, 0.015, 440 + i)[0])
+        else:
+            parts.append(np.full(n, 0x3C10, np.uint16) | (rng.integers(0, 2, n).astype(np.uint16) << 15))
+    w = np.concatenate(parts)
+    for tpb in (64, 256):
+        h = orc.huff_encode_bf16(w, threads_per_block=tpb)
+        out, st = run(eq, h)
+        assert st == 0 and np.array_equal(out, w), tpb
+
+
 def test_single_exponent(eq, orc):
     w = np.full(5000, 0x3F80, np.uint16)
     w[::3] = 0xBF81

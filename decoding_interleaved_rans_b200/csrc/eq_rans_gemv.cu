@@ -153,12 +153,32 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
   uint32_t row_local = 0;
   float sc = bf16_bits_to_float(P.scales[row0]);
   uint32_t q = R.off0;
+  // At batch 1 the ring work (overrun check, refill, wait) runs only once q reaches q_next; with
+  // more accumulators the registers go to them (this bookkeeping spilled) and the checks run
+  // every round.
+  constexpr bool kQuiet = BMAX == 1;
+  const uint32_t q_end = R.off0 + 2 * nwords;
+  uint32_t q_next = 0;
 
   for (uint32_t r = 0; r < rounds; ++r) {
     const bool act = r * S + lane < runs;
-    uint32_t pr[4];  // the round's 8 symbols as 4 pairs (7-bit tables: their values, bf16x2)
+    uint32_t pr[4];  // the round's 8 symbols as 4 pairs (8/7-bit tables: their values, bf16x2)
     if (single) {
       pr[0] = pr[1] = pr[2] = pr[3] = single_pair<FMT, PB>(hdr.single_sym);
+    } else if constexpr (kQuiet) {
+      if (q >= q_next) {
+        if (q > q_end) {
+          status |= EQ_DEV_OVERRUN;
+          break;
+        }
+        R.round_refill(q, lane);
+        if (!R.round_wait(q)) {
+          status |= EQ_DEV_TIMEOUT;
+          break;
+        }
+        q_next = R.quiet_until(q_end);
+      }
+      round_pairs<PB>(pr, x, act, lut, smem, R, q, lt);
     } else {
       if (!R.round_wait(q)) {
         status |= EQ_DEV_TIMEOUT;

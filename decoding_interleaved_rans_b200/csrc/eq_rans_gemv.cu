@@ -41,28 +41,33 @@ struct GemvParams {
   uint32_t rows, cols, chunk_symbols, rows_per_chunk, rounds_per_row, batch, warps;
 };
 
-__device__ __forceinline__ float lo_bf16(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float hi_bf16(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-__device__ __forceinline__ float2 bf16x2_f2(uint32_t v) { return make_float2(lo_bf16(v), hi_bf16(v)); }
+// a.x += lo(w) * lo(x), a.y += hi(w) * hi(x): fp32 FMAs that take their factors as bf16 halves
+// of a register (no conversion; the product of two bf16 is exact, so each is the same single
+// rounding as an fp32 FMA of the converted factors)
+__device__ __forceinline__ void fma_bf16x2(float2 &a, uint32_t w, uint32_t x) {
+  asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+      "mov.b32 {wl, wh}, %2;\n\t"
+      "mov.b32 {xl, xh}, %3;\n\t"
+      "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+      "fma.rn.f32.bf16 %1, wh, xh, %1;\n\t}"
+      : "+f"(a.x), "+f"(a.y)
+      : "r"(w), "r"(x));
+}
 
 // acc[b] += w[i] * x[b][col + i] over one run of 8 weights (packed bf16 pairs), the even columns
-// in acc[b].x and the odd ones in acc[b].y: two-wide fp32 FMAs, half the instructions and half
-// the dependency chain of one running sum
+// in acc[b].x and the odd ones in acc[b].y (two independent sums: half the dependency chain)
 template <int BMAX>
 __device__ __forceinline__ void fma_run(float2 (&acc)[BMAX], uint2 wa, uint2 wb, const uint16_t *x,
                                         uint32_t cols, uint32_t col, uint32_t batch) {
-  const float2 w01 = bf16x2_f2(wa.x), w23 = bf16x2_f2(wa.y), w45 = bf16x2_f2(wb.x),
-               w67 = bf16x2_f2(wb.y);
 #pragma unroll
   for (int b = 0; b < BMAX; ++b) {
     if (b < int(batch)) {
       const uint4 xv = __ldg(reinterpret_cast<const uint4 *>(x + size_t(b) * cols + col));
       float2 a = acc[b];
-      a = __ffma2_rn(w01, bf16x2_f2(xv.x), a);
-      a = __ffma2_rn(w23, bf16x2_f2(xv.y), a);
-      a = __ffma2_rn(w45, bf16x2_f2(xv.z), a);
-      a = __ffma2_rn(w67, bf16x2_f2(xv.w), a);
+      fma_bf16x2(a, wa.x, xv.x);
+      fma_bf16x2(a, wa.y, xv.y);
+      fma_bf16x2(a, wb.x, xv.z);
+      fma_bf16x2(a, wb.y, xv.w);
       acc[b] = a;
     }
   }

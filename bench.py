@@ -688,6 +688,25 @@ def profile_kernel(kind: str, launches: int = 5):
         y = torch.empty(1, t.rows, dtype=torch.float32, device=dev)
         st = eq.new_status(dev)
         fn = lambda: eq.decode_gemv(t, x, y, st)  # noqa: E731
+    elif kind == "decode12":
+        # one LLaMA-2-7B-shaped gate projection (11008 x 4096, N(0, 0.02) with 1% x 8 outliers),
+        # E4M3, 12-bit table: the decode of the model-stack line
+        spec = next(s for s in synth.WORKLOADS["llama2_7b"].tensors if s.rows == 11008)
+        sym, sc = eq.codec.quantize(spec.generate(), eq.EQ_SYM_E4M3)
+        t = eq.DeviceRans.upload(eq.codec.rans_encode(sym, sc, eq.EQ_SYM_E4M3, 65536, 128, 8), dev)
+        out = torch.empty(t.rows, t.cols, dtype=torch.bfloat16, device=dev)
+        st = eq.new_status(dev)
+        fn = lambda: eq.decode([t], [out], st)  # noqa: E731
+    elif kind == "gemv7":
+        # the ~2-bit Int8 weight, one row per chunk, 7-bit table, batch 1
+        wl = synth.WORKLOADS["int8_8k"]
+        sym, sc = eq.codec.quantize(wl.tensors[0].generate(), eq.EQ_SYM_INT8, wl.int8_div)
+        t = eq.DeviceRans.upload(eq.codec.rans_encode(sym, sc, eq.EQ_SYM_INT8, 8192, 32, 8,
+                                                      prob_bits=7), dev)
+        x = torch.randn(1, t.cols, device=dev).to(torch.bfloat16)
+        y = torch.empty(1, t.rows, dtype=torch.float32, device=dev)
+        st = eq.new_status(dev)
+        fn = lambda: eq.decode_gemv(t, x, y, st)  # noqa: E731
     else:
         raise SystemExit(f"unknown kernel {kind}")
     for _ in range(launches):
@@ -699,7 +718,8 @@ def profile_kernel(kind: str, launches: int = 5):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--profile-kernel", default=None, choices=["decode", "huff", "gemv"],
+    ap.add_argument("--profile-kernel", default=None,
+                    choices=["decode", "huff", "gemv", "decode12", "gemv7"],
                     help="launch one kernel a few times and exit (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)

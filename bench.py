@@ -358,6 +358,14 @@ def run_ours(args):
     }
     line["issue_roofline"] = issue_roofline("rans_decode_kernel", numel, mean_s,
                                             line["clocks"].get("sm_mhz"))
+    # the same for the lines whose kernel and kind of weight the other captures cover
+    for e in also:
+        if e["what"].startswith("DFloat11 bf16 decode"):
+            e["issue_roofline"] = issue_roofline("huff_decode_kernel", e["params"], e["ms"] / 1e3,
+                                                 line["clocks"].get("sm_mhz"))
+        elif e["what"] == "fused decode+GEMV, 13B MLP gate/up/down, batch 1":
+            e["issue_roofline"] = issue_roofline("rans_gemv_kernel", e["params"], e["ms"] / 1e3,
+                                                 line["clocks"].get("sm_mhz"))
     if not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(h, numel)
     print(json.dumps(line), flush=True)

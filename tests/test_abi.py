@@ -109,6 +109,32 @@ def test_gemv_and_huff_reject_bad_input_on_host(eq):
     assert L.eq_huff_bf16_decode(C.byref(h), C.c_void_p(1 << 20), C.c_void_p(1 << 20), None) in (1, 3)
 
 
+def test_decode_from_host_rejects_bad_input_on_host(eq):
+    """Argument checks before any copy or launch: no descriptor, a descriptor of another ABI
+    version, missing host arrays, a word count below the last offset (read from the host
+    offsets), a misaligned output."""
+    import numpy as np
+    L = eq.lib()
+    fake = C.c_void_p(1 << 20)
+    good = eq._lib.RansTensorDesc(eq._lib.EQ_ABI_VERSION, 2, 4, 64, 7, 64, 32, 8, 4, 1 << 20,
+                                  1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    states = np.zeros(4 * 32, np.uint32)
+    word_off = np.arange(5, dtype=np.uint64) * 8  # four substreams of 8 words
+    words = np.zeros(32, np.uint16)
+    scales = np.zeros(4, np.uint16)
+    ptr = lambda a: C.c_void_p(a.ctypes.data)  # noqa: E731
+    args = lambda d, st, wo, w, nw, sc, out: (C.byref(d) if d is not None else None, st, wo, w, nw,  # noqa: E731
+                                              sc, 1, out, fake, None, None)
+    assert L.eq_decode_from_host(*args(None, ptr(states), ptr(word_off), ptr(words), 32, ptr(scales), fake)) == 1
+    bad = eq._lib.RansTensorDesc(eq._lib.EQ_ABI_VERSION + 1, 2, 4, 64, 7, 64, 32, 8, 4, 1 << 20,
+                                 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    assert L.eq_decode_from_host(*args(bad, ptr(states), ptr(word_off), ptr(words), 32, ptr(scales), fake)) == 1
+    assert L.eq_decode_from_host(*args(good, None, ptr(word_off), ptr(words), 32, ptr(scales), fake)) == 1
+    assert L.eq_decode_from_host(*args(good, ptr(states), ptr(word_off), ptr(words), 31, ptr(scales), fake)) == 1
+    assert L.eq_decode_from_host(*args(good, ptr(states), ptr(word_off), ptr(words), 32, ptr(scales),
+                                       C.c_void_p((1 << 20) + 2))) == 1
+
+
 class _FakeDev:
     """Stands in for a device tensor: only its address is used, and only by host validation."""
 

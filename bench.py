@@ -686,14 +686,16 @@ def profile_kernel(kind: str, launches: int = 5):
         ob = torch.empty(dh.n, dtype=torch.bfloat16, device=dev)
         st = eq.new_status(dev)
         fn = lambda: eq.huff_bf16_decode(dh, ob, st)  # noqa: E731
-    elif kind == "gemv":
+    elif kind in ("gemv", "gemv16"):
+        # the 13B MLP down projection, batch 1 (CUDA cores) or 16 (tensor-core tile)
+        batch = 16 if kind == "gemv16" else 1
         wl = synth.WORKLOADS["mlp_13b"]
         spec = wl.tensors[2]
         sym, sc = eq.codec.quantize(spec.generate(), eq.EQ_SYM_E4M3)
         t = eq.DeviceRans.upload(eq.codec.rans_encode(sym, sc, eq.EQ_SYM_E4M3, wl.chunk_for(spec),
                                                       wl.streams, wl.run), dev)
-        x = torch.randn(1, t.cols, device=dev).to(torch.bfloat16)
-        y = torch.empty(1, t.rows, dtype=torch.float32, device=dev)
+        x = torch.randn(batch, t.cols, device=dev).to(torch.bfloat16)
+        y = torch.empty(batch, t.rows, dtype=torch.float32, device=dev)
         st = eq.new_status(dev)
         fn = lambda: eq.decode_gemv(t, x, y, st)  # noqa: E731
     elif kind == "decode12":
@@ -727,7 +729,7 @@ def profile_kernel(kind: str, launches: int = 5):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-kernel", default=None,
-                    choices=["decode", "huff", "gemv", "decode12", "gemv7"],
+                    choices=["decode", "huff", "gemv", "gemv16", "decode12", "gemv7"],
                     help="launch one kernel a few times and exit (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)

@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(512, 3) huff_decode_kernel(const __grid_consta
   report(P.status, err);
 }
 
-static bool g_huff_attr[64][2];
+static std::atomic<bool> g_huff_attr[64][2];  // device, integer codes
 
 // validation and launch shared by the DFloat11 and the integer decoders
 template <int MODE>
@@ -391,12 +391,9 @@ static eq_status huff_launch(HuffParams &P, uint64_t n, uint64_t total_bits,
   const uint64_t blocks = (threads + T - 1) / T;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  if (!g_huff_attr[dev][MODE]) {
-    if (cudaFuncSetAttribute(huff_decode_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(huff_smem_bytes(512))) != cudaSuccess)
-      return EQ_ERR_CUDA;
-    g_huff_attr[dev][MODE] = true;
-  }
+  if (smem_optin_once(g_huff_attr[dev][MODE], reinterpret_cast<const void *>(huff_decode_kernel<MODE>),
+                      huff_smem_bytes(512)) != EQ_OK)
+    return EQ_ERR_CUDA;
   // persistent blocks: as many as fit on the device at once, each walking many blocks
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, huff_decode_kernel<MODE>, int(T),

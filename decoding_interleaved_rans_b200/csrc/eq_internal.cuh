@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "eq.h"
 
 namespace eq {
@@ -95,6 +97,18 @@ inline eq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EQ_OK : 
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int device_sm_count();  // SMs of the current device (cached per device)
+
+// A kernel's opt-in to more than 48 KiB of dynamic shared memory, set once per (device, kernel)
+// flag.  Callers may issue library calls from several host threads at once: the flag is atomic,
+// and two threads that both find it clear both make the (idempotent) attribute call.
+inline eq_status smem_optin_once(std::atomic<bool> &done, const void *fn, size_t bytes) {
+  if (done.load(std::memory_order_acquire)) return EQ_OK;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes)) !=
+      cudaSuccess)
+    return EQ_ERR_CUDA;
+  done.store(true, std::memory_order_release);
+  return EQ_OK;
+}
 
 // floor(n / d) for n < 2^40 and 1 <= d < 2^32 as __umul64hi(n, m) with m = ceil(2^64 / d).
 inline uint64_t div_magic(uint64_t d) { return d <= 1 ? 0 : (~0ull) / d + 1; }

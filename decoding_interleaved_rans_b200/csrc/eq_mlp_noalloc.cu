@@ -11,8 +11,6 @@
 // There is one array per device, shared by every call on that device: calls whose work may
 // overlap on the GPU (unordered streams) race on it.  Nothing in it needs to start at zero:
 // each call writes every element it later reads.
-#include <mutex>
-
 #include "eq_internal.cuh"
 
 namespace eq {
@@ -35,22 +33,19 @@ constexpr uint64_t kNoallocBytes = 2 * round256(uint64_t(EQ_MLP_NOALLOC_MAX_ELEM
 
 __device__ __align__(256) unsigned char mlp_noalloc_scratch[kNoallocBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex scratch_mu;
-void *scratch_addr[kMaxDevices];  // the array's address on each device, looked up once
-
-// The array's address on the current device (the device the call's stream belongs to).
-eq_status scratch_on_current_device(unsigned char **out) {
-  int dev = -1;
+// The array's address on the device of the call's stream, which must be the current device
+// (the array exists once per device; a stream of another device gets EQ_ERR_ARG).  The address is
+// looked up on every call rather than cached: cudaGetSymbolAddress is a host-side lookup that
+// allocates nothing, and a fresh lookup stays right when the device's context has been reset and
+// the module loaded again at another address.
+eq_status scratch_for_stream(cudaStream_t stream, unsigned char **out) {
+  int dev = -1, stream_dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return EQ_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return EQ_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(scratch_mu);
-  if (!scratch_addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, mlp_noalloc_scratch) != cudaSuccess || !p) return EQ_ERR_CUDA;
-    scratch_addr[dev] = p;
-  }
-  *out = static_cast<unsigned char *>(scratch_addr[dev]);
+  if (cudaStreamGetDevice(stream, &stream_dev) != cudaSuccess) return EQ_ERR_CUDA;
+  if (stream_dev != dev) return EQ_ERR_ARG;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, mlp_noalloc_scratch) != cudaSuccess || !p) return EQ_ERR_CUDA;
+  *out = static_cast<unsigned char *>(p);
   return EQ_OK;
 }
 
@@ -69,7 +64,7 @@ extern "C" eq_status eq_mlp_decode_noalloc(const eq_rans_tensor *gate, const eq_
   const uint64_t inter = gate->rows;
   if (inter * batch > EQ_MLP_NOALLOC_MAX_ELEMS) return EQ_ERR_UNSUPPORTED;
   unsigned char *p = nullptr;
-  s = scratch_on_current_device(&p);
+  s = scratch_for_stream(static_cast<cudaStream_t>(stream), &p);
   if (s != EQ_OK) return s;
   const uint64_t n = inter * batch;
   float *g = reinterpret_cast<float *>(p);

@@ -23,7 +23,9 @@
 
 namespace eq {
 
-constexpr int kMaxDecodeTensors = 192;
+// descriptors one launch carries as kernel parameters (120 bytes each, within the 32764-byte
+// parameter limit); a larger group goes in several launches of nearly equal size
+constexpr int kMaxDecodeTensors = 256;
 
 struct RansDesc {
   const uint32_t *states;
@@ -317,15 +319,17 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
   return EQ_OK;
 }
 
-static bool g_attr_set[64][2][2][3];  // device, symfmt, run == 8, table (12 / 8 / 7 bits)
+static std::atomic<bool> g_attr_set[64][2][2][3];  // device, symfmt, run == 8, table (12 / 8 / 7 bits)
 
-static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
-                              uint16_t *const *d_out, uint32_t *d_status, cudaStream_t st) {
-  const eq_rans_tensor &t0 = ts[idx[0]];
-  KernelFn fn = pick_kernel(t0.symfmt, t0.run, t0.prob_bits);
-  if (!fn) return EQ_ERR_UNSUPPORTED;
+// One launch over tensors idx[b, e) of one kernel variant.  Every size that shapes the launch
+// (warps per CTA, each tensor's share of the CTAs) comes from the units of these tensors alone.
+static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
+                             size_t b, size_t e, uint16_t *const *d_out, uint32_t *d_status,
+                             cudaStream_t st) {
+  const eq_rans_tensor &t0 = ts[idx[b]];
   uint64_t total_units = 0;
-  for (uint32_t i : idx) total_units += ts[i].num_chunks * (ts[i].streams / 32);
+  for (size_t q = b; q < e; ++q) total_units += ts[idx[q]].num_chunks * (ts[idx[q]].streams / 32);
+  if (total_units == 0) return EQ_OK;
   const uint64_t sms = uint64_t(device_sm_count());
   const bool pair = t0.prob_bits == kRansPairBits;
   uint32_t warps;
@@ -338,55 +342,62 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
     warps = 16;
     while (warps > 1 && (total_units + warps - 1) / warps < 4 * sms) warps >>= 1;
   }
-  const size_t smem = rans_smem_bytes(warps, t0.prob_bits);
+  static thread_local RansDecodeParams P;
+  P.status = d_status;
+  P.warps = warps;
+  P.n = 0;
+  uint64_t ctas = 0;
+  for (size_t q = b; q < e; ++q) {
+    const eq_rans_tensor &t = ts[idx[q]];
+    if (t.num_chunks == 0) continue;
+    RansDesc &D = P.d[P.n++];
+    D.states = t.states;
+    D.word_off = t.word_off;
+    D.words = t.words;
+    D.scales = t.scales;
+    D.table = static_cast<const uint32_t *>(t.tables);
+    D.out = d_out[idx[q]];
+    D.patch_idx = t.patch_idx;
+    D.patch_val = t.patch_val;
+    D.n_patch = t.n_patch;
+    D.numel = uint64_t(t.rows) * t.cols;
+    D.groups = t.streams / 32;
+    D.units = t.num_chunks * D.groups;
+    D.row_magic = div_magic(t.cols);
+    D.rows = t.rows;
+    D.cols = t.cols;
+    D.chunk_symbols = t.chunk_symbols;
+    uint64_t n_ctas = (D.units + warps - 1) / warps;
+    if (pair)  // at most the tensor's share of the SMs, at least one CTA
+      n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, D.units * sms / total_units));
+    D.cta_begin = uint32_t(ctas);
+    D.ctas = uint32_t(n_ctas);
+    ctas += n_ctas;
+  }
+  if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
+  fn<<<uint32_t(ctas), 32 * warps, rans_smem_bytes(warps, t0.prob_bits), st>>>(P);
+  return cuda_status(cudaGetLastError());
+}
+
+static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
+                              uint16_t *const *d_out, uint32_t *d_status, cudaStream_t st) {
+  const eq_rans_tensor &t0 = ts[idx[0]];
+  KernelFn fn = pick_kernel(t0.symfmt, t0.run, t0.prob_bits);
+  if (!fn) return EQ_ERR_UNSUPPORTED;
+  const bool pair = t0.prob_bits == kRansPairBits;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
-  bool &attr = g_attr_set[dev][t0.symfmt - 1][t0.run == 8][pair ? 2 : t0.prob_bits == 8];
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(rans_smem_bytes(pair ? 32 : 16, t0.prob_bits)));
-    if (e != cudaSuccess) return EQ_ERR_CUDA;
-    attr = true;
-  }
-  static thread_local RansDecodeParams P;
-  for (size_t b = 0; b < idx.size(); b += kMaxDecodeTensors) {
-    const size_t e = std::min(idx.size(), b + kMaxDecodeTensors);
-    P.status = d_status;
-    P.warps = warps;
-    P.n = 0;
-    uint64_t ctas = 0;
-    for (size_t q = b; q < e; ++q) {
-      const eq_rans_tensor &t = ts[idx[q]];
-      if (t.num_chunks == 0) continue;
-      RansDesc &D = P.d[P.n++];
-      D.states = t.states;
-      D.word_off = t.word_off;
-      D.words = t.words;
-      D.scales = t.scales;
-      D.table = static_cast<const uint32_t *>(t.tables);
-      D.out = d_out[idx[q]];
-      D.patch_idx = t.patch_idx;
-      D.patch_val = t.patch_val;
-      D.n_patch = t.n_patch;
-      D.numel = uint64_t(t.rows) * t.cols;
-      D.groups = t.streams / 32;
-      D.units = t.num_chunks * D.groups;
-      D.row_magic = div_magic(t.cols);
-      D.rows = t.rows;
-      D.cols = t.cols;
-      D.chunk_symbols = t.chunk_symbols;
-      uint64_t n_ctas = (D.units + warps - 1) / warps;
-      if (pair)  // at most the tensor's share of the SMs, at least one CTA
-        n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, D.units * sms / total_units));
-      D.cta_begin = uint32_t(ctas);
-      D.ctas = uint32_t(n_ctas);
-      ctas += n_ctas;
-    }
-    if (P.n == 0) continue;
-    if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
-    fn<<<uint32_t(ctas), 32 * warps, smem, st>>>(P);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return EQ_ERR_CUDA;
+  if (smem_optin_once(g_attr_set[dev][t0.symfmt - 1][t0.run == 8][pair ? 2 : t0.prob_bits == 8],
+                      reinterpret_cast<const void *>(fn),
+                      rans_smem_bytes(pair ? 32 : 16, t0.prob_bits)) != EQ_OK)
+    return EQ_ERR_CUDA;
+  // launches of nearly equal tensor counts, so that none is a small tail
+  const size_t n = idx.size();
+  const size_t parts = (n + kMaxDecodeTensors - 1) / kMaxDecodeTensors;
+  for (size_t p = 0; p < parts; ++p) {
+    const eq_status s = launch_part(fn, ts, idx, n * p / parts, n * (p + 1) / parts, d_out,
+                                    d_status, st);
+    if (s != EQ_OK) return s;
   }
   return EQ_OK;
 }

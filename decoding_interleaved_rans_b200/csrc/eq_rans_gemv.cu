@@ -496,7 +496,7 @@ static GemvFn pick_pb(uint32_t pb, uint32_t batch, bool tc) {
                                                          : pick_b<FMT, kRansPairBits>(batch, tc);
 }
 
-static bool g_gemv_attr[64][2][3][6];  // device, symfmt, table (12 / 8 / 7 bits), kernel instance
+static std::atomic<bool> g_gemv_attr[64][2][3][6];  // device, symfmt, table (12 / 8 / 7 bits), kernel instance
 
 }  // namespace eq
 
@@ -543,13 +543,10 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
   // one flag per kernel instance that pick_pb can return
   const int bi = tc ? 5 : bmax == 1 ? 0 : bmax == 2 ? 1 : bmax == 4 ? 2 : bmax == 8 ? 3 : 4;
-  bool &attr = g_gemv_attr[dev][t->symfmt - 1][pb == 12 ? 0 : pb == 8 ? 1 : 2][bi];
-  if (!attr) {
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(tc ? gemv_tc_smem_bytes(pb, pair ? 2 : 1) : rans_smem_bytes(max_warps, pb))) != cudaSuccess)
-      return EQ_ERR_CUDA;
-    attr = true;
-  }
+  if (smem_optin_once(g_gemv_attr[dev][t->symfmt - 1][pb == 12 ? 0 : pb == 8 ? 1 : 2][bi],
+                      reinterpret_cast<const void *>(fn),
+                      tc ? gemv_tc_smem_bytes(pb, pair ? 2 : 1) : rans_smem_bytes(max_warps, pb)) != EQ_OK)
+    return EQ_ERR_CUDA;
   GemvParams P;
   P.states = t->states;
   P.word_off = t->word_off;

@@ -201,16 +201,19 @@ static eq_status huff_tables_from_lengths(const uint32_t *len, HuffBuildArgs &a)
   return EQ_OK;
 }
 
-static int g_sm_count[64];
+static std::atomic<int> g_sm_count[64];  // 0 until looked up; any host thread may call
 
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
-  if (dev < 64 && g_sm_count[dev]) return g_sm_count[dev];
+  if (dev < 64) {
+    const int c = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     n = 148;
-  if (dev < 64) g_sm_count[dev] = n;
+  if (dev < 64) g_sm_count[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

@@ -290,10 +290,13 @@ eq_status eq_mlp_decode(const eq_rans_tensor *gate, const eq_rans_tensor *up,
  * for cudaMalloc / cudaFree, which can synchronise the device.  The scratch is one fixed device
  * array per device (placed by the CUDA runtime when it loads the library's code on that device)
  * sized for inter * batch <= EQ_MLP_NOALLOC_MAX_ELEMS (5 MiB); no allocating routine is called.
- * Larger sizes return EQ_ERR_UNSUPPORTED without launching.  The array's address on the current
- * device is looked up on the first call there.  Every call on a device shares the array, so
- * calls whose work may overlap on the GPU (streams not ordered with one another) race: order
- * them.  Nothing needs zeroing beforehand.  Arguments, layouts and other errors as eq_mlp_decode.
+ * Larger sizes return EQ_ERR_UNSUPPORTED without launching.  `stream` must belong to the current
+ * device (EQ_ERR_ARG otherwise): the array used is the current device's, and its address there is
+ * looked up on every call (a host-side lookup that allocates nothing; it also stays right after a
+ * device reset).  The first call on a device may load the library's code there, so make it before
+ * any stream capture.  Every call on a device shares the array, so calls whose work may overlap
+ * on the GPU (streams not ordered with one another) race: order them.  Nothing needs zeroing
+ * beforehand.  Arguments, layouts and other errors as eq_mlp_decode.
  */
 #define EQ_MLP_NOALLOC_MAX_ELEMS 524288u
 eq_status eq_mlp_decode_noalloc(const eq_rans_tensor *gate, const eq_rans_tensor *up,

@@ -1,7 +1,8 @@
 """GPU parity at the format's limits: the largest stream count (1024 = 32 groups per chunk), one
 group's word substream far longer than its ring (thousands of refills), empty tensors inside a
-grouped call, more tensors in one call than one launch's descriptor table holds, and a tensor
-whose chunks hold a single run."""
+grouped call, more tensors of one kernel variant in one call than one launch's descriptor table
+holds (256: the call is split into launches, each sized from its own tensors), a LLaMA-2-7B-shaped
+set of 224 tensors in one call, and a tensor whose chunks hold a single run."""
 import numpy as np
 import pytest
 import torch
@@ -58,9 +59,10 @@ def test_empty_tensors_in_a_grouped_call(eq, orc):
         assert np.array_equal(o, e)
 
 
-def test_more_tensors_than_one_launch_holds(eq, orc):
+def test_mixed_variants_in_one_call(eq, orc):
+    """200 tensors spread over four kernel variants (symbol format x table size)."""
     hosts, want = [], []
-    for i in range(200):  # one launch takes at most 192 descriptors
+    for i in range(200):
         fmt = orc.INT8 if i % 3 else orc.E4M3
         w = synth.normal(4, 256, 0.02, 300 + i)
         sym, sc = orc.quantize(w, fmt, 20.0)
@@ -70,6 +72,44 @@ def test_more_tensors_than_one_launch_holds(eq, orc):
     assert st == 0
     for o, e in zip(outs, want):
         assert np.array_equal(o, e)
+
+
+@pytest.mark.parametrize("pb,fmt,count", [(12, 1, 300), (7, 2, 290), (8, 2, 270)])
+def test_split_launch_of_one_variant(eq, orc, pb, fmt, count):
+    """More tensors of ONE kernel variant than a launch holds (256), so eq_decode splits them.
+    Sizes vary (1 to 40 chunks of 2 to 4 groups) so that each launch's warps per CTA and each
+    tensor's CTA share come from that launch's own units; every output is compared in full."""
+    hosts, want = [], []
+    rng = np.random.default_rng(count)
+    for i in range(count):
+        rows = int(rng.integers(1, 41)) * 16
+        w = synth.normal(rows, 1024, 0.02, 400 + i) if fmt == 1 else \
+            synth.laplace_clipped(rows, 1024, 0.01, 0.06, 400 + i)
+        sym, sc = orc.quantize(w, fmt, synth.INT8_DIV_LAPLACE_8K)
+        streams = 32 * int(rng.integers(2, 5))
+        hosts.append(orc.rans_encode(sym, sc, fmt, 16384, streams, 8, prob_bits=pb))
+        want.append(orc.dequant(sym, sc, fmt).ravel())
+    outs, st = decode(eq, hosts)
+    assert st == 0
+    for i, (o, e) in enumerate(zip(outs, want)):
+        assert np.array_equal(o, e), i
+
+
+def test_llama_shaped_224_tensors_in_one_call(eq, orc):
+    """The LLaMA-2-7B-shaped stack's 224 tensors (32 layers x q, k, v, o, gate, up, down) with
+    their rows cut by 64, coded as the full stack is (E4M3, 12-bit tables, 64 KiB chunks, 128
+    streams), decoded in one eq_decode call and compared in full."""
+    wl = synth.scaled(synth.WORKLOADS["llama2_7b"], row_div=64)
+    assert len(wl.tensors) == 224
+    hosts, want = [], []
+    for spec in wl.tensors:
+        sym, sc = orc.quantize(spec.generate(), orc.E4M3)
+        hosts.append(orc.rans_encode(sym, sc, orc.E4M3, wl.chunk_symbols, wl.streams, wl.run))
+        want.append(orc.dequant(sym, sc, orc.E4M3).ravel())
+    outs, st = decode(eq, hosts)
+    assert st == 0
+    for i, (o, e) in enumerate(zip(outs, want)):
+        assert np.array_equal(o, e), wl.tensors[i].name
 
 
 def test_chunks_of_a_single_run(eq, orc):

@@ -266,6 +266,16 @@ class PinnedRans:
                    pin(np.asarray(h.scales, np.uint16), np.int16),
                    np.asarray(h.word_off, np.uint64).copy())
 
+    @classmethod
+    def from_device(cls, t: "DeviceRans") -> "PinnedRans":
+        """Pinned host copies of a device container's coded arrays."""
+        def pin(x: torch.Tensor) -> torch.Tensor:
+            h = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+            h.copy_(x)
+            return h
+        wo = pin(t.word_off)
+        return cls(pin(t.states), wo, pin(t.words), pin(t.scales), wo.numpy().view(np.uint64).copy())
+
     def h2d_bytes(self) -> int:
         return sum(x.numel() * x.element_size() for x in (self.states, self.word_off, self.words, self.scales))
 

@@ -76,6 +76,12 @@ __device__ __forceinline__ uint32_t pair_dequant(uint32_t vals, uint32_t sc2, bo
   return o;
 }
 
+// the values (bf16x2, first in the low half) of two expanded 12-bit entries' second words (value
+// in bits 31..16)
+__device__ __forceinline__ uint32_t value_pair12(uint32_t w0, uint32_t w1) {
+  return __byte_perm(w0, w1, 0x7632u);
+}
+
 // the bf16 bits of a scale held as fp32 (converted exactly from bf16), in both halves
 __device__ __forceinline__ uint32_t scale_bf16x2(float sc) {
   return __byte_perm(__float_as_uint(sc), 0u, 0x3232u);

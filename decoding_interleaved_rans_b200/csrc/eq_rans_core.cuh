@@ -11,17 +11,25 @@ constexpr uint32_t kSegBytes = 512;  // one bulk copy; >= the 32 * 8 words a rou
 constexpr uint32_t kNumSeg = 4;
 constexpr uint32_t kRingBytes = kSegBytes * kNumSeg;
 constexpr uint32_t kRoundWords = 32 * 8;  // words a group reads at most per round of 8 steps
+// the 12-bit decode kernel's ring: 1 KiB copies, so that the ring work comes half as often
+constexpr uint32_t kSegBytesWide = 1024;
+constexpr uint32_t kRingBytesWide = kSegBytesWide * kNumSeg;
 
 #ifdef __CUDACC__
 
 // ------------------------------------------------------------------------------------------------
 // Per-warp word ring.  Byte offsets are counted from A, the 16-byte-aligned start of the
-// substream's span; segment s (bytes [s * 512, s * 512 + 512) of the span) lands in ring slot
-// s % 4, i.e. at ring byte (offset mod 2048).  Copies are issued by lane 0; every lane waits.
+// substream's span; segment s (bytes [s * SEG, s * SEG + SEG) of the span) lands in ring slot
+// s % 4, i.e. at ring byte (offset mod 4 * SEG).  Copies are issued by lane 0; every lane waits.
+// A slot is refilled only after the wait for its previous copy, so each of the four mbarriers has
+// at most one copy in flight.
 // ------------------------------------------------------------------------------------------------
-struct WordRing {
+template <uint32_t SEG>
+struct WordRingT {
+  static constexpr uint32_t kSeg = SEG;
+  static constexpr uint32_t kBytes = SEG * kNumSeg;
   unsigned char *buf;
-  uint32_t ring_off;  // buf - shared-memory base (a multiple of kRingBytes)
+  uint32_t ring_off;  // buf - shared-memory base (a multiple of kBytes)
   uint64_t *bar;
   const unsigned char *A;
   uint32_t off0;    // bytes from A to the first word
@@ -37,13 +45,13 @@ struct WordRing {
   __device__ __forceinline__ void issue(uint32_t lane) {
     if (lane == 0) {
       const uint32_t s = issued, slot = s % kNumSeg;
-      const uint32_t bytes = min(kSegBytes, span - s * kSegBytes);
+      const uint32_t bytes = min(SEG, span - s * SEG);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_expect_tx(&bar[slot], bytes);
-      bulk_g2s(buf + slot * kSegBytes, A + size_t(s) * kSegBytes, bytes, &bar[slot]);
+      bulk_g2s(buf + slot * SEG, A + size_t(s) * SEG, bytes, &bar[slot]);
     }
     ++issued;
-    refill_at = issued < nseg ? (issued - kNumSeg + 1) * kSegBytes : 0xFFFFFFFFu;
+    refill_at = issued < nseg ? (issued - kNumSeg + 1) * SEG : 0xFFFFFFFFu;
   }
 
   // point the ring at words [w0, w0 + nwords) and start the first copies
@@ -53,7 +61,7 @@ struct WordRing {
     A = reinterpret_cast<const unsigned char *>(reinterpret_cast<uintptr_t>(g) & ~uintptr_t(15));
     off0 = uint32_t(g - A);
     span = (off0 + 2 * nwords + 15u) & ~15u;
-    nseg = (span + kSegBytes - 1) / kSegBytes;
+    nseg = (span + SEG - 1) / SEG;
     issued = 0;
     ready = 0;
     ready_end = 0;
@@ -71,12 +79,12 @@ struct WordRing {
   // every byte below `end` (an offset from A) must have landed; false on timeout
   __device__ __forceinline__ bool wait_below(uint32_t end) {
     if (nseg == 0) return true;
-    const uint32_t last = min(nseg - 1, (end - 1) / kSegBytes);
+    const uint32_t last = min(nseg - 1, (end - 1) / SEG);
     while (ready <= last) {
       if (!wait_slot(ready % kNumSeg)) return false;
       ++ready;
     }
-    ready_end = ready * kSegBytes;
+    ready_end = ready * SEG;
     return true;
   }
 
@@ -103,7 +111,7 @@ struct WordRing {
 
   // hand out the slots of segments lying wholly below offset q
   __device__ __forceinline__ void refill(uint32_t q, uint32_t lane) {
-    const uint32_t cur = q / kSegBytes;
+    const uint32_t cur = q / SEG;
     if (issued < nseg && issued < cur + kNumSeg) {
       __syncwarp();
       do issue(lane);
@@ -121,9 +129,10 @@ struct WordRing {
   }
 
   __device__ __forceinline__ uint32_t word_at(uint32_t q) const {
-    return *reinterpret_cast<const uint16_t *>(buf + (q & (kRingBytes - 1)));
+    return *reinterpret_cast<const uint16_t *>(buf + (q & (kBytes - 1)));
   }
 };
+using WordRing = WordRingT<kSegBytes>;
 
 // ------------------------------------------------------------------------------------------------
 // Decode steps of the lane's state x.  q is the byte offset (from the ring's A) of the group's
@@ -175,6 +184,43 @@ __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, cons
   return e;
 }
 
+// One step with the decode kernel's expanded 12-bit table (entry i = {f, (i - cum) | value << 16},
+// 8 bytes; see decode_lut_bytes) at shared address `base`: x' = f * (x >> 12) + (slot - cum)
+// needs no field extraction but the mask of the low half.  Returns the entry's second word (its
+// high half: the symbol's value as bf16).
+template <bool FULL>
+__device__ __forceinline__ uint32_t rans_value_step(uint32_t &x, bool act, uint32_t base) {
+  uint32_t w1;
+  if constexpr (FULL) {
+    asm volatile(
+        "{\n\t.reg .b32 a, f, b, xs;\n\t"
+        "shl.b32 a, %0, 3;\n\t"
+        "and.b32 a, a, 32760;\n\t"
+        "add.u32 a, a, %2;\n\t"
+        "shr.u32 xs, %0, 12;\n\t"
+        "ld.shared.v2.u32 {f, %1}, [a];\n\t"
+        "and.b32 b, %1, 65535;\n\t"
+        "mad.lo.u32 %0, f, xs, b;\n\t}"
+        : "+r"(x), "=r"(w1)
+        : "r"(base));
+  } else {
+    uint32_t nx;
+    asm volatile(
+        "{\n\t.reg .b32 a, f, b, xs;\n\t"
+        "shl.b32 a, %2, 3;\n\t"
+        "and.b32 a, a, 32760;\n\t"
+        "add.u32 a, a, %3;\n\t"
+        "shr.u32 xs, %2, 12;\n\t"
+        "ld.shared.v2.u32 {f, %1}, [a];\n\t"
+        "and.b32 b, %1, 65535;\n\t"
+        "mad.lo.u32 %0, f, xs, b;\n\t}"
+        : "=r"(nx), "=r"(w1)
+        : "r"(x), "r"(base));
+    if (act) x = nx;
+  }
+  return w1;
+}
+
 // Two decode steps of a 7-bit stream with one pair-table lookup (layout in eq_internal.cuh):
 // x2 = F * (x >> 14) + B.  Returns the two symbols' values as bf16x2 (the first in the low half).
 template <bool FULL>
@@ -213,15 +259,84 @@ constexpr uint32_t kSymShift = PB;
 // A renormalisation point: every lane below 2^16 takes the group's next word, in lane order.
 // All lanes load (the others drop the word), which keeps the step free of branches; the load
 // stays inside the landed part of the ring (see round_wait).
-template <bool FULL>
+template <bool FULL, uint32_t RING = kRingBytes>
 __device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigned char *smem,
                                             uint32_t ring_off, uint32_t &q, uint32_t lt) {
   const bool need = (FULL || act) && x < kRansL;
   const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
-  const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (kRingBytes - 1)) | ring_off;
-  const uint32_t xr = mad_lo(x, 65536u, *reinterpret_cast<const uint16_t *>(smem + a));
-  x = need ? xr : x;
+  const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (RING - 1)) | ring_off;
+  const uint32_t w = *reinterpret_cast<const uint16_t *>(smem + a);
+  if (need) x = mad_lo(x, 65536u, w);
   q = mad_lo(__popc(m), 2u, q);
+}
+
+// One round of a 12-bit stream (run 8) in which every lane holds a run, with the decode kernel's
+// expanded table, as one PTX block: eight steps, each followed by its renormalisation point, and
+// the round's dequantisation (four bf16x2 multiplies of the entries' values by the row scale; for
+// tables without NaN codes).  One block leaves ptxas no moves or reloads between the steps.
+//   tb:   shared address of the expanded table;
+//   ring: shared address of this warp's word ring, a multiple of its size RING, so that a word's
+//         address is one mask-and-or of q + 2 * rank;
+//   lt:   the lanes below this one; sc2: the row scale's bf16 bits in both halves.
+// The lane's "needs a word" predicate feeds both the ballot and the predicated merge.
+#define EQ_R12_STEP(V)                                 \
+  "and.b32 t, %0, 4095;\n\t"                         \
+  "mad.lo.u32 a, t, 8, %6;\n\t"                      \
+  "shr.u32 xs, %0, 12;\n\t"                          \
+  "ld.shared.v2.u32 {f, " V "}, [a];\n\t"            \
+  "and.b32 t, " V ", 65535;\n\t"                     \
+  "mad.lo.u32 %0, f, xs, t;\n\t"                     \
+  "setp.lt.u32 p, %0, 65536;\n\t"                    \
+  "vote.sync.ballot.b32 m, p, 0xffffffff;\n\t"       \
+  "and.b32 r, m, %9;\n\t"                            \
+  "popc.b32 r, r;\n\t"                               \
+  "mad.lo.u32 a, r, 2, %1;\n\t"                      \
+  "and.b32 a, a, %10;\n\t"                           \
+  "or.b32 a, a, %8;\n\t"                             \
+  "ld.shared.u16 w, [a];\n\t"                        \
+  "@p mad.lo.u32 %0, %0, 65536, w;\n\t"              \
+  "popc.b32 m, m;\n\t"                               \
+  "mad.lo.u32 %1, m, 2, %1;\n\t"
+#define EQ_R12_PAIR(OUT)                               \
+  EQ_R12_STEP("va") EQ_R12_STEP("vb")                  \
+  "prmt.b32 va, va, vb, 0x7632;\n\t"                 \
+  "mul.rn.bf16x2 " OUT ", va, %7;\n\t"
+
+template <uint32_t RING>
+__device__ __forceinline__ uint4 rans_round12_full(uint32_t &x, uint32_t &q, uint32_t tb,
+                                                   uint32_t ring, uint32_t lt, uint32_t sc2) {
+  uint4 o;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 t, a, f, va, vb, xs, m, r, w;\n\t"
+      EQ_R12_PAIR("%2") EQ_R12_PAIR("%3") EQ_R12_PAIR("%4") EQ_R12_PAIR("%5")
+      "}"
+      : "+r"(x), "+r"(q), "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+      : "r"(tb), "r"(sc2), "r"(ring), "r"(lt), "n"(RING - 1));
+  return o;
+}
+#undef EQ_R12_PAIR
+#undef EQ_R12_STEP
+
+// A renormalisation point with the ring at absolute shared address `ring` (a multiple of RING):
+// the general form of the one in rans_round12_full, for rounds in which some lanes hold no run.
+template <bool FULL, uint32_t RING>
+__device__ __forceinline__ void rans_renorm_abs(uint32_t &x, bool act, uint32_t ring, uint32_t &q,
+                                                uint32_t lt) {
+  const bool need = (FULL || act) && x < kRansL;
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
+  const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (RING - 1)) | ring;
+  uint32_t w;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(w) : "r"(a));
+  if (need) x = mad_lo(x, 65536u, w);
+  q = mad_lo(__popc(m), 2u, q);
+}
+
+// the lane mask below this lane, read once into a register (a volatile read, so that it is not
+// re-read from the special register at every use)
+__device__ __forceinline__ uint32_t lanemask_lt_once() {
+  uint32_t m;
+  asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
 // one full step of a 12-bit stream (a renormalisation point after every step)
@@ -252,9 +367,10 @@ __device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {
 }
 
 // Init the rings' mbarriers (lane 0 of each warp) -- call before the block-wide sync.
-__device__ __forceinline__ void ring_init(WordRing &R, unsigned char *smem, unsigned char *rings,
+template <class Ring>
+__device__ __forceinline__ void ring_init(Ring &R, unsigned char *smem, unsigned char *rings,
                                           uint64_t *bars, uint32_t warp, uint32_t lane) {
-  R.buf = rings + warp * kRingBytes;
+  R.buf = rings + warp * Ring::kBytes;
   R.ring_off = uint32_t(R.buf - smem);
   R.bar = bars + warp * kNumSeg;
   R.phase = 0;
@@ -277,6 +393,21 @@ __host__ __device__ constexpr uint32_t rans_lut_bytes(uint32_t pb) {
 // shared memory of a CTA: the slot table, then one ring per warp, then the rings' barriers
 __host__ __device__ constexpr size_t rans_smem_bytes(uint32_t warps, uint32_t pb = 12) {
   return rans_lut_bytes(pb) + warps * (kRingBytes + kNumSeg * 8);
+}
+
+// The decode kernel's table: 12-bit tables are expanded on load to 8-byte entries {f, (slot -
+// cum) | value(symbol) << 16} (32 KiB), the 8- and 7-bit ones are used as they are.  Its rings:
+// 4 KiB (1 KiB copies) with 12-bit tables, placed at a shared address that is a multiple of their
+// size (up to one ring of slack), else 2 KiB right after the table.
+__host__ __device__ constexpr uint32_t decode_lut_bytes(uint32_t pb) {
+  return pb == 12 ? (8u << 12) : rans_lut_bytes(pb);
+}
+__host__ __device__ constexpr uint32_t decode_ring_bytes(uint32_t pb) {
+  return pb == 12 ? kRingBytesWide : kRingBytes;
+}
+__host__ __device__ constexpr size_t decode_smem_bytes(uint32_t warps, uint32_t pb) {
+  return decode_lut_bytes(pb) + (pb == 12 ? kRingBytesWide : 0) +
+         warps * (decode_ring_bytes(pb) + kNumSeg * 8);
 }
 
 }  // namespace eq

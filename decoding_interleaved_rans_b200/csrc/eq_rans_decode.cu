@@ -16,6 +16,7 @@
 //   * dequantisation (value * row scale, one rounding) happens in registers before the store.
 // Many tensors go in one launch (the pages decode all weights of a transformer block together).
 #include <algorithm>
+#include <type_traits>
 #include <vector>
 
 #include "eq_dequant.cuh"
@@ -60,12 +61,14 @@ static_assert(sizeof(RansDecodeParams) <= 32764, "kernel parameters above the la
 // renormalises after every step; an 8-bit one (G = 8) after positions 1, 3, 5 and 7, i.e. after
 // every second of its own steps, since each round gives it one whole run.
 // ------------------------------------------------------------------------------------------------
-template <bool FULL, int G, int FMT, uint32_t PB>
+template <bool FULL, int G, int FMT, uint32_t PB, bool MAYBE_NAN = true, class Ring>
 __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
                                              const uint32_t *lut, const unsigned char *smem,
-                                             const WordRing &R, uint32_t &q, uint32_t lt,
-                                             uint16_t *out, float sc, bool nan_codes) {
+                                             const Ring &R, uint32_t &q, uint32_t lt,
+                                             uint16_t *out, float sc, bool nan_codes_) {
   static_assert(PB == 12 || G == 8, "7- and 8-bit tables need whole runs of 8");
+  // MAYBE_NAN false: the table has no NaN code, and the checks compile away
+  const bool nan_codes = MAYBE_NAN && nan_codes_;
   if constexpr (PB == kRansPairBits) {  // one lookup per pair of steps
     uint32_t pv[4];  // the pairs' values (bf16x2)
 #pragma unroll
@@ -79,17 +82,36 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
           make_uint4(pair_dequant(pv[0], sc2, nan_codes), pair_dequant(pv[1], sc2, nan_codes),
                      pair_dequant(pv[2], sc2, nan_codes), pair_dequant(pv[3], sc2, nan_codes));
     }
+  } else if constexpr (PB == 12) {  // the expanded table: each entry carries the symbol's value
+    const uint32_t sc2 = scale_bf16x2(sc);
+    const uint32_t tb = smem_addr(smem);  // the expanded table starts the shared memory
+    const uint32_t ring = smem_addr(R.buf);
+    if constexpr (FULL && !MAYBE_NAN && G == 8) {
+      *reinterpret_cast<uint4 *>(out) = rans_round12_full<Ring::kBytes>(x, q, tb, ring, lt, sc2);
+    } else if constexpr (G == 8) {
+      uint32_t o[4];  // each pair dequantised as soon as both of its steps are done
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t va = rans_value_step<FULL>(x, act, tb);
+        rans_renorm_abs<FULL, Ring::kBytes>(x, act, ring, q, lt);
+        const uint32_t vb = rans_value_step<FULL>(x, act, tb);
+        rans_renorm_abs<FULL, Ring::kBytes>(x, act, ring, q, lt);
+        o[k] = pair_dequant(value_pair12(va, vb), sc2, nan_codes);
+      }
+      if (FULL || act) *reinterpret_cast<uint4 *>(out) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      const uint32_t v = rans_value_step<FULL>(x, act, tb);
+      rans_renorm_abs<FULL, Ring::kBytes>(x, act, ring, q, lt);
+      if (FULL || act) *out = uint16_t(pair_dequant(v >> 16, sc2, nan_codes));
+    }
   } else {
     uint32_t e[G];
 #pragma unroll
     for (int p = 0; p < G; ++p) {
       e[p] = rans_decode_step<FULL, PB>(x, act, lut);
-      if (PB == 12 || (p & 1)) rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
+      if (p & 1) rans_renorm<FULL>(x, act, smem, R.ring_off, q, lt);
     }
-    if (FULL || act) {
-      if constexpr (G == 8) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
-      else *out = dequant1<FMT>((e[0] >> kSymShift<PB>) & 0xFFu, sc);
-    }
+    if (FULL || act) *reinterpret_cast<uint4 *>(out) = dequant8<FMT, PB>(e, sc, nan_codes);
   }
 }
 
@@ -113,10 +135,10 @@ __device__ __forceinline__ uint32_t apply_patches(const RansDesc &D, uint64_t j0
   return __reduce_or_sync(0xFFFFFFFFu, bad);  // lane 0 reports the warp's status
 }
 
-template <int G, int FMT, uint32_t PB>
+template <int G, int FMT, uint32_t PB, class Ring>
 __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32_t *lut,
                                                  const unsigned char *smem, uint32_t flags,
-                                                 uint32_t single_sym, WordRing &R, uint64_t unit,
+                                                 uint32_t single_sym, Ring &R, uint64_t unit,
                                                  uint32_t lane) {
   const uint64_t chunk = unit / D.groups;
   const uint32_t g = uint32_t(unit - chunk * D.groups);
@@ -148,53 +170,71 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
 
   R.start(D.words, w0, nwords, lane);
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (flags & (kRansFlagNaN7F | kRansFlagNaNFF));
-  const uint32_t lt = lanemask_lt();
+  const uint32_t lt = lanemask_lt_once();
   // rounds in which all 32 lanes of this group hold a run
   const uint32_t full = runs >= 32 * g + 32 ? (runs - 32 * g - 32) / S + 1 : 0;
   uint32_t q = R.off0;
   // the lane's first output and its row; both advance by S runs per round
   uint64_t jrun = j0 + uint64_t(s) * G;
   const uint32_t step = S * G, cols = D.cols;
-  uint64_t row = div_by_magic(jrun, D.row_magic);
-  uint32_t col = uint32_t(jrun - row * cols);
+  uint32_t row = uint32_t(div_by_magic(jrun, D.row_magic));
+  uint32_t col = uint32_t(jrun - uint64_t(row) * cols);
   float sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
   uint16_t *out = D.out + jrun;
   // ring checks once per round (12-bit: up to 256 words a round), or once per two rounds
   // (8-bit: up to 128 words a round); round_wait covers 256 words and one more
   constexpr uint32_t kRoundsPerCheck = PB == 12 ? 1 : 2;
+  const uint32_t q_end = R.off0 + 2 * nwords;
+  uint32_t r0 = 0;
+
+  // One round's advance of the lane's output position, row and scale.  ONE_WRAP (rows of at
+  // least S * G symbols): a round crosses at most one row end, so a compare and a conditional
+  // update, no loop.
+  auto advance = [&](auto one_wrap) {
+    out += step;
+    col += step;
+    if constexpr (decltype(one_wrap)::value) {
+      if (col >= cols) {
+        col -= cols;
+        ++row;
+        sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+      }
+    } else if (col >= cols) {
+      do {
+        col -= cols;
+        ++row;
+      } while (col >= cols);
+      if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
+    }
+  };
   // The rounds in which every lane of the group holds a run, with no per-round tests.  The ring
   // work (overrun check, refill, wait) runs only once q reaches q_next; refill comes before the
-  // wait, so every segment a wait needs has been handed to the copy engine.
-  const uint32_t q_end = R.off0 + 2 * nwords;
-  uint32_t q_next = 0;
-  uint32_t r0 = 0;
-  for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
-    if (q >= q_next) {
-      if (q > q_end) {
-        status |= EQ_DEV_OVERRUN;
-        break;
+  // wait, so every segment a wait needs has been handed to the copy engine.  Instantiated for
+  // tables with and without NaN codes and for one or several row ends per round, so that none
+  // of those tests is left in the loop.
+  auto run_full = [&](auto maybe_nan, auto one_wrap) -> uint32_t {
+    uint32_t q_next = 0;
+    for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
+      // q is the same in every lane; the vote tells the compiler so (no reconvergence point)
+      if (__any_sync(0xFFFFFFFFu, q >= q_next)) {
+        if (q > q_end) return EQ_DEV_OVERRUN;
+        R.round_refill(q, lane);
+        if (!R.round_wait(q)) return EQ_DEV_TIMEOUT;
+        q_next = R.quiet_until(q_end);
       }
-      R.round_refill(q, lane);
-      if (!R.round_wait(q)) {
-        status |= EQ_DEV_TIMEOUT;
-        break;
-      }
-      q_next = R.quiet_until(q_end);
-    }
 #pragma unroll
-    for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
-      decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
-      out += step;
-      col += step;
-      if (col >= cols) {
-        do {
-          col -= cols;
-          ++row;
-        } while (col >= cols);
-        if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
+      for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
+        decode_round<true, G, FMT, PB, decltype(maybe_nan)::value>(D, x, true, lut, smem, R, q,
+                                                                   lt, out, sc, true);
+        advance(one_wrap);
       }
     }
-  }
+    return 0u;
+  };
+  using T = std::true_type;
+  using F = std::false_type;
+  if (nan_codes) status = step <= cols ? run_full(T{}, T{}) : run_full(T{}, F{});
+  else status = step <= cols ? run_full(F{}, T{}) : run_full(F{}, F{});
   if (!status) {  // the general loop below waits first: hand out the used-up slots
     if (q > q_end) status |= EQ_DEV_OVERRUN;
     else R.round_refill(q, lane);
@@ -211,15 +251,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
       if (kRoundsPerCheck > 1 && rk >= rounds) break;
       if (rk < full) decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
       else decode_round<false, G, FMT, PB>(D, x, rk * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
-      out += step;
-      col += step;
-      if (col >= cols) {
-        do {
-          col -= cols;
-          ++row;
-        } while (col >= cols);
-        if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
-      }
+      advance(F{});
     }
     if (q - R.off0 > 2 * nwords) {
       status |= EQ_DEV_OVERRUN;
@@ -241,9 +273,18 @@ template <int G, int FMT, uint32_t PB>
 __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
     rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
+  using Ring = WordRingT<PB == 12 ? kSegBytesWide : kSegBytes>;
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
-  unsigned char *rings = smem + rans_lut_bytes(PB);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * kRingBytes);
+  // 12-bit tables: rings at a shared address that is a multiple of their size (the word address
+  // is then one mask-and-or); the others right after the table (a multiple of the ring size from
+  // the base, which the renormalisation ORs in)
+  uint32_t ring_start = decode_lut_bytes(PB);
+  if constexpr (PB == 12) {
+    const uint32_t base = smem_addr(smem);
+    ring_start = ((base + ring_start + Ring::kBytes - 1) & ~(Ring::kBytes - 1)) - base;
+  }
+  unsigned char *rings = smem + ring_start;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + P.warps * Ring::kBytes);
 
   // tensor of this CTA: the last one whose first CTA is <= blockIdx.x
   uint32_t lo = 0, hi = P.n - 1;
@@ -260,10 +301,27 @@ __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
   const bool table_ok = hdr.magic == rans_table_magic<FMT, PB>() && hdr.prob_bits == PB;
   const uint4 *src = reinterpret_cast<const uint4 *>(D.table + sizeof(RansTableHeader) / 4);
   constexpr uint32_t kLutVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
-  if (table_ok)
-    for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x)
-      reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
-  WordRing R;
+  if (table_ok) {
+    if constexpr (PB == 12) {
+      // expand [f:12 | symbol:8 | slot - cum:12] to {f, (slot - cum) | value(symbol) << 16}
+      for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x) {
+        const uint4 e4 = __ldg(src + i);
+        const uint32_t e[4] = {e4.x, e4.y, e4.z, e4.w};
+        uint4 *dst = reinterpret_cast<uint4 *>(lut) + 2 * i;
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          dst[k] = make_uint4(e[2 * k] >> 20,
+                              (e[2 * k] & 0xFFFu) | (symbol_bf16((e[2 * k] >> 12) & 0xFFu, FMT) << 16),
+                              e[2 * k + 1] >> 20,
+                              (e[2 * k + 1] & 0xFFFu) |
+                                  (symbol_bf16((e[2 * k + 1] >> 12) & 0xFFu, FMT) << 16));
+      }
+    } else {
+      for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x)
+        reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+    }
+  }
+  Ring R;
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
@@ -375,7 +433,7 @@ static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::v
     ctas += n_ctas;
   }
   if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
-  fn<<<uint32_t(ctas), 32 * warps, rans_smem_bytes(warps, t0.prob_bits), st>>>(P);
+  fn<<<uint32_t(ctas), 32 * warps, decode_smem_bytes(warps, t0.prob_bits), st>>>(P);
   return cuda_status(cudaGetLastError());
 }
 
@@ -389,7 +447,7 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
   if (smem_optin_once(g_attr_set[dev][t0.symfmt - 1][t0.run == 8][pair ? 2 : t0.prob_bits == 8],
                       reinterpret_cast<const void *>(fn),
-                      rans_smem_bytes(pair ? 32 : 16, t0.prob_bits)) != EQ_OK)
+                      decode_smem_bytes(pair ? 32 : 16, t0.prob_bits)) != EQ_OK)
     return EQ_ERR_CUDA;
   // launches of nearly equal tensor counts, so that none is a small tail
   const size_t n = idx.size();

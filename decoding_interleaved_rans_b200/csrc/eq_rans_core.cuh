@@ -95,6 +95,49 @@ struct WordRingT {
     constexpr uint32_t kAhead = 2 * kRoundWords + 2;
     return (q + kAhead <= ready_end || ready >= nseg) ? true : wait_below(q + kAhead);
   }
+  // round_wait, and when it has to wait, for every segment handed out up to the one two past
+  // q's (those copies went out a segment or more ago), so that the next ring work is the next
+  // refill rather than another wait
+  __device__ __forceinline__ bool round_wait_far(uint32_t q) {
+    constexpr uint32_t kAhead = 2 * kRoundWords + 2;
+    if (q + kAhead <= ready_end || ready >= nseg) return true;
+    const uint32_t far = min(issued, q / SEG + 3) * SEG;
+    return wait_below(max(q + kAhead, far));
+  }
+  // The ring work of the 12-bit decode's full rounds, done once per segment: when q (the warp's
+  // next word) has entered segment cur, segment cur - 1 is used up and its copy was waited for,
+  // so its slot takes segment cur + 3; then segment cur + 1 (handed out a segment ago) is waited
+  // for.  A round reads at most 514 bytes from q and SEG > 514, so the landed segments <= cur + 1
+  // cover it.  edge_begin() sets this up from any state; edge_end() restores the fields the
+  // general checks use.  edge_next: offset of the next segment start.
+  uint32_t edge_next;
+  __device__ __forceinline__ bool edge_begin(uint32_t q, uint32_t lane) {
+    const uint32_t cur = q / SEG;
+    while (issued < nseg && issued <= cur + 3) issue(lane);
+    while (ready < nseg && ready <= cur + 1) {
+      if (!wait_slot(ready % kNumSeg)) return false;
+      ++ready;
+    }
+    edge_next = (cur + 1) * SEG;
+    return true;
+  }
+  __device__ __forceinline__ bool edge(uint32_t lane) {
+    const uint32_t cur = edge_next / SEG;
+    if (issued < nseg && issued <= cur + 3) {
+      __syncwarp();
+      issue(lane);
+    }
+    if (ready < nseg && ready <= cur + 1) {
+      if (!wait_slot(ready % kNumSeg)) return false;
+      ++ready;
+    }
+    edge_next += SEG;
+    return true;
+  }
+  __device__ __forceinline__ void edge_end() {
+    ready_end = ready * SEG;
+    refill_at = issued < nseg ? (issued - kNumSeg + 1) * SEG : 0xFFFFFFFFu;
+  }
   __device__ __forceinline__ void round_refill(uint32_t q, uint32_t lane) {
     if (q >= refill_at) refill(q, lane);
   }
@@ -184,41 +227,27 @@ __device__ __forceinline__ uint32_t rans_decode_step(uint32_t &x, bool act, cons
   return e;
 }
 
-// One step with the decode kernel's expanded 12-bit table (entry i = {f, (i - cum) | value << 16},
-// 8 bytes; see decode_lut_bytes) at shared address `base`: x' = f * (x >> 12) + (slot - cum)
-// needs no field extraction but the mask of the low half.  Returns the entry's second word (its
-// high half: the symbol's value as bf16).
+// One step with the decode kernel's 12-bit table: 4-byte entries rearranged on load to
+// [symbol:8 | f:12 | slot - cum:12] (bits 31..24, 23..12, 11..0; see decode_lut_bytes), at
+// shared address `base`, so that the symbol byte lands where a byte-permute can take it.
+// x' = f * (x >> 12) + (slot - cum).  Returns the entry.
 template <bool FULL>
-__device__ __forceinline__ uint32_t rans_value_step(uint32_t &x, bool act, uint32_t base) {
-  uint32_t w1;
-  if constexpr (FULL) {
-    asm volatile(
-        "{\n\t.reg .b32 a, f, b, xs;\n\t"
-        "shl.b32 a, %0, 3;\n\t"
-        "and.b32 a, a, 32760;\n\t"
-        "add.u32 a, a, %2;\n\t"
-        "shr.u32 xs, %0, 12;\n\t"
-        "ld.shared.v2.u32 {f, %1}, [a];\n\t"
-        "and.b32 b, %1, 65535;\n\t"
-        "mad.lo.u32 %0, f, xs, b;\n\t}"
-        : "+r"(x), "=r"(w1)
-        : "r"(base));
-  } else {
-    uint32_t nx;
-    asm volatile(
-        "{\n\t.reg .b32 a, f, b, xs;\n\t"
-        "shl.b32 a, %2, 3;\n\t"
-        "and.b32 a, a, 32760;\n\t"
-        "add.u32 a, a, %3;\n\t"
-        "shr.u32 xs, %2, 12;\n\t"
-        "ld.shared.v2.u32 {f, %1}, [a];\n\t"
-        "and.b32 b, %1, 65535;\n\t"
-        "mad.lo.u32 %0, f, xs, b;\n\t}"
-        : "=r"(nx), "=r"(w1)
-        : "r"(x), "r"(base));
-    if (act) x = nx;
-  }
-  return w1;
+__device__ __forceinline__ uint32_t rans_sym_step(uint32_t &x, bool act, uint32_t base) {
+  uint32_t e, nx;
+  asm volatile(
+      "{\n\t.reg .b32 a, f, b, xs;\n\t"
+      "and.b32 a, %2, 4095;\n\t"
+      "mad.lo.u32 a, a, 4, %3;\n\t"
+      "shr.u32 xs, %2, 12;\n\t"
+      "ld.shared.u32 %1, [a];\n\t"
+      "shr.u32 f, %1, 12;\n\t"
+      "and.b32 f, f, 4095;\n\t"
+      "and.b32 b, %1, 4095;\n\t"
+      "mad.lo.u32 %0, f, xs, b;\n\t}"
+      : "=r"(nx), "=r"(e)
+      : "r"(x), "r"(base));
+  if (FULL || act) x = nx;
+  return e;
 }
 
 // Two decode steps of a 7-bit stream with one pair-table lookup (layout in eq_internal.cuh):
@@ -270,21 +299,29 @@ __device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigne
   q = mad_lo(__popc(m), 2u, q);
 }
 
-// One round of a 12-bit stream (run 8) in which every lane holds a run, with the decode kernel's
-// expanded table, as one PTX block: eight steps, each followed by its renormalisation point, and
-// the round's dequantisation (four bf16x2 multiplies of the entries' values by the row scale; for
-// tables without NaN codes).  One block leaves ptxas no moves or reloads between the steps.
-//   tb:   shared address of the expanded table;
+// One round of a 12-bit stream (run 8) of Float8-E4M3 symbols in which every lane holds a run,
+// as one PTX block: eight steps (rans_sym_step), each followed by its renormalisation point, and
+// the round's dequantisation.  The dequantisation uses an exact identity of the E4M3 format: for
+// every finite code c, the bf16 bit pattern (c & 0x80) << 8 | (c & 0x7F) << 4 is the value of c
+// times 2^-120 (normal codes map to normal bf16 values, subnormal codes to subnormal ones, +-0 to
+// +-0), so two codes become a bf16x2 pair with one byte-permute (the permute's sign-replicate
+// mode supplies the sign bits) and two logic operations, and one bf16x2 multiply by the row scale
+// times 2^120 gives bf16_rne(value * scale): both factors are exact and the product is rounded
+// once.  Valid for tables without NaN codes and row scales below 2^8 in magnitude (the scale
+// times 2^120 is then finite and exact).  One PTX block leaves ptxas no moves between the steps.
+//   tb:   shared address of the table;
 //   ring: shared address of this warp's word ring, a multiple of its size RING, so that a word's
 //         address is one mask-and-or of q + 2 * rank;
-//   lt:   the lanes below this one; sc2: the row scale's bf16 bits in both halves.
+//   lt:   the lanes below this one; sc2e: bf16 bits of scale * 2^120 in both halves.
 // The lane's "needs a word" predicate feeds both the ballot and the predicated merge.
-#define EQ_R12_STEP(V)                                 \
+#define EQ_E4_STEP(V)                                  \
   "and.b32 t, %0, 4095;\n\t"                         \
-  "mad.lo.u32 a, t, 8, %6;\n\t"                      \
+  "mad.lo.u32 a, t, 4, %6;\n\t"                      \
   "shr.u32 xs, %0, 12;\n\t"                          \
-  "ld.shared.v2.u32 {f, " V "}, [a];\n\t"            \
-  "and.b32 t, " V ", 65535;\n\t"                     \
+  "ld.shared.u32 " V ", [a];\n\t"                    \
+  "shr.u32 f, " V ", 12;\n\t"                        \
+  "and.b32 f, f, 4095;\n\t"                          \
+  "and.b32 t, " V ", 4095;\n\t"                      \
   "mad.lo.u32 %0, f, xs, t;\n\t"                     \
   "setp.lt.u32 p, %0, 65536;\n\t"                    \
   "vote.sync.ballot.b32 m, p, 0xffffffff;\n\t"       \
@@ -297,28 +334,38 @@ __device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigne
   "@p mad.lo.u32 %0, %0, 65536, w;\n\t"              \
   "popc.b32 m, m;\n\t"                               \
   "mad.lo.u32 %1, m, 2, %1;\n\t"
-#define EQ_R12_PAIR(OUT)                               \
-  EQ_R12_STEP("va") EQ_R12_STEP("vb")                  \
-  "prmt.b32 va, va, vb, 0x7632;\n\t"                 \
+#define EQ_E4_PAIR(OUT)                                \
+  EQ_E4_STEP("va") EQ_E4_STEP("vb")                    \
+  "prmt.b32 va, va, vb, 0xF7B3;\n\t"                 \
+  "and.b32 vb, va, 0x007F007F;\n\t"                  \
+  "shl.b32 vb, vb, 4;\n\t"                           \
+  "and.b32 va, va, 0x80008000;\n\t"                  \
+  "or.b32 va, va, vb;\n\t"                           \
   "mul.rn.bf16x2 " OUT ", va, %7;\n\t"
 
 template <uint32_t RING>
-__device__ __forceinline__ uint4 rans_round12_full(uint32_t &x, uint32_t &q, uint32_t tb,
-                                                   uint32_t ring, uint32_t lt, uint32_t sc2) {
+__device__ __forceinline__ uint4 rans_round12_e4m3(uint32_t &x, uint32_t &q, uint32_t tb,
+                                                   uint32_t ring, uint32_t lt, uint32_t sc2e) {
   uint4 o;
   asm volatile(
       "{\n\t.reg .pred p;\n\t.reg .b32 t, a, f, va, vb, xs, m, r, w;\n\t"
-      EQ_R12_PAIR("%2") EQ_R12_PAIR("%3") EQ_R12_PAIR("%4") EQ_R12_PAIR("%5")
+      EQ_E4_PAIR("%2") EQ_E4_PAIR("%3") EQ_E4_PAIR("%4") EQ_E4_PAIR("%5")
       "}"
       : "+r"(x), "+r"(q), "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
-      : "r"(tb), "r"(sc2), "r"(ring), "r"(lt), "n"(RING - 1));
+      : "r"(tb), "r"(sc2e), "r"(ring), "r"(lt), "n"(RING - 1));
   return o;
 }
-#undef EQ_R12_PAIR
-#undef EQ_R12_STEP
+#undef EQ_E4_PAIR
+#undef EQ_E4_STEP
+
+// bf16 bits of scale * 2^120 in both halves (the factor of rans_round12_e4m3); exact for
+// |scale| < 2^8 (a finite bf16 held exactly as fp32; the fp32 product is a power-of-two scaling)
+__device__ __forceinline__ uint32_t scale_e4m3_offset(float sc) {
+  return __byte_perm(__float_as_uint(sc * 1.329227995784916e36f), 0u, 0x3232u);
+}
 
 // A renormalisation point with the ring at absolute shared address `ring` (a multiple of RING):
-// the general form of the one in rans_round12_full, for rounds in which some lanes hold no run.
+// the general form of the one in rans_round12_e4m3, for rounds in which some lanes hold no run.
 template <bool FULL, uint32_t RING>
 __device__ __forceinline__ void rans_renorm_abs(uint32_t &x, bool act, uint32_t ring, uint32_t &q,
                                                 uint32_t lt) {
@@ -395,12 +442,12 @@ __host__ __device__ constexpr size_t rans_smem_bytes(uint32_t warps, uint32_t pb
   return rans_lut_bytes(pb) + warps * (kRingBytes + kNumSeg * 8);
 }
 
-// The decode kernel's table: 12-bit tables are expanded on load to 8-byte entries {f, (slot -
-// cum) | value(symbol) << 16} (32 KiB), the 8- and 7-bit ones are used as they are.  Its rings:
-// 4 KiB (1 KiB copies) with 12-bit tables, placed at a shared address that is a multiple of their
-// size (up to one ring of slack), else 2 KiB right after the table.
+// The decode kernel's table: 12-bit entries are rearranged on load to [symbol | f | slot - cum]
+// (16 KiB), the 8- and 7-bit tables are used as they are.  Its rings: 4 KiB (1 KiB copies) with
+// 12-bit tables, placed at a shared address that is a multiple of their size (up to one ring of
+// slack), else 2 KiB right after the table.
 __host__ __device__ constexpr uint32_t decode_lut_bytes(uint32_t pb) {
-  return pb == 12 ? (8u << 12) : rans_lut_bytes(pb);
+  return rans_lut_bytes(pb);
 }
 __host__ __device__ constexpr uint32_t decode_ring_bytes(uint32_t pb) {
   return pb == 12 ? kRingBytesWide : kRingBytes;

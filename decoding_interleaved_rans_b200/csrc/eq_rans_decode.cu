@@ -16,6 +16,7 @@
 //   * dequantisation (value * row scale, one rounding) happens in registers before the store.
 // Many tensors go in one launch (the pages decode all weights of a transformer block together).
 #include <algorithm>
+#include <mutex>
 #include <type_traits>
 #include <vector>
 
@@ -24,9 +25,9 @@
 
 namespace eq {
 
-// descriptors one launch carries as kernel parameters (120 bytes each, within the 32764-byte
+// descriptors one launch carries as kernel parameters (128 bytes each, within the 32764-byte
 // parameter limit); a larger group goes in several launches of nearly equal size
-constexpr int kMaxDecodeTensors = 256;
+constexpr int kMaxDecodeTensors = 255;
 
 struct RansDesc {
   const uint32_t *states;
@@ -41,6 +42,7 @@ struct RansDesc {
   uint64_t numel;
   uint64_t units;         // num_chunks * groups: one warp each
   uint64_t row_magic;     // floor(j / cols) = __umul64hi(j, row_magic) (0: cols == 1)
+  uint64_t group_magic;   // the same for floor(unit / groups)
   uint32_t rows, cols;
   uint32_t chunk_symbols;
   uint32_t groups;        // streams / 32
@@ -65,7 +67,8 @@ template <bool FULL, int G, int FMT, uint32_t PB, bool MAYBE_NAN = true, class R
 __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, bool act,
                                              const uint32_t *lut, const unsigned char *smem,
                                              const Ring &R, uint32_t &q, uint32_t lt,
-                                             uint16_t *out, float sc, bool nan_codes_) {
+                                             uint16_t *out, float sc, bool nan_codes_,
+                                             uint32_t tb = 0, uint32_t ring = 0) {
   static_assert(PB == 12 || G == 8, "7- and 8-bit tables need whole runs of 8");
   // MAYBE_NAN false: the table has no NaN code, and the checks compile away
   const bool nan_codes = MAYBE_NAN && nan_codes_;
@@ -82,27 +85,31 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
           make_uint4(pair_dequant(pv[0], sc2, nan_codes), pair_dequant(pv[1], sc2, nan_codes),
                      pair_dequant(pv[2], sc2, nan_codes), pair_dequant(pv[3], sc2, nan_codes));
     }
-  } else if constexpr (PB == 12) {  // the expanded table: each entry carries the symbol's value
-    const uint32_t sc2 = scale_bf16x2(sc);
-    const uint32_t tb = smem_addr(smem);  // the expanded table starts the shared memory
-    const uint32_t ring = smem_addr(R.buf);
-    if constexpr (FULL && !MAYBE_NAN && G == 8) {
-      *reinterpret_cast<uint4 *>(out) = rans_round12_full<Ring::kBytes>(x, q, tb, ring, lt, sc2);
+  } else if constexpr (PB == 12) {  // entries [symbol | f | slot - cum]
+    // tb, ring: shared addresses of the table (the start of the shared memory) and of this
+    // warp's ring, converted once per unit by the caller
+    if constexpr (FULL && !MAYBE_NAN && G == 8 && FMT == EQ_SYM_E4M3) {
+      // E4M3, no NaN codes, |scale| < 2^8 (the caller checked the unit's rows)
+      *reinterpret_cast<uint4 *>(out) =
+          rans_round12_e4m3<Ring::kBytes>(x, q, tb, ring, lt, scale_e4m3_offset(sc));
     } else if constexpr (G == 8) {
-      uint32_t o[4];  // each pair dequantised as soon as both of its steps are done
+      uint32_t e[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t va = rans_value_step<FULL>(x, act, tb);
+      for (int p = 0; p < 8; ++p) {
+        e[p] = rans_sym_step<FULL>(x, act, tb);
         rans_renorm_abs<FULL, Ring::kBytes>(x, act, ring, q, lt);
-        const uint32_t vb = rans_value_step<FULL>(x, act, tb);
-        rans_renorm_abs<FULL, Ring::kBytes>(x, act, ring, q, lt);
-        o[k] = pair_dequant(value_pair12(va, vb), sc2, nan_codes);
       }
-      if (FULL || act) *reinterpret_cast<uint4 *>(out) = make_uint4(o[0], o[1], o[2], o[3]);
+      if (FULL || act) {
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          o[k] = dequant2<FMT>(__byte_perm(e[2 * k], e[2 * k + 1], 0x0073u), sc, nan_codes);
+        *reinterpret_cast<uint4 *>(out) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     } else {
-      const uint32_t v = rans_value_step<FULL>(x, act, tb);
+      const uint32_t e = rans_sym_step<FULL>(x, act, tb);
       rans_renorm_abs<FULL, Ring::kBytes>(x, act, ring, q, lt);
-      if (FULL || act) *out = uint16_t(pair_dequant(v >> 16, sc2, nan_codes));
+      if (FULL || act) *out = dequant1<FMT>(e >> 24, sc);
     }
   } else {
     uint32_t e[G];
@@ -140,7 +147,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
                                                  const unsigned char *smem, uint32_t flags,
                                                  uint32_t single_sym, Ring &R, uint64_t unit,
                                                  uint32_t lane) {
-  const uint64_t chunk = unit / D.groups;
+  const uint64_t chunk = div_by_magic(unit, D.group_magic);
   const uint32_t g = uint32_t(unit - chunk * D.groups);
   const uint32_t S = 32 * D.groups, s = 32 * g + lane;
   const uint64_t j0 = chunk * uint64_t(D.chunk_symbols);
@@ -171,6 +178,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   R.start(D.words, w0, nwords, lane);
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (flags & (kRansFlagNaN7F | kRansFlagNaNFF));
   const uint32_t lt = lanemask_lt_once();
+  const uint32_t tb = smem_addr(smem), ring = smem_addr(R.buf);
   // rounds in which all 32 lanes of this group hold a run
   const uint32_t full = runs >= 32 * g + 32 ? (runs - 32 * g - 32) / S + 1 : 0;
   uint32_t q = R.off0;
@@ -212,29 +220,89 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   // wait, so every segment a wait needs has been handed to the copy engine.  Instantiated for
   // tables with and without NaN codes and for one or several row ends per round, so that none
   // of those tests is left in the loop.
-  auto run_full = [&](auto maybe_nan, auto one_wrap) -> uint32_t {
-    uint32_t q_next = 0;
-    for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
-      // q is the same in every lane; the vote tells the compiler so (no reconvergence point)
-      if (__any_sync(0xFFFFFFFFu, q >= q_next)) {
+  // The ring work before a full round.  12-bit tables: once per segment (edge); otherwise the
+  // general checks, run only once q reaches q_next.  q is the same in every lane; the vote tells
+  // the compiler so (no reconvergence point).
+  uint32_t q_next = 0;
+  auto ring_work = [&]() -> uint32_t {
+    if constexpr (PB == 12) {
+      if (__any_sync(0xFFFFFFFFu, q >= R.edge_next)) {
         if (q > q_end) return EQ_DEV_OVERRUN;
-        R.round_refill(q, lane);
-        if (!R.round_wait(q)) return EQ_DEV_TIMEOUT;
-        q_next = R.quiet_until(q_end);
+        if (!R.edge(lane)) return EQ_DEV_TIMEOUT;
       }
+    } else if (__any_sync(0xFFFFFFFFu, q >= q_next)) {
+      if (q > q_end) return EQ_DEV_OVERRUN;
+      R.round_refill(q, lane);
+      if (!R.round_wait(q)) return EQ_DEV_TIMEOUT;
+      q_next = R.quiet_until(q_end);
+    }
+    return 0u;
+  };
+  auto run_full = [&](auto maybe_nan, auto one_wrap) -> uint32_t {
+    for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
+      if (const uint32_t st = ring_work()) return st;
 #pragma unroll
       for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
         decode_round<true, G, FMT, PB, decltype(maybe_nan)::value>(D, x, true, lut, smem, R, q,
-                                                                   lt, out, sc, true);
+                                                                   lt, out, sc, true, tb, ring);
         advance(one_wrap);
       }
     }
     return 0u;
   };
+  // Rounds that never straddle a row (cols and the chunk length multiples of S * G): row and
+  // scale are the same in every lane and change every cols / step rounds, so a loop over rows
+  // and, inside it, over the row's rounds, with nothing tracked per round but the output
+  // position.  Afterwards each lane's row, column and scale are recomputed for the general loop.
+  auto run_rows = [&](auto maybe_nan) -> uint32_t {
+    const uint32_t per_row = cols / step;
+    uint32_t row_u = uint32_t(div_by_magic(j0, D.row_magic));
+    uint32_t left = per_row - uint32_t(j0 - uint64_t(row_u) * cols) / step;
+    uint32_t st = 0;
+    while (r0 < full && !st) {
+      const uint32_t nr = min(left, full - r0);
+      const float sc_u = bf16_bits_to_float(D.scales[row_u]);
+      for (uint32_t k = 0; k < nr; ++k) {
+        if ((st = ring_work())) break;
+        decode_round<true, G, FMT, PB, decltype(maybe_nan)::value>(D, x, true, lut, smem, R, q,
+                                                                   lt, out, sc_u, true, tb, ring);
+        out += step;
+        ++r0;
+      }
+      left -= nr;
+      if (left == 0) {
+        left = per_row;
+        ++row_u;
+      }
+    }
+    const uint64_t j = j0 + (uint64_t(r0) * S + s) * G;
+    row = uint32_t(div_by_magic(j, D.row_magic));
+    col = uint32_t(j - uint64_t(row) * cols);
+    sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+    return st;
+  };
   using T = std::true_type;
   using F = std::false_type;
-  if (nan_codes) status = step <= cols ? run_full(T{}, T{}) : run_full(T{}, F{});
+  // The full rounds go without NaN checks when the table has no NaN code; for 12-bit tables that
+  // also selects the E4M3 round block, which needs Float8-E4M3 symbols and every row scale of the
+  // unit below 2^8 in magnitude (checked here, one scale per lane).
+  if constexpr (PB == 12)
+    if (!R.edge_begin(q, lane)) status = EQ_DEV_TIMEOUT;
+  bool plain = !nan_codes;
+  if constexpr (PB == 12) {
+    if (FMT != EQ_SYM_E4M3) plain = false;
+    const uint32_t r_first = uint32_t(div_by_magic(j0, D.row_magic));
+    const uint32_t r_last = uint32_t(div_by_magic(j0 + n - 1, D.row_magic));
+    bool ok = true;
+    for (uint32_t r = r_first + lane; r <= r_last; r += 32) ok &= (D.scales[r] & 0x7FFFu) < 0x4380u;
+    plain = __all_sync(0xFFFFFFFFu, ok) && plain;
+  }
+  const bool row_rounds = G == 8 && cols % step == 0 && D.chunk_symbols % step == 0;
+  if (status) {
+  } else if (row_rounds) status = plain ? run_rows(F{}) : run_rows(T{});
+  else if (!plain) status = step <= cols ? run_full(T{}, T{}) : run_full(T{}, F{});
   else status = step <= cols ? run_full(F{}, T{}) : run_full(F{}, F{});
+  if constexpr (PB == 12) R.edge_end();
   if (!status) {  // the general loop below waits first: hand out the used-up slots
     if (q > q_end) status |= EQ_DEV_OVERRUN;
     else R.round_refill(q, lane);
@@ -249,8 +317,8 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
     for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
       const uint32_t rk = r + k;
       if (kRoundsPerCheck > 1 && rk >= rounds) break;
-      if (rk < full) decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes);
-      else decode_round<false, G, FMT, PB>(D, x, rk * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes);
+      if (rk < full) decode_round<true, G, FMT, PB>(D, x, true, lut, smem, R, q, lt, out, sc, nan_codes, tb, ring);
+      else decode_round<false, G, FMT, PB>(D, x, rk * S + s < runs, lut, smem, R, q, lt, out, sc, nan_codes, tb, ring);
       advance(F{});
     }
     if (q - R.off0 > 2 * nwords) {
@@ -303,18 +371,11 @@ __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
   constexpr uint32_t kLutVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
   if (table_ok) {
     if constexpr (PB == 12) {
-      // expand [f:12 | symbol:8 | slot - cum:12] to {f, (slot - cum) | value(symbol) << 16}
+      // [f:12 | symbol:8 | slot - cum:12] -> [symbol:8 | f:12 | slot - cum:12]
+      auto sfb = [](uint32_t v) { return (v << 12 & 0xFF000000u) | (v >> 20) << 12 | (v & 0xFFFu); };
       for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x) {
-        const uint4 e4 = __ldg(src + i);
-        const uint32_t e[4] = {e4.x, e4.y, e4.z, e4.w};
-        uint4 *dst = reinterpret_cast<uint4 *>(lut) + 2 * i;
-#pragma unroll
-        for (int k = 0; k < 2; ++k)
-          dst[k] = make_uint4(e[2 * k] >> 20,
-                              (e[2 * k] & 0xFFFu) | (symbol_bf16((e[2 * k] >> 12) & 0xFFu, FMT) << 16),
-                              e[2 * k + 1] >> 20,
-                              (e[2 * k + 1] & 0xFFFu) |
-                                  (symbol_bf16((e[2 * k + 1] >> 12) & 0xFFu, FMT) << 16));
+        const uint4 e = __ldg(src + i);
+        reinterpret_cast<uint4 *>(lut)[i] = make_uint4(sfb(e.x), sfb(e.y), sfb(e.z), sfb(e.w));
       }
     } else {
       for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x)
@@ -325,7 +386,9 @@ __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
-  uint64_t unit = uint64_t(blockIdx.x - D.cta_begin) * P.warps + warp;
+  // units go to the tensor's CTAs round-robin (CTA c, warp w: unit w * ctas + c, then every
+  // ctas * warps), so that a launch of fewer units than warp slots spreads them evenly
+  uint64_t unit = uint64_t(warp) * D.ctas + (blockIdx.x - D.cta_begin);
   if (unit >= D.units) return;
   const uint64_t stride = uint64_t(D.ctas) * P.warps;
   uint32_t status = table_ok ? 0u : EQ_DEV_CORRUPT_STATE;
@@ -379,6 +442,39 @@ eq_status validate_rans_tensor(const eq_rans_tensor &t) {
 
 static std::atomic<bool> g_attr_set[64][2][2][3];  // device, symfmt, run == 8, table (12 / 8 / 7 bits)
 
+// CTAs of `fn` that fit on one SM with `threads` threads and `smem` bytes of dynamic shared
+// memory (the occupancy query, cached per device, kernel and block size; at least 1).  Lookups
+// take no lock; an entry is filled under a mutex and published by its kernel pointer.
+static int ctas_per_sm(KernelFn fn, uint32_t threads, size_t smem) {
+  struct Entry {
+    std::atomic<const void *> fn{nullptr};
+    uint32_t threads = 0;
+    int n = 0;
+  };
+  static Entry cache[64][16];
+  static std::mutex fill;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  const void *key = reinterpret_cast<const void *>(fn);
+  for (auto &c : cache[dev])
+    if (c.fn.load(std::memory_order_acquire) == key && c.threads == threads) return c.n;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, int(threads), smem) != cudaSuccess || n < 1)
+    n = 1;
+  std::lock_guard<std::mutex> lock(fill);
+  for (auto &c : cache[dev]) {
+    const void *f = c.fn.load(std::memory_order_relaxed);
+    if (f == key && c.threads == threads) break;  // another thread filled it
+    if (f == nullptr) {
+      c.threads = threads;
+      c.n = n;
+      c.fn.store(key, std::memory_order_release);
+      break;
+    }
+  }
+  return n;
+}
+
 // One launch over tensors idx[b, e) of one kernel variant.  Every size that shapes the launch
 // (warps per CTA, each tensor's share of the CTAs) comes from the units of these tensors alone.
 static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::vector<uint32_t> &idx,
@@ -396,10 +492,19 @@ static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::v
     // unit about once (larger tensors: the warps loop)
     warps = uint32_t(std::min<uint64_t>(32, std::max<uint64_t>(1, (total_units + sms - 1) / sms)));
   } else {
-    // warps (= groups) per CTA: 16 when the work covers every SM several times over
-    warps = 16;
-    while (warps > 1 && (total_units + warps - 1) / warps < 4 * sms) warps >>= 1;
+    // warps (= groups) per CTA sharing one copy of the table: 12 with 12-bit tables (three such
+    // CTAs fit an SM beside their 4 KiB rings: 36 warps; 16-warp CTAs fit two), else 16
+    warps = t0.prob_bits == 12 ? 12 : 16;
   }
+  // CTAs of this kernel one wave holds (occupancy: registers and shared memory)
+  const uint64_t wave = sms * uint64_t(ctas_per_sm(fn, 32 * warps, decode_smem_bytes(warps, t0.prob_bits)));
+  uint64_t natural = 0;  // one CTA per `warps` units of each tensor
+  for (size_t q = b; q < e; ++q)
+    natural += (ts[idx[q]].num_chunks * (ts[idx[q]].streams / 32) + warps - 1) / warps;
+  // A launch of under two waves: at most one wave of CTAs, each tensor's share of them in
+  // proportion to its units (the kernel spreads a tensor's units over its CTAs round-robin), so
+  // every SM gets about the same work instead of some holding one CTA more.
+  const bool spread = !pair && natural < 2 * wave;
   static thread_local RansDecodeParams P;
   P.status = d_status;
   P.warps = warps;
@@ -422,12 +527,15 @@ static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::v
     D.groups = t.streams / 32;
     D.units = t.num_chunks * D.groups;
     D.row_magic = div_magic(t.cols);
+    D.group_magic = div_magic(D.groups);
     D.rows = t.rows;
     D.cols = t.cols;
     D.chunk_symbols = t.chunk_symbols;
     uint64_t n_ctas = (D.units + warps - 1) / warps;
     if (pair)  // at most the tensor's share of the SMs, at least one CTA
       n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, D.units * sms / total_units));
+    else if (spread)  // the tensor's share of one wave
+      n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, (D.units * wave + total_units / 2) / total_units));
     D.cta_begin = uint32_t(ctas);
     D.ctas = uint32_t(n_ctas);
     ctas += n_ctas;
@@ -447,7 +555,7 @@ static eq_status launch_group(const eq_rans_tensor *ts, const std::vector<uint32
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
   if (smem_optin_once(g_attr_set[dev][t0.symfmt - 1][t0.run == 8][pair ? 2 : t0.prob_bits == 8],
                       reinterpret_cast<const void *>(fn),
-                      decode_smem_bytes(pair ? 32 : 16, t0.prob_bits)) != EQ_OK)
+                      decode_smem_bytes(pair ? 32 : t0.prob_bits == 12 ? 12 : 16, t0.prob_bits)) != EQ_OK)
     return EQ_ERR_CUDA;
   // launches of nearly equal tensor counts, so that none is a small tail
   const size_t n = idx.size();

@@ -1,8 +1,10 @@
 // eq_mlp_decode: a LLaMA-style MLP block y = W_down (silu(W_gate x) * (W_up x)) straight from the
 // rANS-coded weights.  The pages name fused decode + compute kernels as the next step ("Float8@2bits"
-// summary, closing section); the gate, up and down products run in eq_decode_gemv's kernels, so no
-// decoded weight ever reaches memory, and the SiLU gate is applied between them in one small
-// kernel that also rounds the hidden activations to bf16 (the dtype the down projection reads).
+// summary, closing section); no decoded weight ever reaches memory.  For batch <= 4 one kernel
+// takes each row of gate and up in the same warp and writes the gated hidden vector h =
+// bf16(silu(g) * u) directly (rans_gate_up_kernel); otherwise the gate and up products run in
+// eq_decode_gemv's kernels and the SiLU gate in one small kernel that also rounds h to bf16 (the
+// dtype the down projection reads).  Either way the down product then runs in eq_decode_gemv.
 // The caller provides the scratch for the intermediate vectors (eq_mlp_scratch_bytes).
 #include <algorithm>
 
@@ -13,6 +15,9 @@
 namespace eq {
 
 eq_status validate_rans_tensor(const eq_rans_tensor &t);  // eq_rans_decode.cu
+eq_status gate_up_launch(const eq_rans_tensor *g, const eq_rans_tensor *u, const uint16_t *d_x,
+                         uint32_t batch, uint16_t *d_h, uint32_t *d_status,
+                         cudaStream_t st);  // eq_rans_gemv.cu
 
 // h = bf16( silu(g) * u ), silu(v) = v / (1 + e^-v)
 __global__ void __launch_bounds__(256) silu_mul_kernel(const float *__restrict__ g,
@@ -31,10 +36,16 @@ size_t mlp_scratch_bytes(uint64_t inter, uint64_t batch) {
   return 2 * align256(inter * batch * 4) + align256(inter * batch * 2);
 }
 
-// the three products and the gate, given scratch already split into g, u, h
+// the three products and the gate, given scratch already split into g, u, h.  With batch <= 4
+// and gate/up in the fused kernel's layout, gate, up and the gate are one launch writing h (the
+// products never leave the warps); otherwise two products, the gate kernel, and h.
 eq_status mlp_run(const eq_rans_tensor *gate, const eq_rans_tensor *up,
                   const eq_rans_tensor *down, const uint16_t *d_x, uint32_t batch, float *d_y,
                   float *g, float *u, uint16_t *h, uint32_t *d_status, void *stream) {
+  const eq_status f = gate_up_launch(gate, up, d_x, batch, h, d_status,
+                                     static_cast<cudaStream_t>(stream));
+  if (f == EQ_OK) return eq_decode_gemv(down, h, batch, d_y, d_status, stream);
+  if (f != EQ_ERR_UNSUPPORTED) return f;
   eq_status s = eq_decode_gemv(gate, d_x, batch, g, d_status, stream);
   if (s != EQ_OK) return s;
   s = eq_decode_gemv(up, d_x, batch, u, d_status, stream);

@@ -294,8 +294,8 @@ __device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigne
   const bool need = (FULL || act) && x < kRansL;
   const uint32_t m = __ballot_sync(0xFFFFFFFFu, need);
   const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (RING - 1)) | ring_off;
-  const uint32_t w = *reinterpret_cast<const uint16_t *>(smem + a);
-  if (need) x = mad_lo(x, 65536u, w);
+  const uint32_t xr = mad_lo(x, 65536u, *reinterpret_cast<const uint16_t *>(smem + a));
+  x = need ? xr : x;
   q = mad_lo(__popc(m), 2u, q);
 }
 
@@ -329,7 +329,7 @@ __device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigne
   "popc.b32 r, r;\n\t"                               \
   "mad.lo.u32 a, r, 2, %1;\n\t"                      \
   "and.b32 a, a, %10;\n\t"                           \
-  "or.b32 a, a, %8;\n\t"                             \
+  RING_JOIN " a, a, %8;\n\t"                         \
   "ld.shared.u16 w, [a];\n\t"                        \
   "@p mad.lo.u32 %0, %0, 65536, w;\n\t"              \
   "popc.b32 m, m;\n\t"                               \
@@ -343,20 +343,41 @@ __device__ __forceinline__ void rans_renorm(uint32_t &x, bool act, const unsigne
   "or.b32 va, va, vb;\n\t"                           \
   "mul.rn.bf16x2 " OUT ", va, %7;\n\t"
 
-template <uint32_t RING>
+// ALIGNED: `ring` is a multiple of RING (the word address is then a mask-and-or); otherwise any
+// shared address, and the masked offset is added to it.
+template <uint32_t RING, bool ALIGNED = true>
 __device__ __forceinline__ uint4 rans_round12_e4m3(uint32_t &x, uint32_t &q, uint32_t tb,
                                                    uint32_t ring, uint32_t lt, uint32_t sc2e) {
   uint4 o;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b32 t, a, f, va, vb, xs, m, r, w;\n\t"
-      EQ_E4_PAIR("%2") EQ_E4_PAIR("%3") EQ_E4_PAIR("%4") EQ_E4_PAIR("%5")
-      "}"
-      : "+r"(x), "+r"(q), "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
-      : "r"(tb), "r"(sc2e), "r"(ring), "r"(lt), "n"(RING - 1));
+  if constexpr (ALIGNED) {
+#define RING_JOIN "or.b32"
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 t, a, f, va, vb, xs, m, r, w;\n\t"
+        EQ_E4_PAIR("%2") EQ_E4_PAIR("%3") EQ_E4_PAIR("%4") EQ_E4_PAIR("%5")
+        "}"
+        : "+r"(x), "+r"(q), "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+        : "r"(tb), "r"(sc2e), "r"(ring), "r"(lt), "n"(RING - 1));
+#undef RING_JOIN
+  } else {
+#define RING_JOIN "add.u32"
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b32 t, a, f, va, vb, xs, m, r, w;\n\t"
+        EQ_E4_PAIR("%2") EQ_E4_PAIR("%3") EQ_E4_PAIR("%4") EQ_E4_PAIR("%5")
+        "}"
+        : "+r"(x), "+r"(q), "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+        : "r"(tb), "r"(sc2e), "r"(ring), "r"(lt), "n"(RING - 1));
+#undef RING_JOIN
+  }
   return o;
 }
 #undef EQ_E4_PAIR
 #undef EQ_E4_STEP
+
+// [f:12 | symbol:8 | slot - cum:12] (the 12-bit table eq_build_tables writes) rearranged to the
+// shared-memory layout [symbol:8 | f:12 | slot - cum:12] that rans_sym_step reads
+__device__ __forceinline__ uint32_t sym_first_entry(uint32_t v) {
+  return (v << 12 & 0xFF000000u) | (v >> 20) << 12 | (v & 0xFFFu);
+}
 
 // bf16 bits of scale * 2^120 in both halves (the factor of rans_round12_e4m3); exact for
 // |scale| < 2^8 (a finite bf16 held exactly as fp32; the fp32 product is a power-of-two scaling)
@@ -374,7 +395,8 @@ __device__ __forceinline__ void rans_renorm_abs(uint32_t &x, bool act, uint32_t 
   const uint32_t a = (mad_lo(__popc(m & lt), 2u, q) & (RING - 1)) | ring;
   uint32_t w;
   asm volatile("ld.shared.u16 %0, [%1];" : "=r"(w) : "r"(a));
-  if (need) x = mad_lo(x, 65536u, w);
+  const uint32_t xr = mad_lo(x, 65536u, w);
+  x = need ? xr : x;
   q = mad_lo(__popc(m), 2u, q);
 }
 

@@ -54,6 +54,7 @@ struct RansDecodeParams {
   uint32_t *status;
   uint32_t n;
   uint32_t warps;  // warps (= groups decoded) per CTA
+  uint32_t spread; // units dealt out round-robin over a tensor's CTAs (see the kernel)
   RansDesc d[kMaxDecodeTensors];
 };
 static_assert(sizeof(RansDecodeParams) <= 32764, "kernel parameters above the launch limit");
@@ -230,7 +231,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
         if (q > q_end) return EQ_DEV_OVERRUN;
         if (!R.edge(lane)) return EQ_DEV_TIMEOUT;
       }
-    } else if (__any_sync(0xFFFFFFFFu, q >= q_next)) {
+    } else if (q >= q_next) {
       if (q > q_end) return EQ_DEV_OVERRUN;
       R.round_refill(q, lane);
       if (!R.round_wait(q)) return EQ_DEV_TIMEOUT;
@@ -297,7 +298,8 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
     for (uint32_t r = r_first + lane; r <= r_last; r += 32) ok &= (D.scales[r] & 0x7FFFu) < 0x4380u;
     plain = __all_sync(0xFFFFFFFFu, ok) && plain;
   }
-  const bool row_rounds = G == 8 && cols % step == 0 && D.chunk_symbols % step == 0;
+  // (12-bit tables; the 8- and 7-bit ones check the ring every second round in run_full)
+  const bool row_rounds = PB == 12 && G == 8 && cols % step == 0 && D.chunk_symbols % step == 0;
   if (status) {
   } else if (row_rounds) status = plain ? run_rows(F{}) : run_rows(T{});
   else if (!plain) status = step <= cols ? run_full(T{}, T{}) : run_full(T{}, F{});
@@ -372,10 +374,10 @@ __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
   if (table_ok) {
     if constexpr (PB == 12) {
       // [f:12 | symbol:8 | slot - cum:12] -> [symbol:8 | f:12 | slot - cum:12]
-      auto sfb = [](uint32_t v) { return (v << 12 & 0xFF000000u) | (v >> 20) << 12 | (v & 0xFFFu); };
       for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x) {
         const uint4 e = __ldg(src + i);
-        reinterpret_cast<uint4 *>(lut)[i] = make_uint4(sfb(e.x), sfb(e.y), sfb(e.z), sfb(e.w));
+        reinterpret_cast<uint4 *>(lut)[i] = make_uint4(sym_first_entry(e.x), sym_first_entry(e.y),
+                                                       sym_first_entry(e.z), sym_first_entry(e.w));
       }
     } else {
       for (uint32_t i = threadIdx.x; i < kLutVec; i += blockDim.x)
@@ -386,9 +388,12 @@ __global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
   ring_init(R, smem, rings, bars, warp, lane);
   __syncthreads();
 
-  // units go to the tensor's CTAs round-robin (CTA c, warp w: unit w * ctas + c, then every
-  // ctas * warps), so that a launch of fewer units than warp slots spreads them evenly
-  uint64_t unit = uint64_t(warp) * D.ctas + (blockIdx.x - D.cta_begin);
+  // A CTA's warps take consecutive units (CTA c, warp w: unit c * warps + w, then every
+  // ctas * warps), so that an SM writes a few contiguous stretches of the output.  A launch of
+  // fewer units than warp slots (P.spread) deals them out round-robin instead (unit w * ctas + c),
+  // so that every CTA, and so every SM, gets about the same number.
+  const uint64_t cta = blockIdx.x - D.cta_begin;
+  uint64_t unit = P.spread ? uint64_t(warp) * D.ctas + cta : cta * P.warps + warp;
   if (unit >= D.units) return;
   const uint64_t stride = uint64_t(D.ctas) * P.warps;
   uint32_t status = table_ok ? 0u : EQ_DEV_CORRUPT_STATE;
@@ -508,6 +513,7 @@ static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::v
   static thread_local RansDecodeParams P;
   P.status = d_status;
   P.warps = warps;
+  P.spread = spread ? 1u : 0u;
   P.n = 0;
   uint64_t ctas = 0;
   for (size_t q = b; q < e; ++q) {
@@ -534,8 +540,8 @@ static eq_status launch_part(KernelFn fn, const eq_rans_tensor *ts, const std::v
     uint64_t n_ctas = (D.units + warps - 1) / warps;
     if (pair)  // at most the tensor's share of the SMs, at least one CTA
       n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, D.units * sms / total_units));
-    else if (spread)  // the tensor's share of one wave
-      n_ctas = std::min<uint64_t>(n_ctas, std::max<uint64_t>(1, (D.units * wave + total_units / 2) / total_units));
+    else if (spread)  // the tensor's share of one wave (some of its warps may have no unit)
+      n_ctas = std::max<uint64_t>(1, (D.units * wave + total_units / 2) / total_units);
     D.cta_begin = uint32_t(ctas);
     D.ctas = uint32_t(n_ctas);
     ctas += n_ctas;

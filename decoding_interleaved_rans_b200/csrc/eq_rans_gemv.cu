@@ -87,16 +87,25 @@ __device__ __forceinline__ void round_pairs(uint32_t (&pr)[4], uint32_t &x, bool
       pr[k] = rans_pair_step<false>(x, act, lut);
       rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
     }
+  } else if constexpr (PB == 12) {  // the table rearranged to [symbol | f | slot - cum]
+    const uint32_t tb = smem_addr(lut);
+    uint32_t e[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      e[p] = rans_sym_step<false>(x, act, tb);
+      rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pr[k] = __byte_perm(e[2 * k], e[2 * k + 1], 0x0073u);
   } else {
     uint32_t e[8];
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       e[p] = rans_decode_step<false, PB>(x, act, lut);
-      if (PB == 12 || (p & 1)) rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
+      if (p & 1) rans_renorm<false>(x, act, smem, R.ring_off, q, lt);
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      pr[k] = PB == 8 ? value_pair8(e[2 * k], e[2 * k + 1]) : sym_pair(e[2 * k], e[2 * k + 1]);
+    for (int k = 0; k < 4; ++k) pr[k] = value_pair8(e[2 * k], e[2 * k + 1]);
   }
 }
 
@@ -124,17 +133,25 @@ __device__ __forceinline__ bool load_table(uint32_t *lut, const uint32_t *table,
   const bool ok = hdr.magic == rans_table_magic<FMT, PB>() && hdr.prob_bits == PB;
   constexpr uint32_t kVec = PB == kRansPairBits ? kRansPairEntries / 2 : (1u << PB) / 4;
   const uint4 *src = reinterpret_cast<const uint4 *>(table + sizeof(RansTableHeader) / 4);
-  if (ok)
-    for (uint32_t i = threadIdx.x; i < kVec; i += blockDim.x) reinterpret_cast<uint4 *>(lut)[i] = __ldg(src + i);
+  if (ok) {
+    for (uint32_t i = threadIdx.x; i < kVec; i += blockDim.x) {
+      uint4 e = __ldg(src + i);
+      if constexpr (PB == 12)  // [symbol | f | slot - cum], as the decode kernel holds it
+        e = make_uint4(sym_first_entry(e.x), sym_first_entry(e.y), sym_first_entry(e.z),
+                       sym_first_entry(e.w));
+      reinterpret_cast<uint4 *>(lut)[i] = e;
+    }
+  }
   return ok;
 }
 
 // One warp = one chunk of whole rows, 32 streams (one per lane), run length 8.
-template <int FMT, int BMAX, uint32_t PB>
+// SUMS: the chunk is one row, and its sums go to sums[b] (in every lane) instead of y.
+template <int FMT, int BMAX, uint32_t PB, bool SUMS = false>
 __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chunk,
                                                const RansTableHeader &hdr, const uint32_t *lut,
                                                const unsigned char *smem, WordRing &R,
-                                               uint32_t lane) {
+                                               uint32_t lane, float *sums = nullptr) {
   constexpr uint32_t S = 32;
   uint32_t status = 0;
   const bool single = hdr.flags & kRansFlagSingle;
@@ -165,8 +182,91 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
   const uint32_t q_end = R.off0 + 2 * nwords;
   uint32_t q_next = 0;
 
+  // 12-bit tables of E4M3 symbols without NaN codes: rounds in which every lane holds a run go
+  // through the decode kernel's E4M3 round block (the weights come out dequantised), while the
+  // row's scale is below 2^8 in magnitude
+  const uint32_t tb = smem_addr(lut), ring_abs = smem_addr(R.buf);
+  auto e4_row = [&](uint32_t row) {
+    return PB == 12 && FMT == EQ_SYM_E4M3 && !nan_codes && !single &&
+           (P.scales[row] & 0x7FFFu) < 0x4380u;
+  };
+  bool e4 = e4_row(row0);
+
+  // One row per chunk in whole rounds with the E4M3 round block (no super weights): a loop with
+  // nothing in it but the ring work, the round and its products, then the row's sum.
+  if constexpr (PB == 12 && FMT == EQ_SYM_E4M3) {
+    if (e4 && P.rows_per_chunk == 1 && runs % S == 0 && P.n_patch == 0) {
+      const uint32_t sc2e = scale_e4m3_offset(sc);
+      for (uint32_t r = 0; r < rounds; ++r) {
+        if (q >= q_next) {
+          if (q > q_end) {
+            status |= EQ_DEV_OVERRUN;
+            break;
+          }
+          R.round_refill(q, lane);
+          if (!R.round_wait(q)) {
+            status |= EQ_DEV_TIMEOUT;
+            break;
+          }
+          q_next = R.quiet_until(q_end);
+        }
+        const uint4 o = rans_round12_e4m3<kRingBytes, false>(x, q, tb, ring_abs, lt, sc2e);
+        fma_run<BMAX>(acc, make_uint2(o.x, o.y), make_uint2(o.z, o.w), P.x, P.cols,
+                      (r * S + lane) * 8, batch);
+      }
+      if (!status && !__all_sync(0xFFFFFFFFu, q - R.off0 == 2 * nwords && x == kRansL))
+        status |= EQ_DEV_CORRUPT_STATE;
+      if (!status) {
+#pragma unroll
+        for (int b = 0; b < BMAX; ++b) {
+          float v = acc[b].x + acc[b].y;
+#pragma unroll
+          for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, d);
+          if constexpr (SUMS) sums[b] = v;
+          else if (lane == 0 && b < int(batch)) P.y[size_t(b) * P.rows + row0] = v;
+        }
+      }
+      status |= R.drain();
+      return status;
+    }
+  }
+
   for (uint32_t r = 0; r < rounds; ++r) {
     const bool act = r * S + lane < runs;
+    if constexpr (PB == 12 && FMT == EQ_SYM_E4M3) {
+      if (e4 && (r + 1) * S <= runs) {  // every lane holds a run
+        if constexpr (kQuiet) {
+          if (q >= q_next) {
+            if (q > q_end) {
+              status |= EQ_DEV_OVERRUN;
+              break;
+            }
+            R.round_refill(q, lane);
+            if (!R.round_wait(q)) {
+              status |= EQ_DEV_TIMEOUT;
+              break;
+            }
+            q_next = R.quiet_until(q_end);
+          }
+        } else if (!R.round_wait(q)) {
+          status |= EQ_DEV_TIMEOUT;
+          break;
+        }
+        const uint4 o = rans_round12_e4m3<kRingBytes, false>(x, q, tb, ring_abs, lt,
+                                                             scale_e4m3_offset(sc));
+        if constexpr (!kQuiet) {
+          if (q - R.off0 > 2 * nwords) {
+            status |= EQ_DEV_OVERRUN;
+            break;
+          }
+          R.round_refill(q, lane);
+        }
+        const uint32_t col = (r * S + lane) * 8 - row_local * P.cols;
+        fma_run<BMAX>(acc, make_uint2(o.x, o.y), make_uint2(o.z, o.w), P.x, P.cols, col, batch);
+        goto row_end_check;
+      }
+    }
+    {
     uint32_t pr[4];  // the round's 8 symbols as 4 pairs (8/7-bit tables: their values, bf16x2)
     if (single) {
       pr[0] = pr[1] = pr[2] = pr[3] = single_pair<FMT, PB>(hdr.single_sym);
@@ -202,6 +302,8 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
       const uint2 wb = make_uint2(weights2<FMT, PB>(pr[2], sc, nan_codes), weights2<FMT, PB>(pr[3], sc, nan_codes));
       fma_run<BMAX>(acc, wa, wb, P.x, P.cols, col, batch);
     }
+    }
+  row_end_check:
     // end of a weight row: add its super weights' products, reduce across the warp, write y
     const bool row_end = (r + 1 == rounds) || (P.rows_per_chunk > 1 && (r + 1) % P.rounds_per_row == 0);
     if (row_end) {
@@ -222,12 +324,15 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
         float v = acc[b].x + acc[b].y;
 #pragma unroll
         for (int d = 16; d > 0; d >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, d);
-        if (lane == 0 && b < int(batch)) P.y[size_t(b) * P.rows + row0 + row_local] = v;
+        if constexpr (SUMS) sums[b] = v;
+        else if (lane == 0 && b < int(batch)) P.y[size_t(b) * P.rows + row0 + row_local] = v;
         acc[b] = make_float2(0.0f, 0.0f);
       }
       ++row_local;
-      if (row_local < P.rows_per_chunk && r + 1 < rounds)
+      if (row_local < P.rows_per_chunk && r + 1 < rounds) {
         sc = bf16_bits_to_float(P.scales[row0 + row_local]);
+        e4 = e4_row(row0 + row_local);
+      }
     }
   }
   if (!status) {
@@ -273,6 +378,61 @@ __global__ void __launch_bounds__(32 * gemv_max_warps(PB, BMAX), gemv_min_ctas(P
   for (; chunk < P.num_chunks && !status; chunk += stride)
     status = gemv_chunk<FMT, BMAX, PB>(P, chunk, hdr, lut, smem, R, lane);
   if (lane == 0) report(P.status, status);
+}
+
+// ------------------------------------------------------------------------------------------------
+// The gate and up products of a LLaMA-style MLP block and its SiLU gate in one kernel: a warp
+// takes row r of gate and then row r of up (one row per chunk; the CTA holds both tables and
+// the warp's ring takes one substream after the other), and writes h[b][r] = bf16(silu(g) * u)
+// with silu(v) = v / (1 + e^-v).  The gate's and up's products never leave the warp.
+// ------------------------------------------------------------------------------------------------
+struct GateUpParams {
+  GemvParams g, u;  // gate and up (their y is not used)
+  uint16_t *h;      // bf16 [batch][rows]
+};
+
+constexpr uint32_t kGateUpWarps = 8;
+
+template <int FMT, int BMAX, uint32_t PB>
+__global__ void __launch_bounds__(32 * kGateUpWarps, 4)
+    rans_gate_up_kernel(const __grid_constant__ GateUpParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint32_t *lut_g = reinterpret_cast<uint32_t *>(smem);
+  uint32_t *lut_u = reinterpret_cast<uint32_t *>(smem + rans_lut_bytes(PB));
+  unsigned char *rings = smem + 2 * rans_lut_bytes(PB);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(rings + kGateUpWarps * kRingBytes);
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const RansTableHeader hg = *reinterpret_cast<const RansTableHeader *>(P.g.table);
+  const RansTableHeader hu = *reinterpret_cast<const RansTableHeader *>(P.u.table);
+  const bool ok_g = load_table<FMT, PB>(lut_g, P.g.table, hg);
+  const bool ok_u = load_table<FMT, PB>(lut_u, P.u.table, hu);
+  WordRing R;
+  ring_init(R, smem, rings, bars, warp, lane);
+  __syncthreads();
+
+  uint32_t status = ok_g && ok_u ? 0u : EQ_DEV_CORRUPT_STATE;
+  for (uint64_t row = uint64_t(blockIdx.x) * kGateUpWarps + warp; row < P.g.num_chunks && !status;
+       row += uint64_t(gridDim.x) * kGateUpWarps) {
+    float sg[BMAX], su[BMAX];
+    status = gemv_chunk<FMT, BMAX, PB, true>(P.g, row, hg, lut_g, smem, R, lane, sg);
+    if (!status) status = gemv_chunk<FMT, BMAX, PB, true>(P.u, row, hu, lut_u, smem, R, lane, su);
+    if (!status && lane == 0) {
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) {
+        if (b < int(P.g.batch)) {
+          const float v = sg[b];
+          const __nv_bfloat16 hb = __float2bfloat16_rn(v / (1.0f + expf(-v)) * su[b]);
+          P.h[size_t(b) * P.g.rows + row] = *reinterpret_cast<const uint16_t *>(&hb);
+        }
+      }
+    }
+  }
+  if (lane == 0) report(P.g.status, status);
+}
+
+__host__ __device__ constexpr size_t gate_up_smem_bytes(uint32_t pb) {
+  return 2 * rans_lut_bytes(pb) + kGateUpWarps * (kRingBytes + kNumSeg * 8);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -385,6 +545,22 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
 
     for (uint32_t r = 0; r < rounds; ++r) {
       const bool act = valid && !status && r * S + lane < runs;
+      // this warp's slice of x for the round's product, loaded before the decode so that the
+      // loads' latency passes while the round decodes: columns col0, col0 + 8 of batch rows
+      // nt * 8 + grp (a 16-column k-step per warp)
+      uint32_t xb[2][2] = {{0u, 0u}, {0u, 0u}};
+      {
+        const uint32_t col0 = (r % rpr) * 256 + hw * 16 + 2 * tig;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const uint32_t b = nt * 8 + grp;
+          if (uint32_t(nt) < ntiles && b < P.batch) {
+            const uint16_t *xr = P.x + size_t(b) * P.cols + col0;
+            xb[nt][0] = __ldg(reinterpret_cast<const uint32_t *>(xr));
+            xb[nt][1] = __ldg(reinterpret_cast<const uint32_t *>(xr + 8));
+          }
+        }
+      }
       uint32_t pr[4] = {0u, 0u, 0u, 0u};
       if (live) {
         if (!R.round_wait(q)) {
@@ -418,20 +594,9 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
         uint32_t a[4];
         const uint32_t arow = lane & 15, acol = (lane >> 4) * 8 + hw * 16;
         ldmatrix_x4(a, tiles_addr + (r & 1) * kTcTileBytes + arow * kTcRowBytes + acol * 2);
-        const uint32_t col0 = (r % rpr) * 256 + hw * 16 + 2 * tig;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          if (uint32_t(nt) < ntiles) {
-            const uint32_t b = nt * 8 + grp;
-            uint32_t b0 = 0, b1 = 0;
-            if (b < P.batch) {
-              const uint16_t *xr = P.x + size_t(b) * P.cols + col0;
-              b0 = __ldg(reinterpret_cast<const uint32_t *>(xr));
-              b1 = __ldg(reinterpret_cast<const uint32_t *>(xr + 8));
-            }
-            mma_bf16_16816(c[nt], a, b0, b1);
-          }
-        }
+        for (int nt = 0; nt < 2; ++nt)
+          if (uint32_t(nt) < ntiles) mma_bf16_16816(c[nt], a, xb[nt][0], xb[nt][1]);
       }
       // end of a weight row: sum the 16 warps' partial products in a fixed order
       if ((r + 1) % rpr == 0) {
@@ -496,7 +661,76 @@ static GemvFn pick_pb(uint32_t pb, uint32_t batch, bool tc) {
                                                          : pick_b<FMT, kRansPairBits>(batch, tc);
 }
 
-static std::atomic<bool> g_gemv_attr[64][2][3][6];  // device, symfmt, table (12 / 8 / 7 bits), kernel instance
+static std::atomic<bool> g_gemv_attr[64][2][3][6];
+static std::atomic<bool> g_gate_up_attr[64][2][2][3];  // device, symfmt, table (12 / 8), batch kind
+
+// the kernel parameters of one tensor's product
+static GemvParams gemv_params(const eq_rans_tensor *t, const uint16_t *d_x, uint32_t batch,
+                              float *d_y, uint32_t *d_status, uint32_t warps) {
+  const uint32_t rpc = t->chunk_symbols / t->cols;
+  GemvParams P;
+  P.states = t->states;
+  P.word_off = t->word_off;
+  P.words = t->words;
+  P.scales = t->scales;
+  P.table = static_cast<const uint32_t *>(t->tables);
+  P.x = d_x;
+  P.y = d_y;
+  P.status = d_status;
+  P.patch_idx = t->patch_idx;
+  P.patch_val = t->patch_val;
+  P.n_patch = t->n_patch;
+  P.numel = uint64_t(t->rows) * t->cols;
+  P.num_chunks = t->num_chunks;
+  P.rows = t->rows;
+  P.cols = t->cols;
+  P.chunk_symbols = t->chunk_symbols;
+  P.rows_per_chunk = rpc;
+  P.rounds_per_row = rpc > 1 ? t->cols / (t->streams * 8) : 0;
+  P.batch = batch;
+  P.warps = warps;
+  return P;
+}
+
+template <int FMT, uint32_t PB>
+static void (*pick_gate_up(uint32_t batch))(GateUpParams) {
+  if (batch <= 1) return rans_gate_up_kernel<FMT, 1, PB>;
+  if (batch <= 2) return rans_gate_up_kernel<FMT, 2, PB>;
+  return rans_gate_up_kernel<FMT, 4, PB>;
+}
+
+// The gate and up products and the SiLU gate of an MLP block in one launch, h = bf16(silu(W_gate
+// x) * (W_up x)), when both tensors take the fused kernel: batch <= 4, 12- or 8-bit tables of one
+// symbol format, one row per chunk (chunk_symbols == cols), 32 streams, run 8.  EQ_ERR_UNSUPPORTED
+// (nothing launched) otherwise.  Both descriptors were validated by the caller.
+eq_status gate_up_launch(const eq_rans_tensor *g, const eq_rans_tensor *u, const uint16_t *d_x,
+                         uint32_t batch, uint16_t *d_h, uint32_t *d_status, cudaStream_t st) {
+  if (batch > 4 || g->symfmt != u->symfmt || g->prob_bits != u->prob_bits) return EQ_ERR_UNSUPPORTED;
+  if (g->prob_bits != 12 && g->prob_bits != 8) return EQ_ERR_UNSUPPORTED;
+  for (const eq_rans_tensor *t : {g, u})
+    if (t->run != 8 || t->streams != 32 || t->chunk_symbols != t->cols || t->rows != g->rows ||
+        t->cols != g->cols)
+      return EQ_ERR_UNSUPPORTED;
+  if (!d_x || !d_h || !aligned(d_x, 16)) return EQ_ERR_ARG;
+  const uint32_t pb = g->prob_bits;
+  auto fn = g->symfmt == EQ_SYM_E4M3
+                ? (pb == 12 ? pick_gate_up<EQ_SYM_E4M3, 12>(batch) : pick_gate_up<EQ_SYM_E4M3, 8>(batch))
+                : (pb == 12 ? pick_gate_up<EQ_SYM_INT8, 12>(batch) : pick_gate_up<EQ_SYM_INT8, 8>(batch));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return EQ_ERR_CUDA;
+  const int bi = batch <= 1 ? 0 : batch <= 2 ? 1 : 2;
+  if (smem_optin_once(g_gate_up_attr[dev][g->symfmt - 1][pb == 12 ? 0 : 1][bi],
+                      reinterpret_cast<const void *>(fn), gate_up_smem_bytes(pb)) != EQ_OK)
+    return EQ_ERR_CUDA;
+  GateUpParams P;
+  P.g = gemv_params(g, d_x, batch, nullptr, d_status, kGateUpWarps);
+  P.u = gemv_params(u, d_x, batch, nullptr, d_status, kGateUpWarps);
+  P.h = d_h;
+  const uint64_t ctas = (uint64_t(g->rows) + kGateUpWarps - 1) / kGateUpWarps;
+  if (ctas >= (1ull << 31)) return EQ_ERR_UNSUPPORTED;
+  fn<<<uint32_t(ctas), 32 * kGateUpWarps, gate_up_smem_bytes(pb), st>>>(P);
+  return cuda_status(cudaGetLastError());
+}  // device, symfmt, table (12 / 8 / 7 bits), kernel instance
 
 }  // namespace eq
 
@@ -547,27 +781,7 @@ extern "C" eq_status eq_decode_gemv(const eq_rans_tensor *t, const uint16_t *d_x
                       reinterpret_cast<const void *>(fn),
                       tc ? gemv_tc_smem_bytes(pb, pair ? 2 : 1) : rans_smem_bytes(max_warps, pb)) != EQ_OK)
     return EQ_ERR_CUDA;
-  GemvParams P;
-  P.states = t->states;
-  P.word_off = t->word_off;
-  P.words = t->words;
-  P.scales = t->scales;
-  P.table = static_cast<const uint32_t *>(t->tables);
-  P.x = d_x;
-  P.y = d_y;
-  P.status = d_status;
-  P.patch_idx = t->patch_idx;
-  P.patch_val = t->patch_val;
-  P.n_patch = t->n_patch;
-  P.numel = uint64_t(t->rows) * t->cols;
-  P.num_chunks = t->num_chunks;
-  P.rows = t->rows;
-  P.cols = t->cols;
-  P.chunk_symbols = t->chunk_symbols;
-  P.rows_per_chunk = rpc;
-  P.rounds_per_row = rpc > 1 ? t->cols / (t->streams * 8) : 0;
-  P.batch = batch;
-  P.warps = warps;
+  const GemvParams P = gemv_params(t, d_x, batch, d_y, d_status, warps);
   fn<<<uint32_t(ctas), 32 * warps, tc ? gemv_tc_smem_bytes(pb, pair ? 2 : 1) : rans_smem_bytes(warps, pb),
        static_cast<cudaStream_t>(stream)>>>(P);
   return cuda_status(cudaGetLastError());

@@ -478,7 +478,7 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&a)[4], uint32_t addr) {
 // Each half of the CTA takes group after group of 16 chunks; every warp of a half runs the same
 // rounds, so its barriers line up.
 template <int FMT, uint32_t PB, int HALVES>
-__global__ void __launch_bounds__(HALVES * kTcWarps * 32)
+__global__ void __launch_bounds__(HALVES * kTcWarps * 32, HALVES == 1 ? 2 : 1)
     rans_gemv_tc_kernel(const __grid_constant__ GemvParams P) {
   constexpr uint32_t S = 32;
   constexpr bool kAlias = HALVES > 1;  // the reduction buffer lies over the half's tiles
@@ -511,6 +511,7 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
   const uint32_t rpr = P.rows_per_chunk > 1 ? P.rounds_per_row : rounds;
   const uint32_t ntiles = (P.batch + 7) / 8;
   const uint32_t tiles_addr = smem_addr(tiles);
+  const uint32_t tb = smem_addr(lut), ring_abs = smem_addr(R.buf);
   const uint64_t ngroups = (P.num_chunks + kTcWarps - 1) / kTcWarps;
   // sticky: a warp whose chunk failed feeds zeros from then on (the launch reports the failure)
   uint32_t status = 0;
@@ -542,6 +543,11 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
     float c[2][4] = {};
     uint32_t row_local = 0;
     float sc = valid ? bf16_bits_to_float(P.scales[row0]) : 0.0f;
+    auto e4_row = [&](uint32_t row) {
+      return PB == 12 && FMT == EQ_SYM_E4M3 && !nan_codes && !single &&
+             (P.scales[row] & 0x7FFFu) < 0x4380u;
+    };
+    bool e4 = valid && e4_row(row0);
 
     for (uint32_t r = 0; r < rounds; ++r) {
       const bool act = valid && !status && r * S + lane < runs;
@@ -562,15 +568,26 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
         }
       }
       uint32_t pr[4] = {0u, 0u, 0u, 0u};
+      // E4M3 rounds in which every lane holds a run (no NaN codes, row scale below 2^8): the
+      // decode kernel's round block, whose weights come out dequantised
+      bool done = false;
+      uint4 wv = make_uint4(0u, 0u, 0u, 0u);
       if (live) {
         if (!R.round_wait(q)) {
           status |= EQ_DEV_TIMEOUT;
           live = false;
         } else {
-          round_pairs<PB>(pr, x, act, lut, smem, R, q, lt);
+          if constexpr (PB == 12 && FMT == EQ_SYM_E4M3) {
+            if (e4 && (r + 1) * S <= runs) {
+              wv = rans_round12_e4m3<kRingBytes, false>(x, q, tb, ring_abs, lt, scale_e4m3_offset(sc));
+              done = true;
+            }
+          }
+          if (!done) round_pairs<PB>(pr, x, act, lut, smem, R, q, lt);
           if (q - R.off0 > 2 * nwords) {
             status |= EQ_DEV_OVERRUN;
             live = false;
+            wv = make_uint4(0u, 0u, 0u, 0u);
           } else {
             R.round_refill(q, lane);
           }
@@ -579,8 +596,7 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
         pr[0] = pr[1] = pr[2] = pr[3] = single_pair<FMT, PB>(hdr.single_sym);
       }
       // this warp's 256 weights of the round -> tile row hw
-      uint4 wv = make_uint4(0u, 0u, 0u, 0u);
-      if (act && !status) {
+      if (act && !status && !done) {
         wv.x = weights2<FMT, PB>(pr[0], sc, nan_codes);
         wv.y = weights2<FMT, PB>(pr[1], sc, nan_codes);
         wv.z = weights2<FMT, PB>(pr[2], sc, nan_codes);
@@ -629,8 +645,10 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32)
         }
         if constexpr (kAlias) half_sync();  // the sums are read before the tiles are rewritten
         ++row_local;
-        if (valid && !status && row_local < P.rows_per_chunk)
+        if (valid && !status && row_local < P.rows_per_chunk) {
           sc = bf16_bits_to_float(P.scales[row0 + row_local]);
+          e4 = e4_row(row0 + row_local);
+        }
       }
     }
     if (valid && !status) {

@@ -922,6 +922,36 @@ def profile_kernel(kind: str, launches: int = 5):
         out = torch.empty(t.rows, t.cols, dtype=torch.bfloat16, device=dev)
         st = eq.new_status(dev)
         fn = lambda: eq.decode([t], [out], st)  # noqa: E731
+    elif kind == "layer":
+        # one LLaMA-2-7B-shaped layer (q, k, v, o, gate, up, down; the headline stack's first
+        # layer, drawn from the seeded generators and coded on the GPU), decoded in one call: the
+        # headline's kernel in the headline's launch shape
+        import torch as _t
+        wl = synth.WORKLOADS["llama2_7b"]
+        ts = []
+        for spec in wl.tensors[:7]:
+            w = _t.from_numpy(spec.generate()).to(dev)
+            sym, sc = eq.quantize_device(w, eq.EQ_SYM_E4M3)
+            ts.append(eq.rans_encode_device(sym, sc, eq.EQ_SYM_E4M3, wl.chunk_symbols, wl.streams,
+                                            wl.run))
+            del w, sym
+        outs = [_t.empty(t.rows, t.cols, dtype=_t.bfloat16, device=dev) for t in ts]
+        st = eq.new_status(dev)
+        fn = lambda: eq.decode(ts, outs, st)  # noqa: E731
+    elif kind == "gateup":
+        # the 13B MLP block at batch 1: gate and up in the fused kernel (then the down product)
+        wl = synth.WORKLOADS["mlp_13b"]
+        mats = []
+        for spec in wl.tensors:
+            sym, sc = eq.codec.quantize(spec.generate(), eq.EQ_SYM_E4M3)
+            mats.append(eq.DeviceRans.upload(eq.codec.rans_encode(
+                sym, sc, eq.EQ_SYM_E4M3, wl.chunk_for(spec), wl.streams, wl.run), dev))
+        g, u, d = mats
+        x = torch.randn(1, g.cols, device=dev).to(torch.bfloat16)
+        y = torch.empty(1, d.rows, dtype=torch.float32, device=dev)
+        scratch = torch.empty(eq.mlp_scratch_bytes(g.rows, 1), dtype=torch.uint8, device=dev)
+        st = eq.new_status(dev)
+        fn = lambda: eq.mlp_decode(g, u, d, x, y, scratch, st)  # noqa: E731
     elif kind == "gemv7":
         # the ~2-bit Int8 weight, one row per chunk, 7-bit table, batch 1
         wl = synth.WORKLOADS["int8_8k"]
@@ -945,7 +975,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-kernel", default=None,
                     choices=["decode", "huff", "huffint", "gemv", "gemv4", "gemv16", "decode12",
-                             "gemv7"],
+                             "gemv7", "layer", "gateup"],
                     help="launch one kernel a few times and exit (for ncu)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)

@@ -165,27 +165,48 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
       : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+// try_wait / bounded wait on an mbarrier given by its shared address
+__device__ __forceinline__ bool mbar_try_wait_s(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
       " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
 }
 
 // Wait for phase `parity` of an mbarrier, giving up after ~1 s (or 2^26 polls).  Returns false on
 // timeout; the caller records EQ_DEV_TIMEOUT and stops using the buffer.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool mbar_wait_bounded_s(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait_s(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 0; i < (1u << 26); ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_s(bar, parity)) return true;
     if ((i & 255u) == 255u && global_timer_ns() - t0 > 1000000000ull) break;
   }
   return false;
+}
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+  return mbar_wait_bounded_s(smem_addr(bar), parity);
+}
+
+// One 1-D bulk copy of `bytes` bytes (a multiple of 16) from global `src` to shared address
+// `dst`, completing on the mbarrier at shared address `bar`, issued by the lanes with `issuer`
+// set (one lane): the proxy fence that orders the warp's earlier reads of the destination before
+// the copy engine's writes, the arrival with the expected byte count, the copy.  Predicated
+// rather than branched, so the warp does not diverge around it.
+__device__ __forceinline__ void bulk_g2s_issue(bool issuer, uint32_t dst, const void *src,
+                                               uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %0, 0;\n"
+      " @p fence.proxy.async.shared::cta;\n"
+      " @p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%4], %3;\n"
+      " @p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%1], [%2], %3, [%4];\n"
+      "}\n" ::"r"(uint32_t(issuer)),
+      "r"(dst), "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void report(uint32_t *d_status, uint32_t bits) {

@@ -20,17 +20,18 @@ constexpr uint32_t kRingBytesWide = kSegBytesWide * kNumSeg;
 // ------------------------------------------------------------------------------------------------
 // Per-warp word ring.  Byte offsets are counted from A, the 16-byte-aligned start of the
 // substream's span; segment s (bytes [s * SEG, s * SEG + SEG) of the span) lands in ring slot
-// s % 4, i.e. at ring byte (offset mod 4 * SEG).  Copies are issued by lane 0; every lane waits.
-// A slot is refilled only after the wait for its previous copy, so each of the four mbarriers has
-// at most one copy in flight.
+// s % 4, i.e. at ring byte (offset mod 4 * SEG).  Copies are issued by lane 0 (predicated, the
+// warp does not branch); every lane waits.  A slot is refilled only after the wait for its
+// previous copy, so each of the four mbarriers has at most one copy in flight.  The ring and its
+// barriers are held by their shared addresses.
 // ------------------------------------------------------------------------------------------------
 template <uint32_t SEG>
 struct WordRingT {
   static constexpr uint32_t kSeg = SEG;
   static constexpr uint32_t kBytes = SEG * kNumSeg;
-  unsigned char *buf;
-  uint32_t ring_off;  // buf - shared-memory base (a multiple of kBytes)
-  uint64_t *bar;
+  uint32_t buf_s;     // shared address of the ring (a multiple of kBytes)
+  uint32_t ring_off;  // the ring's offset from the shared-memory base (a multiple of kBytes)
+  uint32_t bar_s;     // shared address of the ring's first mbarrier (four, 8 bytes apart)
   const unsigned char *A;
   uint32_t off0;    // bytes from A to the first word
   uint32_t span;    // bytes to copy (multiple of 16)
@@ -42,13 +43,20 @@ struct WordRingT {
   uint32_t phase;      // bit s: the phase the next wait on slot s's barrier waits for (it
                        // carries over from one substream to the next a warp decodes)
 
+  // hand segment `issued` to the copy engine (its slot's previous copy has been waited for):
+  // predicated (the batch edges, where it keeps the warp from branching) or in a branch of lane 0
+  // (the per-round checks, where the branch keeps the copy's operands out of the loop)
+  __device__ __forceinline__ void issue_next(uint32_t lane) {
+    const uint32_t s = issued, slot = s % kNumSeg;
+    bulk_g2s_issue(lane == 0, buf_s + slot * SEG, A + size_t(s) * SEG, min(SEG, span - s * SEG),
+                   bar_s + slot * 8u);
+    ++issued;
+  }
   __device__ __forceinline__ void issue(uint32_t lane) {
     if (lane == 0) {
       const uint32_t s = issued, slot = s % kNumSeg;
-      const uint32_t bytes = min(SEG, span - s * SEG);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_expect_tx(&bar[slot], bytes);
-      bulk_g2s(buf + slot * SEG, A + size_t(s) * SEG, bytes, &bar[slot]);
+      bulk_g2s_issue(true, buf_s + slot * SEG, A + size_t(s) * SEG, min(SEG, span - s * SEG),
+                     bar_s + slot * 8u);
     }
     ++issued;
     refill_at = issued < nseg ? (issued - kNumSeg + 1) * SEG : 0xFFFFFFFFu;
@@ -71,7 +79,7 @@ struct WordRingT {
 
   // the copy into `slot` has landed (bounded wait); false on timeout
   __device__ __forceinline__ bool wait_slot(uint32_t slot) {
-    if (!mbar_wait_bounded(&bar[slot], (phase >> slot) & 1u)) return false;
+    if (!mbar_wait_bounded_s(bar_s + slot * 8u, (phase >> slot) & 1u)) return false;
     phase ^= 1u << slot;
     return true;
   }
@@ -95,46 +103,53 @@ struct WordRingT {
     constexpr uint32_t kAhead = 2 * kRoundWords + 2;
     return (q + kAhead <= ready_end || ready >= nseg) ? true : wait_below(q + kAhead);
   }
-  // round_wait, and when it has to wait, for every segment handed out up to the one two past
-  // q's (those copies went out a segment or more ago), so that the next ring work is the next
-  // refill rather than another wait
-  __device__ __forceinline__ bool round_wait_far(uint32_t q) {
-    constexpr uint32_t kAhead = 2 * kRoundWords + 2;
-    if (q + kAhead <= ready_end || ready >= nseg) return true;
-    const uint32_t far = min(issued, q / SEG + 3) * SEG;
-    return wait_below(max(q + kAhead, far));
+  // The batch protocol of the 12-bit decode's full rounds.  Once q (the warp's next word) has
+  // entered segment cur, segments up to cur + 2 have landed and cur + 3 is in flight (or the
+  // substream has no more), so every byte below safe_end = (cur + 3) * SEG can be read.  A round
+  // of run G reads below q + 64 G + 2 and moves q by at most 64 G bytes, so the rounds of a batch
+  // need no check: as many as keep their reads below safe_end, at least four with G = 8 and
+  // SEG = 1024.  After a batch, each segment start q has passed (edge_next) is one edge: the slot
+  // of the segment before it is used up and takes segment cur + 3, and segment cur + 2 (handed
+  // out one segment earlier) is waited for.  batch_begin() sets this up from any state;
+  // batch_end() restores the fields the per-round checks use.
+  uint32_t edge_next;  // offset of the next segment start
+  uint32_t safe_end;   // bytes below this offset have landed (0xFFFFFFFF: the whole substream)
+  __device__ __forceinline__ void set_safe_end() {
+    safe_end = ready >= nseg ? 0xFFFFFFFFu : ready * SEG;
   }
-  // The ring work of the 12-bit decode's full rounds, done once per segment: when q (the warp's
-  // next word) has entered segment cur, segment cur - 1 is used up and its copy was waited for,
-  // so its slot takes segment cur + 3; then segment cur + 1 (handed out a segment ago) is waited
-  // for.  A round reads at most 514 bytes from q and SEG > 514, so the landed segments <= cur + 1
-  // cover it.  edge_begin() sets this up from any state; edge_end() restores the fields the
-  // general checks use.  edge_next: offset of the next segment start.
-  uint32_t edge_next;
-  __device__ __forceinline__ bool edge_begin(uint32_t q, uint32_t lane) {
+  __device__ __forceinline__ bool batch_begin(uint32_t q, uint32_t lane) {
     const uint32_t cur = q / SEG;
     while (issued < nseg && issued <= cur + 3) issue(lane);
-    while (ready < nseg && ready <= cur + 1) {
+    while (ready < nseg && ready <= cur + 2) {
       if (!wait_slot(ready % kNumSeg)) return false;
       ++ready;
     }
     edge_next = (cur + 1) * SEG;
+    set_safe_end();
     return true;
   }
-  __device__ __forceinline__ bool edge(uint32_t lane) {
-    const uint32_t cur = edge_next / SEG;
-    if (issued < nseg && issued <= cur + 3) {
+  // rounds of run G that can start at q without a check (at least 1 after batch_begin or the
+  // edges of the last batch)
+  template <int G>
+  __device__ __forceinline__ uint32_t batch_rounds(uint32_t q) const {
+    constexpr uint32_t kRound = 64u * G;
+    return (safe_end - q - (kRound + 2u)) / kRound + 1u;
+  }
+  // one segment start passed: issued == cur + 3 and ready == cur + 2 whenever below nseg
+  __device__ __forceinline__ bool batch_edge(uint32_t lane) {
+    if (issued < nseg) {
       __syncwarp();
-      issue(lane);
+      issue_next(lane);
     }
-    if (ready < nseg && ready <= cur + 1) {
+    if (ready < nseg) {
       if (!wait_slot(ready % kNumSeg)) return false;
       ++ready;
     }
     edge_next += SEG;
+    set_safe_end();
     return true;
   }
-  __device__ __forceinline__ void edge_end() {
+  __device__ __forceinline__ void batch_end() {
     ready_end = ready * SEG;
     refill_at = issued < nseg ? (issued - kNumSeg + 1) * SEG : 0xFFFFFFFFu;
   }
@@ -169,10 +184,6 @@ struct WordRingT {
       ++ready;
     }
     return 0;
-  }
-
-  __device__ __forceinline__ uint32_t word_at(uint32_t q) const {
-    return *reinterpret_cast<const uint16_t *>(buf + (q & (kBytes - 1)));
   }
 };
 using WordRing = WordRingT<kSegBytes>;
@@ -439,12 +450,12 @@ __device__ __forceinline__ uint32_t sym_pair(uint32_t e0, uint32_t e1) {
 template <class Ring>
 __device__ __forceinline__ void ring_init(Ring &R, unsigned char *smem, unsigned char *rings,
                                           uint64_t *bars, uint32_t warp, uint32_t lane) {
-  R.buf = rings + warp * Ring::kBytes;
-  R.ring_off = uint32_t(R.buf - smem);
-  R.bar = bars + warp * kNumSeg;
+  R.buf_s = smem_addr(rings) + warp * Ring::kBytes;
+  R.ring_off = uint32_t(rings - smem) + warp * Ring::kBytes;
+  R.bar_s = smem_addr(bars) + warp * kNumSeg * 8u;
   R.phase = 0;
   if (lane == 0) {
-    for (uint32_t s = 0; s < kNumSeg; ++s) mbar_init(&R.bar[s], 1);
+    for (uint32_t s = 0; s < kNumSeg; ++s) mbar_init(&bars[warp * kNumSeg + s], 1);
     fence_mbar_init();
   }
 }

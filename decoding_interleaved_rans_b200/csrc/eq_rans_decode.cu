@@ -88,12 +88,9 @@ __device__ __forceinline__ void decode_round(const RansDesc &D, uint32_t &x, boo
     }
   } else if constexpr (PB == 12) {  // entries [symbol | f | slot - cum]
     // tb, ring: shared addresses of the table (the start of the shared memory) and of this
-    // warp's ring, converted once per unit by the caller
-    if constexpr (FULL && !MAYBE_NAN && G == 8 && FMT == EQ_SYM_E4M3) {
-      // E4M3, no NaN codes, |scale| < 2^8 (the caller checked the unit's rows)
-      *reinterpret_cast<uint4 *>(out) =
-          rans_round12_e4m3<Ring::kBytes>(x, q, tb, ring, lt, scale_e4m3_offset(sc));
-    } else if constexpr (G == 8) {
+    // warp's ring, converted once per unit by the caller.  (The caller runs the E4M3 round block
+    // itself where it applies.)
+    if constexpr (G == 8) {
       uint32_t e[8];
 #pragma unroll
       for (int p = 0; p < 8; ++p) {
@@ -179,7 +176,7 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
   R.start(D.words, w0, nwords, lane);
   const bool nan_codes = (FMT == EQ_SYM_E4M3) && (flags & (kRansFlagNaN7F | kRansFlagNaNFF));
   const uint32_t lt = lanemask_lt_once();
-  const uint32_t tb = smem_addr(smem), ring = smem_addr(R.buf);
+  const uint32_t tb = smem_addr(smem), ring = R.buf_s;
   // rounds in which all 32 lanes of this group hold a run
   const uint32_t full = runs >= 32 * g + 32 ? (runs - 32 * g - 32) / S + 1 : 0;
   uint32_t q = R.off0;
@@ -216,32 +213,20 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
       if (row < D.rows) sc = bf16_bits_to_float(D.scales[row]);
     }
   };
-  // The rounds in which every lane of the group holds a run, with no per-round tests.  The ring
-  // work (overrun check, refill, wait) runs only once q reaches q_next; refill comes before the
-  // wait, so every segment a wait needs has been handed to the copy engine.  Instantiated for
-  // tables with and without NaN codes and for one or several row ends per round, so that none
-  // of those tests is left in the loop.
-  // The ring work before a full round.  12-bit tables: once per segment (edge); otherwise the
-  // general checks, run only once q reaches q_next.  q is the same in every lane; the vote tells
-  // the compiler so (no reconvergence point).
+  // 8- and 7-bit tables: the rounds in which every lane of the group holds a run, the ring work
+  // (overrun check, refill, wait) every second round and only once q reaches q_next; refill comes
+  // before the wait, so every segment a wait needs has been handed to the copy engine.
+  // Instantiated for tables with and without NaN codes and for one or several row ends per
+  // round, so that none of those tests is left in the loop.
   uint32_t q_next = 0;
-  auto ring_work = [&]() -> uint32_t {
-    if constexpr (PB == 12) {
-      if (__any_sync(0xFFFFFFFFu, q >= R.edge_next)) {
-        if (q > q_end) return EQ_DEV_OVERRUN;
-        if (!R.edge(lane)) return EQ_DEV_TIMEOUT;
-      }
-    } else if (q >= q_next) {
-      if (q > q_end) return EQ_DEV_OVERRUN;
-      R.round_refill(q, lane);
-      if (!R.round_wait(q)) return EQ_DEV_TIMEOUT;
-      q_next = R.quiet_until(q_end);
-    }
-    return 0u;
-  };
   auto run_full = [&](auto maybe_nan, auto one_wrap) -> uint32_t {
     for (; r0 + kRoundsPerCheck <= full; r0 += kRoundsPerCheck) {
-      if (const uint32_t st = ring_work()) return st;
+      if (q >= q_next) {
+        if (q > q_end) return EQ_DEV_OVERRUN;
+        R.round_refill(q, lane);
+        if (!R.round_wait(q)) return EQ_DEV_TIMEOUT;
+        q_next = R.quiet_until(q_end);
+      }
 #pragma unroll
       for (uint32_t k = 0; k < kRoundsPerCheck; ++k) {
         decode_round<true, G, FMT, PB, decltype(maybe_nan)::value>(D, x, true, lut, smem, R, q,
@@ -251,44 +236,106 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
     }
     return 0u;
   };
-  // Rounds that never straddle a row (cols and the chunk length multiples of S * G): row and
-  // scale are the same in every lane and change every cols / step rounds, so a loop over rows
-  // and, inside it, over the row's rounds, with nothing tracked per round but the output
-  // position.  Afterwards each lane's row, column and scale are recomputed for the general loop.
-  auto run_rows = [&](auto maybe_nan) -> uint32_t {
-    const uint32_t per_row = cols / step;
-    uint32_t row_u = uint32_t(div_by_magic(j0, D.row_magic));
-    uint32_t left = per_row - uint32_t(j0 - uint64_t(row_u) * cols) / step;
-    uint32_t st = 0;
-    while (r0 < full && !st) {
-      const uint32_t nr = min(left, full - r0);
-      const float sc_u = bf16_bits_to_float(D.scales[row_u]);
-      for (uint32_t k = 0; k < nr; ++k) {
-        if ((st = ring_work())) break;
-        decode_round<true, G, FMT, PB, decltype(maybe_nan)::value>(D, x, true, lut, smem, R, q,
-                                                                   lt, out, sc_u, true, tb, ring);
-        out += step;
-        ++r0;
-      }
-      left -= nr;
-      if (left == 0) {
-        left = per_row;
-        ++row_u;
-      }
+  // 12-bit tables: the full rounds in batches (the ring's batch protocol), each batch a loop with
+  // nothing in it but the round, its store and the row tracking; the edges after it.  FAST: the
+  // E4M3 round block (Float8-E4M3 symbols, no NaN code in the table, every row scale of the unit
+  // below 2^8 in magnitude), with the row scale as its factor scale * 2^120.  MODE 0: rounds
+  // never straddle a row (cols and the chunk length multiples of S * G), so the row and its
+  // scale are the warp's and change every cols / step rounds (with the E4M3 block the unit's
+  // row factors are held one row per lane, 32 rows at a time, and a row change is a shuffle),
+  // and each lane's row, column and scale are recomputed afterwards for the general loop;
+  // MODE 1: a round crosses at most one row end (a compare and a conditional update); MODE 2:
+  // rows shorter than a round.
+  auto run_batches = [&](auto fast, auto maybe_nan, auto mode) -> uint32_t {
+    constexpr bool FAST = decltype(fast)::value;
+    constexpr int MODE = decltype(mode)::value;
+    uint32_t per_row = 0, left = 0;
+    if constexpr (MODE == 0) {
+      per_row = cols / step;
+      row = uint32_t(div_by_magic(j0, D.row_magic));
+      left = per_row - uint32_t(j0 - uint64_t(row) * cols) / step;
+      sc = bf16_bits_to_float(D.scales[row]);
     }
-    const uint64_t j = j0 + (uint64_t(r0) * S + s) * G;
-    row = uint32_t(div_by_magic(j, D.row_magic));
-    col = uint32_t(j - uint64_t(row) * cols);
-    sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+    uint32_t sc2e = FAST ? scale_e4m3_offset(sc) : 0u;
+    uint32_t tab_base = row, tab = 0;  // MODE 0 with FAST: row tab_base + lane's factor
+    auto load_tab = [&]() {
+      const uint32_t r = tab_base + lane;
+      tab = scale_e4m3_offset(bf16_bits_to_float(D.scales[r < D.rows ? r : 0]));
+    };
+    if constexpr (MODE == 0 && FAST) load_tab();
+    uint32_t st = 0;
+    while (r0 < full) {
+      uint32_t nb = min(R.template batch_rounds<G>(q), full - r0);
+      r0 += nb;
+      auto one_round = [&]() {
+        if constexpr (FAST)
+          *reinterpret_cast<uint4 *>(out) = rans_round12_e4m3<Ring::kBytes>(x, q, tb, ring, lt, sc2e);
+        else
+          decode_round<true, G, FMT, PB, decltype(maybe_nan)::value>(D, x, true, lut, smem, R, q,
+                                                                     lt, out, sc, true, tb, ring);
+        out += step;
+      };
+      if constexpr (MODE == 0) {
+        do {
+          one_round();
+          if (--left == 0) {
+            left = per_row;
+            ++row;
+            if constexpr (FAST) {
+              if (row - tab_base == 32) {
+                tab_base = row;
+                load_tab();
+              }
+              sc2e = __shfl_sync(0xFFFFFFFFu, tab, row - tab_base);
+            } else {
+              sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+            }
+          }
+        } while (--nb);
+      } else {
+        do {
+          one_round();
+          col += step;
+          if (col >= cols) {
+            do {
+              col -= cols;
+              ++row;
+            } while (MODE == 2 && col >= cols);
+            sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+            if constexpr (FAST) sc2e = scale_e4m3_offset(sc);
+          }
+        } while (--nb);
+      }
+      while (q >= R.edge_next) {
+        if (q > q_end) {
+          st = EQ_DEV_OVERRUN;
+          break;
+        }
+        if (!R.batch_edge(lane)) {
+          st = EQ_DEV_TIMEOUT;
+          break;
+        }
+      }
+      if (st) break;
+    }
+    if constexpr (MODE == 0) {
+      const uint64_t j = j0 + (uint64_t(r0) * S + s) * G;
+      row = uint32_t(div_by_magic(j, D.row_magic));
+      col = uint32_t(j - uint64_t(row) * cols);
+      sc = bf16_bits_to_float(D.scales[row < D.rows ? row : 0]);
+    }
     return st;
   };
   using T = std::true_type;
   using F = std::false_type;
+  using M0 = std::integral_constant<int, 0>;
+  using M1 = std::integral_constant<int, 1>;
+  using M2 = std::integral_constant<int, 2>;
   // The full rounds go without NaN checks when the table has no NaN code; for 12-bit tables that
   // also selects the E4M3 round block, which needs Float8-E4M3 symbols and every row scale of the
   // unit below 2^8 in magnitude (checked here, one scale per lane).
   if constexpr (PB == 12)
-    if (!R.edge_begin(q, lane)) status = EQ_DEV_TIMEOUT;
+    if (!R.batch_begin(q, lane)) status = EQ_DEV_TIMEOUT;
   bool plain = !nan_codes;
   if constexpr (PB == 12) {
     if (FMT != EQ_SYM_E4M3) plain = false;
@@ -298,13 +345,22 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
     for (uint32_t r = r_first + lane; r <= r_last; r += 32) ok &= (D.scales[r] & 0x7FFFu) < 0x4380u;
     plain = __all_sync(0xFFFFFFFFu, ok) && plain;
   }
-  // (12-bit tables; the 8- and 7-bit ones check the ring every second round in run_full)
-  const bool row_rounds = PB == 12 && G == 8 && cols % step == 0 && D.chunk_symbols % step == 0;
-  if (status) {
-  } else if (row_rounds) status = plain ? run_rows(F{}) : run_rows(T{});
-  else if (!plain) status = step <= cols ? run_full(T{}, T{}) : run_full(T{}, F{});
-  else status = step <= cols ? run_full(F{}, T{}) : run_full(F{}, F{});
-  if constexpr (PB == 12) R.edge_end();
+  if constexpr (PB == 12) {
+    const bool row_rounds = G == 8 && cols % step == 0 && D.chunk_symbols % step == 0;
+    auto dispatch = [&](auto fast, auto maybe_nan) -> uint32_t {
+      if constexpr (G == 8)
+        if (row_rounds) return run_batches(fast, maybe_nan, M0{});
+      return step <= cols ? run_batches(fast, maybe_nan, M1{}) : run_batches(fast, maybe_nan, M2{});
+    };
+    if (!status) {
+      if constexpr (G == 8 && FMT == EQ_SYM_E4M3) status = plain ? dispatch(T{}, F{}) : dispatch(F{}, T{});
+      else status = dispatch(F{}, T{});
+    }
+    R.batch_end();
+  } else if (!status) {
+    if (!plain) status = step <= cols ? run_full(T{}, T{}) : run_full(T{}, F{});
+    else status = step <= cols ? run_full(F{}, T{}) : run_full(F{}, F{});
+  }
   if (!status) {  // the general loop below waits first: hand out the used-up slots
     if (q > q_end) status |= EQ_DEV_OVERRUN;
     else R.round_refill(q, lane);
@@ -338,9 +394,16 @@ __device__ __forceinline__ uint32_t decode_group(const RansDesc &D, const uint32
 }
 
 // 7-bit tables: one CTA of up to 32 warps per SM shares the 128 KiB pair table, each warp
-// decoding unit after unit; otherwise up to 16 warps per CTA, one unit each.
+// decoding unit after unit; otherwise CTAs of 12 warps (12-bit tables, three per SM) or 16 warps
+// (8-bit tables, two per SM), one unit each.  The launch bounds give the register allocator the
+// budget of that occupancy.
+constexpr uint32_t decode_max_threads(uint32_t pb) {
+  return pb == kRansPairBits ? 1024 : pb == 12 ? 384 : 512;
+}
+constexpr uint32_t decode_min_ctas(uint32_t pb) { return pb == kRansPairBits ? 1 : pb == 12 ? 3 : 2; }
+
 template <int G, int FMT, uint32_t PB>
-__global__ void __launch_bounds__(PB == kRansPairBits ? 1024 : 512)
+__global__ void __launch_bounds__(decode_max_threads(PB), decode_min_ctas(PB))
     rans_decode_kernel(const __grid_constant__ RansDecodeParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   using Ring = WordRingT<PB == 12 ? kSegBytesWide : kSegBytes>;

@@ -185,7 +185,7 @@ __device__ __forceinline__ uint32_t gemv_chunk(const GemvParams &P, uint64_t chu
   // 12-bit tables of E4M3 symbols without NaN codes: rounds in which every lane holds a run go
   // through the decode kernel's E4M3 round block (the weights come out dequantised), while the
   // row's scale is below 2^8 in magnitude
-  const uint32_t tb = smem_addr(lut), ring_abs = smem_addr(R.buf);
+  const uint32_t tb = smem_addr(lut), ring_abs = R.buf_s;
   auto e4_row = [&](uint32_t row) {
     return PB == 12 && FMT == EQ_SYM_E4M3 && !nan_codes && !single &&
            (P.scales[row] & 0x7FFFu) < 0x4380u;
@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(HALVES * kTcWarps * 32, HALVES == 1 ? 2 : 1)
   const uint32_t rpr = P.rows_per_chunk > 1 ? P.rounds_per_row : rounds;
   const uint32_t ntiles = (P.batch + 7) / 8;
   const uint32_t tiles_addr = smem_addr(tiles);
-  const uint32_t tb = smem_addr(lut), ring_abs = smem_addr(R.buf);
+  const uint32_t tb = smem_addr(lut), ring_abs = R.buf_s;
   const uint64_t ngroups = (P.num_chunks + kTcWarps - 1) / kTcWarps;
   // sticky: a warp whose chunk failed feeds zeros from then on (the launch reports the failure)
   uint32_t status = 0;

@@ -67,3 +67,76 @@ def test_table_of_the_other_format_is_reported(eq, orc, pb):
         _, status = eq.decode_gemv(t, x)
         torch.cuda.synchronize()
         assert int(status.item()) & eq.EQ_DEV_CORRUPT_STATE
+
+
+def finite_e4m3_codes() -> np.ndarray:
+    c = np.arange(256, dtype=np.uint16)
+    return c[(c & 0x7F) != 0x7F]  # 254 codes: all but the two NaN patterns
+
+
+@pytest.mark.parametrize("case", ["e4m3_finite_rows", "e4m3_finite_ragged", "e4m3_with_nan",
+                                  "int8"])
+def test_12bit_every_code_times_every_finite_scale(eq, orc, case):
+    """12-bit tables carry no values: E4M3 tables without NaN codes take the exponent-offset
+    dequantisation (the code's bits placed in a bf16 scaled by 2^-120, times scale * 2^120),
+    which the decoder chooses per unit of rows only while every row scale is below 2^8 in
+    magnitude; other units, tables holding a NaN code and Int8 take the per-symbol product.
+    Rows are sorted by scale bit pattern, so units of small scales, units of large scales and
+    units holding both all occur, and every (code, finite scale) pair is compared with the
+    oracle's one-rounding product.  The 256-column cases take the whole-row loop, the 264-column
+    one (chunks cutting rows) the general loop."""
+    sc = finite_bf16_scales()
+    rows = sc.size
+    fmt = orc.INT8 if case == "int8" else orc.E4M3
+    if case == "e4m3_finite_ragged":  # 264 columns: a multiple of the run, not of a round
+        codes = np.concatenate([finite_e4m3_codes(), finite_e4m3_codes()[:10]])
+    elif case == "e4m3_finite_rows":
+        codes = np.concatenate([finite_e4m3_codes(), np.array([0x00, 0x80], np.uint16)])
+    else:
+        codes = np.arange(256, dtype=np.uint16)
+    k = codes.size
+    sym = codes[(np.arange(k)[None, :] + np.arange(rows)[:, None]) % k].astype(np.uint8)
+    h = orc.rans_encode(sym, sc, fmt, 16384, 32, 8, prob_bits=12)
+    t = eq.DeviceRans.upload(h)
+    (out,), st = eq.decode([t])
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    got = eq.bf16_bits(out)
+    want = orc.dequant(sym, sc, fmt)
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, [(int(sym[r, c]), hex(int(sc[r])), hex(int(got[r, c])), hex(int(want[r, c])))
+                           for r, c in bad[:8]]
+
+
+@pytest.mark.parametrize("chunk_rows", [1, 4])
+def test_12bit_e4m3_gemv_one_hot_every_code_times_every_finite_scale(eq, orc, chunk_rows):
+    """The fused GEMV's exponent-offset path (12-bit E4M3 tables without NaN codes, per row while
+    the scale is below 2^8 in magnitude) against the oracle's dequantisation: with one-hot
+    activations each output is one decoded weight (every other product is an exact zero and one
+    is the weight times one), so over all columns every (code, finite scale) pair is compared
+    exactly, at batch 1 (one row per chunk: the one-row loop), 4 and 16 (tensor-core kernel).
+    Rows whose products overflow to infinity turn into NaN through infinity times zero; the
+    oracle's dequantisation of those rows holds an infinity, and the kernel's outputs there are NaN."""
+    sc = finite_bf16_scales()
+    rows = sc.size
+    codes = np.concatenate([finite_e4m3_codes(), np.array([0x00, 0x80], np.uint16)])
+    cols = codes.size
+    sym = codes[(np.arange(cols)[None, :] + np.arange(rows)[:, None]) % cols].astype(np.uint8)
+    h = orc.rans_encode(sym, sc, orc.E4M3, cols * chunk_rows, 32, 8, prob_bits=12)
+    t = eq.DeviceRans.upload(h)
+    want = orc.dequant(sym, sc, orc.E4M3).astype(np.uint32) << 16
+    wantf = want.view(np.float32)
+    finite = np.isfinite(wantf).all(axis=1)
+    assert 0 < finite.sum() < rows
+    for batch in (1, 4, 16):
+        for j0 in range(0, cols, batch):
+            x = torch.zeros(batch, cols, dtype=torch.bfloat16, device="cuda")
+            x[torch.arange(batch), j0 + torch.arange(batch)] = 1.0
+            y, st = eq.decode_gemv(t, x)
+            torch.cuda.synchronize()
+            assert int(st.item()) == 0
+            y = y.cpu().numpy()
+            ref = wantf[:, j0:j0 + batch].T
+            ok = np.equal(y[:, finite], ref[:, finite])
+            assert ok.all(), (batch, j0, np.argwhere(~ok)[:4])
+            assert np.isnan(y[:, ~finite]).all(), (batch, j0)

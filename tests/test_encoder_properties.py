@@ -77,3 +77,25 @@ def test_host_df11_encoder_matches_oracle(eq, orc, rows, cols, tpb, kind, seed):
     assert a.total_bits == b.total_bits
     for f in ("enc_exp", "sign_mant", "gaps", "block_out"):
         assert np.array_equal(getattr(a, f), getattr(b, f)), f
+
+
+@settings(max_examples=30, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(rows=st.integers(1, 30), cols=st.integers(1, 500), bits=st.sampled_from([8, 4]),
+       tpb=st.sampled_from([1, 32, 256]), spread=st.floats(1e-6, 10.0), shift=st.floats(-1.0, 1.0),
+       seed=st.integers(0, 2**31 - 1))
+def test_host_integer_code_encoder_matches_oracle(eq, orc, rows, cols, bits, tpb, spread, shift,
+                                                  seed):
+    """EntroLLM-style integer codes: the per-tensor quantiser and the byte-stream Huffman coder."""
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((rows, cols)) * spread + shift * spread).astype(np.float32)
+    for scheme in (0, 1):
+        a = eq.codec.intq_quantize(w, bits, scheme)
+        b = orc.intq_quantize(w, bits, scheme)
+        assert np.array_equal(a[0], b[0]) and a[1:] == b[1:]
+    h = eq.codec.entrollm_encode(w, bits, threads_per_block=tpb)
+    sym, sc, z, _ = orc.entrollm_quantize(w, bits)
+    o = orc.huff_encode_sym(sym, bits, sc, z, threads_per_block=tpb)
+    assert (h.scale, h.zero, h.total_bits) == (o.scale, o.zero, o.total_bits)
+    assert np.array_equal(h.lengths, o.lengths)
+    for f in ("enc", "gaps", "block_out"):
+        assert np.array_equal(getattr(h, f), getattr(o, f)), f

@@ -58,10 +58,16 @@ RECORD_SOURCES = {
 
 
 def kernel_sources_sha(key: str) -> str:
+    """sha256 of the kernel's sources with comments removed and whitespace collapsed, so that an
+    edit of a comment keeps a capture valid and any change of code does not."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in RECORD_SOURCES[key]:
-        h.update(open(os.path.join(ROOT, "decoding_interleaved_rans_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "decoding_interleaved_rans_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()
 
 

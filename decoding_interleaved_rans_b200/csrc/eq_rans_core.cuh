@@ -20,10 +20,9 @@ constexpr uint32_t kRingBytesWide = kSegBytesWide * kNumSeg;
 // ------------------------------------------------------------------------------------------------
 // Per-warp word ring.  Byte offsets are counted from A, the 16-byte-aligned start of the
 // substream's span; segment s (bytes [s * SEG, s * SEG + SEG) of the span) lands in ring slot
-// s % 4, i.e. at ring byte (offset mod 4 * SEG).  Copies are issued by lane 0 (predicated, the
-// warp does not branch); every lane waits.  A slot is refilled only after the wait for its
-// previous copy, so each of the four mbarriers has at most one copy in flight.  The ring and its
-// barriers are held by their shared addresses.
+// s % 4, i.e. at ring byte (offset mod 4 * SEG).  Copies are issued by lane 0; every lane waits.
+// A slot is refilled only after the wait for its previous copy, so each of the four mbarriers has
+// at most one copy in flight.  The ring and its barriers are held by their shared addresses.
 // ------------------------------------------------------------------------------------------------
 template <uint32_t SEG>
 struct WordRingT {
